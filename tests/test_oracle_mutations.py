@@ -1,0 +1,126 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check that a pin catches each one.
+
+Every mutation is applied with monkeypatch to ``oracle.sla_oracle`` and undone
+after the test; the pins themselves are the functions of test_oracle_pins.
+"""
+
+import glob
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle.sla_oracle as so
+from tests import test_oracle_pins as pins
+
+GOLDEN = sorted(glob.glob(os.path.join(os.path.dirname(__file__), "golden", "hand_example_*.json")))
+
+
+def _patch(monkeypatch, name, fn):
+    """Replace ``name`` both in the implementation module and in the package namespace."""
+    import oracle
+
+    monkeypatch.setattr(so, name, fn)
+    if hasattr(oracle, name):
+        monkeypatch.setattr(oracle, name, fn)
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except AssertionError:
+        return True
+    return False
+
+
+def _golden_any_fails():
+    return any(_fails(pins.test_golden_hand_examples, p) for p in GOLDEN)
+
+
+def test_mutation_phi_without_plus_one(monkeypatch):
+    _patch(monkeypatch, "phi", lambda x: np.where(np.asarray(x) > 0, x, np.expm1(np.minimum(x, 0))) + 1e-3)
+    assert _golden_any_fails()
+
+
+def test_mutation_missing_score_scale(monkeypatch):
+    orig = so.sparse_branch
+
+    def unscaled(q_blk, k, v, crit, bk):
+        return orig(q_blk * math.sqrt(k.shape[1]), k, v, crit, bk)
+
+    _patch(monkeypatch, "sparse_branch", unscaled)
+    assert _golden_any_fails()
+
+
+def test_mutation_tie_break_reversed(monkeypatch):
+    orig = so.route_from_scores
+
+    def reversed_ties(S, kc, kn):
+        return orig(S[..., ::-1], kc, kn)[..., ::-1]
+
+    _patch(monkeypatch, "route_from_scores", reversed_ties)
+    assert _fails(pins.test_route_exact_ties_prefer_lower_index)
+
+
+def test_mutation_critical_count_rounded_down(monkeypatch):
+    orig = so.block_counts
+
+    def floor_counts(N, bq, bk, kh, kl):
+        Nq, Nk, kc, kn = orig(N, bq, bk, kh, kl)
+        return Nq, Nk, (int(round(kh * 1e6)) * Nk) // 1_000_000, kn
+
+    _patch(monkeypatch, "block_counts", floor_counts)
+    assert _fails(pins.test_block_counts, (32760, 128, 64, 0.05, 0.10), (256, 512, 26, 51))
+
+
+def test_mutation_alpha_on_wrong_branch(monkeypatch):
+    orig = so.forward
+
+    def swapped(q, k, v, alpha, *a, **kw):
+        return orig(q, k, v, 1.0 - so.as_f64(alpha), *a, **kw)
+
+    _patch(monkeypatch, "forward", swapped)
+    assert _golden_any_fails()
+
+
+def test_mutation_transposed_state(monkeypatch):
+    orig = so.kv_states
+
+    def transposed(k, v, bk):
+        h, z = orig(k, v, bk)
+        return np.swapaxes(h, -1, -2), z
+
+    _patch(monkeypatch, "kv_states", transposed)
+    assert _fails(pins.test_forward_matches_token_level_bruteforce, 0, 24, 8, 4)
+
+
+def test_mutation_negligible_counted_as_marginal(monkeypatch):
+    def wrong_sums(rows, h, z):
+        w = (rows != so.CRITICAL).astype(np.float64)
+        Nk, D = z.shape
+        return (w @ h.reshape(Nk, D * D)).reshape(-1, D, D), w @ z
+
+    _patch(monkeypatch, "marginal_sums", wrong_sums)
+    assert _golden_any_fails()
+
+
+def test_mutation_pool_sum_instead_of_mean(monkeypatch):
+    def pool_sum(x, block):
+        N = x.shape[-2]
+        return np.stack([x[..., s:min(N, s + block), :].sum(axis=-2) for s in range(0, N, block)], axis=-2)
+
+    _patch(monkeypatch, "pool_mean", pool_sum)
+    assert _fails(pins.test_pool_mean_tail_closed_form)
+
+
+def test_mutation_softmax_over_all_keys(monkeypatch):
+    # Not re-normalising over the critical set: the softmax runs over every key.
+    orig = so.sparse_branch
+
+    def all_keys(q_blk, k, v, crit, bk):
+        every = list(range(-(-k.shape[0] // bk)))
+        return orig(q_blk, k, v, every if len(crit) else crit, bk)
+
+    _patch(monkeypatch, "sparse_branch", all_keys)
+    assert _golden_any_fails()
