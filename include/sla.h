@@ -1,0 +1,125 @@
+/*
+ * sla.h - C ABI of the B200 (sm_100a) sparse-plus-linear block attention forward.
+ *
+ * The method: "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
+ * Sparse-Linear Attention" (Abstract) splits attention weights into critical
+ * (exact softmax attention), marginal (linear attention) and negligible
+ * (skipped) parts at block granularity; "SLA2: Sparse-Linear Attention with
+ * Learnable Routing and QAT" (§2.A) blends the two branch outputs as
+ *     O = alpha * O_s + (1 - alpha) * O_l,
+ * with a router (§2.B) that pools adjacent Q and K tokens and keeps a hard
+ * top-k at inference.
+ *
+ * What this library computes, per batch b, head h and query block i
+ * (block_q query tokens) against KV blocks j (block_kv = 64 tokens):
+ *   qbar_i, kbar_j  mean of the valid tokens of the block (fp64)
+ *   S_ij            qbar_i . kbar_j / sqrt(D)
+ *   labels          per row i, total order (S desc, j asc): first kc blocks
+ *                   critical (2), last kn negligible (0), the rest marginal (1);
+ *                   kc = ceil(kh_ppm * Nk / 1e6), kn = floor(kl_ppm * Nk / 1e6),
+ *                   kh_ppm = round(kh * 1e6), kl_ppm = round(kl * 1e6)
+ *   O_s             softmax(q k^T / sqrt(D)) v over the tokens of the critical
+ *                   blocks only (0 when there is none)
+ *   O_l             phi(q) H_i / (phi(q) . Z_i), H_i = sum h_j, Z_i = sum z_j over
+ *                   the marginal blocks, h_j = phi(K_j)^T V_j, z_j = colsum phi(K_j),
+ *                   phi(x) = elu(x) + 1 (0 when there is no marginal block)
+ *   O               alpha[h, :] * O_s + (1 - alpha[h, :]) * O_l
+ *
+ * Conventions (all entry points):
+ *   - Tensors are device pointers owned by the caller; the library allocates
+ *     no device memory. Q, K, V and O are [B, H, N, D] bf16, contiguous, D
+ *     fastest, 16-byte aligned. alpha is [H, D] fp32.
+ *   - Supported: D in {64, 128}; block_q in {64, 128}; block_kv = 64;
+ *     1 <= N; Nk = ceil(N / 64) <= 16384; 0 <= kh, kl and kh + kl <= 1.
+ *   - Work is enqueued on the caller's stream; calls return before it runs.
+ *   - Argument errors are found on the host before anything is enqueued; then
+ *     nothing is written. Errors found on the device (a bounded wait that ran
+ *     out, a caller label outside {0,1,2}) are recorded in the workspace's
+ *     error word and reported by sla_check.
+ *   - No entry point throws or exits; each returns an sla_status, and
+ *     sla_last_error() gives a message for the calling thread's last failure.
+ *   - The workspace (ws, ws_bytes >= sla_workspace_size) is caller memory,
+ *     256-byte aligned; its first 256 bytes hold the device error word and
+ *     must be zero before the first call that uses it (sla_check clears it).
+ *     Concurrent calls must not share a workspace.
+ */
+#ifndef SLA_H_
+#define SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or fraction */
+  SLA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. D = 96) */
+  SLA_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+  SLA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+  SLA_ERR_TIMEOUT = 5,     /* a device-side bounded wait ran out (reported by sla_check) */
+  SLA_ERR_BAD_MASK = 6     /* caller label outside {0,1,2} (reported by sla_check) */
+} sla_status;
+
+/* Problem shape. kh / kl: critical / negligible fractions of the KV blocks per row. */
+typedef struct {
+  int B, H, N, D;
+  int block_q, block_kv;
+  float kh, kl;
+} sla_problem;
+
+/* Block counts: Nq = ceil(N / block_q), Nk = ceil(N / block_kv), kc and kn as above.
+ * Host only. Any output pointer may be NULL. */
+sla_status sla_counts(const sla_problem* p, int* Nq, int* Nk, int* kc, int* kn);
+
+/* Bytes of workspace sla_route / sla_forward need for this shape (0 on invalid shape).
+ * Host only. */
+size_t sla_workspace_size(const sla_problem* p);
+
+/* Block router (SLA2 §2.B; SLA Abstract).
+ *   q, k          [B,H,N,D] bf16 device
+ *   mask_out      [B,H,Nq,Nk] int8 device: 2 critical, 1 marginal, 0 negligible
+ *   crit_idx_out  [B,H,Nq,kc] int32 device, critical block indices ascending (nullable)
+ *   scores_out    [B,H,Nq,Nk] fp64 device, raw compressed scores S (nullable)
+ *   ws, ws_bytes  workspace
+ *   stream        cudaStream_t (0 = legacy default stream) */
+sla_status sla_route(const sla_problem* p, const void* q, const void* k, int8_t* mask_out,
+                     int32_t* crit_idx_out, double* scores_out, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Per-KV-block linear-attention states (SLA Abstract: O(N) branch).
+ *   k, v   [B,H,N,D] bf16 device
+ *   h_out  [B,H,Nk,D,D] fp32 device, h_j = phi(K_j)^T V_j over the block's valid tokens
+ *   z_out  [B,H,Nk,D] fp32 device, z_j = colsum phi(K_j)
+ *   ws     workspace for the error word (nullable: device errors then go unreported) */
+sla_status sla_kv_states(const sla_problem* p, const void* k, const void* v, float* h_out,
+                         float* z_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Fused forward (SLA Abstract; SLA2 §2.A blend).
+ *   q, k, v   [B,H,N,D] bf16 device
+ *   alpha     [H,D] fp32 device, blend ratio per head and channel
+ *   mask      [B,H,Nq,Nk] int8 device labels replacing the router (nullable);
+ *             with a mask, kh and kl are ignored and each row may hold any counts
+ *   out       [B,H,N,D] bf16 device; must not alias q, k or v
+ *   ws        workspace */
+sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const void* v,
+                       const float* alpha, const int8_t* mask, void* out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Synchronise the stream, read and clear the workspace's device error word.
+ * Returns SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_BAD_MASK (or SLA_ERR_CUDA). */
+sla_status sla_check(void* ws, void* stream);
+
+/* Message for the calling thread's most recent failed call ("" if none). */
+const char* sla_last_error(void);
+
+/* Library version string. */
+const char* sla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H_ */

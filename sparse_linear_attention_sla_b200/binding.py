@@ -1,0 +1,206 @@
+"""Python binding over the C ABI in include/sla.h (argument marshalling only).
+
+Every step of the computation runs in libsla.so's CUDA kernels; this module
+checks tensor shapes/dtypes, takes the current torch CUDA stream, allocates
+outputs and workspaces with torch, and calls the library through ctypes. There
+is no CPU path: without the built library, or without a CUDA device, every
+call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsla.so")
+
+SLA_OK = 0
+_STATUS = {
+    0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_WORKSPACE",
+    4: "SLA_ERR_CUDA", 5: "SLA_ERR_TIMEOUT", 6: "SLA_ERR_BAD_MASK",
+}
+
+# Every symbol include/sla.h declares.
+EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sla_forward",
+           "sla_check", "sla_last_error", "sla_version")
+
+
+class SlaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("D", ctypes.c_int),
+                ("block_q", ctypes.c_int), ("block_kv", ctypes.c_int),
+                ("kh", ctypes.c_float), ("kl", ctypes.c_float)]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsla.so and declare its signatures. Raises if the library is missing."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m sparse_linear_attention_sla_b200.build` "
+                "(there is no CPU fallback)")
+        lib = ctypes.CDLL(path)
+        P = ctypes.POINTER(Problem)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.sla_counts.argtypes = [P, ip, ip, ip, ip]
+        lib.sla_workspace_size.argtypes = [P]
+        lib.sla_workspace_size.restype = sz
+        lib.sla_route.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_kv_states.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_check.argtypes = [vp, vp]
+        lib.sla_last_error.restype = ctypes.c_char_p
+        lib.sla_version.restype = ctypes.c_char_p
+        for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_check"):
+            getattr(lib, name).restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _raise(status: int):
+    if status != SLA_OK:
+        msg = load_library().sla_last_error().decode(errors="replace")
+        raise SlaError(status, msg)
+
+
+def problem(B, H, N, D, block_q, block_kv, kh=0.0, kl=0.0) -> Problem:
+    return Problem(int(B), int(H), int(N), int(D), int(block_q), int(block_kv), float(kh), float(kl))
+
+
+def counts(p: Problem) -> Tuple[int, int, int, int]:
+    """(Nq, Nk, kc, kn) as the library computes them (host only)."""
+    out = [ctypes.c_int(0) for _ in range(4)]
+    _raise(load_library().sla_counts(ctypes.byref(p), *[ctypes.byref(o) for o in out]))
+    return tuple(o.value for o in out)
+
+
+def workspace_size(p: Problem) -> int:
+    return int(load_library().sla_workspace_size(ctypes.byref(p)))
+
+
+def new_workspace(p: Problem, device) -> torch.Tensor:
+    """A zero-headed workspace for problem p on device (bytes, 256-byte aligned by the allocator)."""
+    n = workspace_size(p)
+    if n == 0:
+        counts(p)  # raises with the library's message
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def _stream_handle(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check_act(name, t, B, H, N, D, device):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16 or tuple(t.shape) != (B, H, N, D) or not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous bf16 of shape {(B, H, N, D)}, got {t.dtype} {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def route(q, k, block_q, block_kv, kh, kl, want_scores=False, want_crit=False, ws=None):
+    """Block labels [B,H,Nq,Nk] int8 (2 critical, 1 marginal, 0 negligible).
+
+    Returns (mask, crit_idx or None, scores or None).
+    """
+    B, H, N, D = q.shape
+    _check_act("q", q, B, H, N, D, q.device)
+    _check_act("k", k, B, H, N, D, q.device)
+    p = problem(B, H, N, D, block_q, block_kv, kh, kl)
+    Nq, Nk, kc, _ = counts(p)
+    dev = q.device
+    mask = torch.empty(B, H, Nq, Nk, dtype=torch.int8, device=dev)
+    crit = torch.empty(B, H, Nq, kc, dtype=torch.int32, device=dev) if want_crit else None
+    scores = torch.empty(B, H, Nq, Nk, dtype=torch.float64, device=dev) if want_scores else None
+    if ws is None:
+        ws = new_workspace(p, dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_route(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(mask), _ptr(crit), _ptr(scores), _ptr(ws),
+                           ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+    _raise(st)
+    return mask, crit, scores
+
+
+def kv_states(k, v, block_kv=64, ws=None):
+    """Per-KV-block states h [B,H,Nk,D,D] and z [B,H,Nk,D], fp32."""
+    B, H, N, D = k.shape
+    _check_act("k", k, B, H, N, D, k.device)
+    _check_act("v", v, B, H, N, D, k.device)
+    p = problem(B, H, N, D, 128 if D == 128 else 64, block_kv)
+    _, Nk, _, _ = counts(p)
+    dev = k.device
+    h = torch.empty(B, H, Nk, D, D, dtype=torch.float32, device=dev)
+    z = torch.empty(B, H, Nk, D, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_kv_states(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(h), _ptr(z), _ptr(ws),
+                               ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+    _raise(st)
+    return h, z
+
+
+def forward(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, out=None, ws=None):
+    """Fused SLA forward: O = alpha * O_s + (1 - alpha) * O_l, bf16 [B,H,N,D]."""
+    B, H, N, D = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_act(name, t, B, H, N, D, dev)
+    if alpha.dtype != torch.float32 or tuple(alpha.shape) != (H, D) or not alpha.is_contiguous() or alpha.device != dev:
+        raise ValueError(f"alpha must be contiguous fp32 [{H}, {D}] on {dev}")
+    p = problem(B, H, N, D, block_q, block_kv, kh, kl)
+    Nq, Nk, _, _ = counts(p)
+    if mask is not None:
+        if mask.dtype != torch.int8 or tuple(mask.shape) != (B, H, Nq, Nk) or not mask.is_contiguous() \
+                or mask.device != dev:
+            raise ValueError(f"mask must be contiguous int8 [{B}, {H}, {Nq}, {Nk}] on {dev}")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_act("out", out, B, H, N, D, dev)
+    if ws is None:
+        ws = new_workspace(p, dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(mask), _ptr(out),
+                             _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+    _raise(st)
+    return out
+
+
+def check(ws: torch.Tensor):
+    """Synchronise and raise if a kernel recorded a device-side error in ws."""
+    lib = load_library()
+    with torch.cuda.device(ws.device):
+        _raise(lib.sla_check(_ptr(ws), _stream_handle(ws.device)))
+
+
+def version() -> str:
+    return load_library().sla_version().decode()

@@ -1,0 +1,377 @@
+// Fused SLA attention tile: one CTA computes the output of one query block
+// (128 query rows) of one (batch, head):
+//
+//   sparse branch  O_s = softmax over the keys of the critical KV blocks only
+//                        (online softmax, renormalised over that set)
+//   linear branch  O_l = phi(Q_i) H_i / (phi(Q_i) Z_i), H_i, Z_i = sums of the
+//                        marginal blocks' states (precomputed per row)
+//   blend          O   = alpha_h * O_s + (1 - alpha_h) * O_l        (per channel)
+//
+// Sources: "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
+// Sparse-Linear Attention", Abstract (exact attention for critical weights,
+// linear attention for marginal ones, negligible ones skipped, one fused
+// kernel); "SLA2: Sparse-Linear Attention with Learnable Routing and QAT" §1
+// item 1 (the sparse branch renormalises over its keys) and §2.A
+// (O = alpha * O_s + (1 - alpha) * O_l).
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: Q tile, H_i tile, then K_j / V_j of every
+//               critical block j through an NS-stage ring.
+//   warp 1      TMEM owner and single-thread tcgen05 MMA issuer:
+//               S = Q K_j^T (M=128, N=64), O_s += P V_j (M=128, N=D),
+//               O_l = phi(Q) H_i (M=128, N=D).
+//   warps 2..5  softmax / epilogue warpgroup: thread <-> query row <-> TMEM lane.
+//
+// TMEM columns: S ping-pong [0,64) [64,128), O_s [128,128+D), O_l [128+D,128+2D).
+// An empty critical set gives O_s = 0; an empty marginal set gives Z_i = 0 and
+// O_l = 0.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace sla {
+
+struct AttnArgs {
+  int H, N, Nq, block_q;
+  const int32_t* crit;      // [BH*Nq, crit_ld] critical KV block indices, ascending
+  int crit_ld;
+  const int32_t* crit_cnt;  // [BH*Nq]
+  const float* Zagg;        // [BH*Nq, D]
+  const float* alpha;       // [H, D]
+  float scale_log2;         // log2(e) / sqrt(D)
+  uint32_t* err;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void wg_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int D>
+struct AttnSmem {
+  static constexpr uint32_t Q = 128 * D * 2;       // Q tile (later phi(Q), then the output staging)
+  static constexpr uint32_t KV = 64 * D * 2;       // one K or V stage
+  static constexpr uint32_t P = 128 * 64 * 2;      // one P buffer
+  static constexpr uint32_t HT = D * D * 2;        // H_i tile
+  template <int NS>
+  static constexpr uint32_t total() { return Q + 2 * NS * KV + 2 * P + HT + 1024; }
+};
+
+template <int D, int NS>
+__global__ void __launch_bounds__(192, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
+                const __grid_constant__ CUtensorMap map_o, AttnArgs a) {
+  using L = AttnSmem<D>;
+  constexpr int DB = D / 64;                    // 64-column boxes per row
+  constexpr uint32_t TMEM_COLS = (128 + 2 * D) <= 256 ? 256 : 512;
+  constexpr uint32_t OS = 128, OL = 128 + D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;
+  uint8_t* sK = sQ + L::Q;
+  uint8_t* sV = sK + NS * L::KV;
+  uint8_t* sP = sV + NS * L::KV;
+  uint8_t* sH = sP + 2 * L::P;
+
+  __shared__ uint64_t q_full, h_full, phiq_full, ol_done, drain;
+  __shared__ uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
+  __shared__ uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+  __shared__ float sZ[D], sAlpha[D];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
+  const int row_id = bh * a.Nq + i;
+  const int kc = a.crit_cnt[row_id];
+  const int32_t* clist = a.crit + static_cast<size_t>(row_id) * a.crit_ld;
+
+  if (tid == 0) {
+    mbar_init(&q_full, 1);
+    mbar_init(&h_full, 1);
+    mbar_init(&phiq_full, 128);
+    mbar_init(&ol_done, 1);
+    mbar_init(&drain, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 128);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&map_q);
+      prefetch_tmap(&map_k);
+      prefetch_tmap(&map_v);
+      prefetch_tmap(&map_h);
+      mbar_arrive_expect_tx(&q_full, L::Q);
+      for (int b = 0; b < DB; ++b) tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * a.block_q, bh);
+      mbar_arrive_expect_tx(&h_full, L::HT);
+      for (int dh = 0; dh < DB; ++dh)
+        for (int eh = 0; eh < DB; ++eh)
+          tma_load_2d(sH + (dh * DB + eh) * 8192, &map_h, &h_full, eh * 64, row_id * D + dh * 64);
+      int last_round[NS];
+      for (int s = 0; s < NS; ++s) last_round[s] = -1;
+      for (int n = 0; n < kc; ++n) {
+        const int s = n % NS, r = n / NS;
+        const int j = clist[n];
+        if (r > 0 && !mbar_wait(&k_empty[s], (r - 1) & 1, a.err, &abort_flag)) break;
+        mbar_arrive_expect_tx(&k_full[s], L::KV);
+        for (int b = 0; b < DB; ++b) tma_load_3d(sK + s * L::KV + b * 8192, &map_k, &k_full[s], b * 64, j * 64, bh);
+        if (r > 0 && !mbar_wait(&v_empty[s], (r - 1) & 1, a.err, &abort_flag)) {
+          last_round[s] = r;  // the K half of this stage is in flight
+          mbar_wait(&k_full[s], r & 1, nullptr, nullptr);
+          last_round[s] = -1;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[s], L::KV);
+        for (int b = 0; b < DB; ++b) tma_load_3d(sV + s * L::KV + b * 8192, &map_v, &v_full[s], b * 64, j * 64, bh);
+        last_round[s] = r;
+      }
+      if (abort_flag) {  // let every load still in flight land before the CTA retires
+        mbar_wait(&q_full, 0, nullptr, nullptr);
+        mbar_wait(&h_full, 0, nullptr, nullptr);
+        for (int s = 0; s < NS; ++s)
+          if (last_round[s] >= 0) {
+            mbar_wait(&k_full[s], last_round[s] & 1, nullptr, nullptr);
+            mbar_wait(&v_full[s], last_round[s] & 1, nullptr, nullptr);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);
+      const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV), p0 = smem_u32(sP), h0 = smem_u32(sH);
+      bool ok = mbar_wait(&q_full, 0, a.err, &abort_flag);
+      auto issue_pv = [&](int m) -> bool {
+        const int b = m & 1, s = m % NS;
+        if (!mbar_wait(&p_full[b], (m >> 1) & 1, a.err, &abort_flag)) return false;
+        if (!mbar_wait(&v_full[s], (m / NS) & 1, a.err, &abort_flag)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = smem_desc_sw128(p0 + b * L::P + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(v0 + s * L::KV + kk * 2048, 8192, 1024);
+          umma_bf16_ss(tmem + OS, ad, bd, id_o, (m > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done[b]);
+        umma_commit(&v_empty[s]);
+        return true;
+      };
+      for (int n = 0; ok && n < kc; ++n) {
+        const int s = n % NS, b = n & 1;
+        if (!mbar_wait(&k_full[s], (n / NS) & 1, a.err, &abort_flag)) { ok = false; break; }
+        if (n >= 2 && !mbar_wait(&s_free[b], ((n >> 1) - 1) & 1, a.err, &abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(k0 + s * L::KV + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          umma_bf16_ss(tmem + b * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[b]);
+        umma_commit(&k_empty[s]);
+        if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
+      }
+      if (ok && kc > 0) ok = issue_pv(kc - 1);
+      // linear branch: O_l = phi(Q) H_i once the warpgroup has rewritten Q as phi(Q)
+      if (ok) ok = mbar_wait(&h_full, 0, a.err, &abort_flag);
+      if (ok) ok = mbar_wait(&phiq_full, 0, a.err, &abort_flag);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(h0 + (kk >> 2) * DB * 8192 + (kk & 3) * 2048, 8192, 1024);
+          umma_bf16_ss(tmem + OL, ad, bd, id_o, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&ol_done);
+      }
+      umma_commit(&drain);  // every MMA issued above has finished once this arrives
+      mbar_wait(&drain, 0, nullptr, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue warpgroup
+    const int wt = tid - 64;                    // 0..127
+    const int quarter = warp & 3;               // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;          // query row within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    for (int c = wt; c < D; c += 128) {
+      sZ[c] = a.Zagg[static_cast<size_t>(row_id) * D + c];
+      sAlpha[c] = a.alpha[h * D + c];
+    }
+    wg_barrier();
+
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int n = 0; n < kc; ++n) {
+      const int b = n & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (n >> 1) & 1, a.err, &abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld32(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(lane_addr + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[b]);
+
+      const int j = clist[n];
+      const int valid = min(64, a.N - j * 64);
+      float x[64];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        x[c] = c < valid ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      if (n == 0) {
+        m_run = mx;
+      } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
+        // The running maximum grew by more than 2^8: rescale O_s (needs PV_{n-1} finished).
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, &abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const float m_new = fmaxf(m_run, mx);
+        const float f = fast_exp2(m_run - m_new);
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + OS + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+          tmem_st32(lane_addr + OS + c0, o);
+        }
+        tmem_wait_st();
+        l_run *= f;
+        m_run = m_new;
+      }
+      float ps = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float e0 = fast_exp2(x[c] - m_run), e1 = fast_exp2(x[c + 1] - m_run);
+        ps += e0 + e1;
+        pk[c >> 1] = pack_bf16x2(e0, e1);
+      }
+      l_run += ps;
+      if (n >= 2) {  // P buffer b is free once PV_{n-2} has finished
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[b], ((n - 2) >> 1) & 1, a.err, &abort_flag));
+        if (!ok) break;
+      }
+      uint8_t* prow = sP + b * L::P;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8)
+        *reinterpret_cast<uint4*>(prow + sw128_offset(r, c8 * 16)) =
+            make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    // Every MMA that reads Q has finished once the last PV has (commits complete in order).
+    if (ok && kc > 0)
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(kc - 1) & 1], ((kc - 1) >> 1) & 1, a.err, &abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, a.err, &abort_flag));
+
+    // phi(Q) in place (bf16), and the linear-branch denominator phi(q) . Z_i with the
+    // same rounded phi(q) the MMA sees.
+    float den = 0.f;
+    if (ok) {
+#pragma unroll
+      for (int c8 = 0; c8 < D / 8; ++c8) {
+        uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
+        uint4 u = *p;
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 f = unpack_bf16x2(w[e]);
+          const float g0 = f.x > 0.f ? f.x + 1.f : __expf(f.x);
+          const float g1 = f.y > 0.f ? f.y + 1.f : __expf(f.y);
+          w[e] = pack_bf16x2(g0, g1);
+          const float2 gr = unpack_bf16x2(w[e]);
+          den = fmaf(gr.x, sZ[c8 * 8 + 2 * e], den);
+          den = fmaf(gr.y, sZ[c8 * 8 + 2 * e + 1], den);
+        }
+        *p = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    mbar_arrive(&phiq_full);
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, 0, a.err, &abort_flag));
+
+    // Epilogue: O = alpha * O_s / l + (1 - alpha) * O_l / den -> bf16 staging (reuses sQ) -> TMA store.
+    const uint32_t box_bytes = static_cast<uint32_t>(a.block_q) * 128u;
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv_d = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t os[32], ol[32];
+        tmem_ld32(lane_addr + OS + c0, os);
+        tmem_ld32(lane_addr + OL + c0, ol);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float al0 = sAlpha[c0 + c], al1 = sAlpha[c0 + c + 1];
+          const float y0 = al0 * (kc > 0 ? __uint_as_float(os[c]) * inv_l : 0.f) +
+                           (1.f - al0) * (__uint_as_float(ol[c]) * inv_d);
+          const float y1 = al1 * (kc > 0 ? __uint_as_float(os[c + 1]) * inv_l : 0.f) +
+                           (1.f - al1) * (__uint_as_float(ol[c + 1]) * inv_d);
+          pk[c >> 1] = pack_bf16x2(y0, y1);
+        }
+        if (r < a.block_q) {
+          uint8_t* box = sQ + (c0 >> 6) * box_bytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(box + sw128_offset(r, ((c0 & 63) >> 3) * 16 + q * 16)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    wg_barrier();
+    if (wt == 0 && !abort_flag) {
+      for (int bcol = 0; bcol < DB; ++bcol) tma_store_3d(&map_o, sQ + bcol * box_bytes, bcol * 64, i * a.block_q, bh);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace sla

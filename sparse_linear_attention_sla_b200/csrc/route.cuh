@@ -1,0 +1,229 @@
+// Block router for the SLA forward.
+//
+//   score_kernel : S_ij = qbar_i . kbar_j / sqrt(D) in fp64 (compressed scores)
+//   select_kernel: per query-block row, label every KV block critical (2),
+//                  marginal (1) or negligible (0): the first kc blocks in the
+//                  total order (S descending, j ascending) are critical, the
+//                  last kn are negligible.
+//   mask_lists_kernel: the same outputs from a caller-supplied label mask.
+//
+// Sources: "SLA2: Sparse-Linear Attention with Learnable Routing and QAT" §2.B
+// (pooled Q/K, compressed scores, hard top-k at inference); "SLA: Beyond
+// Sparsity in Diffusion Transformers via Fine-Tunable Sparse-Linear Attention",
+// Abstract (critical / marginal / negligible). The softmax of the compressed
+// scores is monotone, so ranking the raw scores gives the same labels.
+//
+// The decision is taken in fp64 (pooled sums of bf16 inputs are exact in fp64
+// for ordinary inputs), so labels differ from an fp64 reference only where two
+// scores agree to the last bits.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace sla {
+
+// ---------------------------------------------------------------- scores
+// grid: (ceil(Nk/64), ceil(Nq/64), BH); block 256. Each thread computes a 4 x 4 patch.
+template <int D>
+__global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
+                                                    double* __restrict__ S, int Nq, int Nk) {
+  constexpr int T = 64, DC = 32;
+  __shared__ double sq[DC][T + 1];
+  __shared__ double sk[DC][T + 1];
+  const int bh = blockIdx.z, i0 = blockIdx.y * T, j0 = blockIdx.x * T;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  const double* qb = qbar + static_cast<size_t>(bh) * Nq * D;
+  const double* kb = kbar + static_cast<size_t>(bh) * Nk * D;
+  double acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+  for (int d0 = 0; d0 < D; d0 += DC) {
+    for (int e = tid; e < T * DC; e += 256) {
+      const int r = e / DC, d = e % DC;
+      sq[d][r] = (i0 + r < Nq) ? qb[static_cast<size_t>(i0 + r) * D + d0 + d] : 0.0;
+      sk[d][r] = (j0 + r < Nk) ? kb[static_cast<size_t>(j0 + r) * D + d0 + d] : 0.0;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int d = 0; d < DC; ++d) {
+      double qa[4], kb4[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) qa[a] = sq[d][ty + 16 * a];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) kb4[b] = sk[d][tx + 16 * b];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fma(qa[a], kb4[b], acc[a][b]);
+    }
+    __syncthreads();
+  }
+  const double rs = sqrt(static_cast<double>(D));
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int i = i0 + ty + 16 * a;
+    if (i >= Nq) continue;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int j = j0 + tx + 16 * b;
+      if (j < Nk) S[(static_cast<size_t>(bh) * Nq + i) * Nk + j] = acc[a][b] / rs;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- selection
+
+// Order-preserving map from a double to an unsigned key (larger key = larger value).
+// -0.0 is folded onto +0.0 so that the two compare equal, as they do as numbers.
+__device__ __forceinline__ uint64_t order_key(double s) {
+  s = s + 0.0;
+  const uint64_t u = static_cast<uint64_t>(__double_as_longlong(s));
+  return (u >> 63) ? ~u : (u | (1ull << 63));
+}
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Largest t with #{keys >= t} >= k (the k-th largest key), k >= 1, by bisection on the bits.
+// If flip, keys are complemented first (gives the complement of the k-th smallest key).
+__device__ __forceinline__ uint64_t kth_largest(const uint64_t* keys, int n, int k, bool flip) {
+  const int lane = threadIdx.x & 31;
+  uint64_t T = 0;
+  for (int bit = 63; bit >= 0; --bit) {
+    const uint64_t cand = T | (1ull << bit);
+    int c = 0;
+    for (int j = lane; j < n; j += 32) {
+      const uint64_t key = flip ? ~keys[j] : keys[j];
+      c += key >= cand;
+    }
+    if (warp_sum(c) >= k) T = cand;
+  }
+  return T;
+}
+
+struct SelectArgs {
+  const double* S;      // [rows, Nk]
+  int rows, Nk, kc, kn;
+  int8_t* mask;         // [rows, Nk] labels (nullable)
+  int32_t* crit;        // [rows, crit_ld] critical block indices, ascending (nullable)
+  int crit_ld;
+  int32_t* crit_cnt;    // [rows] (nullable)
+  __nv_bfloat16* W;     // [rows, w_ld] marginal indicator (1 marginal, else 0), zero padded (nullable)
+  int w_ld;
+};
+
+// One warp per row; dynamic smem = warps_per_cta * Nk * 8 bytes of keys.
+__global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
+  extern __shared__ uint64_t keys_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpc = blockDim.x >> 5;
+  const int row = blockIdx.x * wpc + warp;
+  if (row >= a.rows) return;  // whole warp leaves; nothing below synchronises the CTA
+  uint64_t* keys = keys_all + static_cast<size_t>(warp) * a.Nk;
+  const double* srow = a.S + static_cast<size_t>(row) * a.Nk;
+  for (int j = lane; j < a.Nk; j += 32) keys[j] = order_key(srow[j]);
+  __syncwarp();
+
+  // Critical: the kc largest in (key desc, index asc). Tc = kc-th largest key;
+  // every key > Tc is critical and the first (kc - #{> Tc}) keys == Tc by index.
+  uint64_t Tc = 0, Tn = 0;
+  int need_c = 0, need_n = 0, tot_eq_n = 0;
+  if (a.kc > 0) {
+    Tc = kth_largest(keys, a.Nk, a.kc, false);
+    int gt = 0;
+    for (int j = lane; j < a.Nk; j += 32) gt += keys[j] > Tc;
+    need_c = a.kc - warp_sum(gt);
+  }
+  // Negligible: the kn last in the same order = the kn smallest keys, ties
+  // resolved towards the higher index. Tn = kn-th smallest key.
+  if (a.kn > 0) {
+    Tn = ~kth_largest(keys, a.Nk, a.kn, true);
+    int lt = 0, eq = 0;
+    for (int j = lane; j < a.Nk; j += 32) {
+      lt += keys[j] < Tn;
+      eq += keys[j] == Tn;
+    }
+    need_n = a.kn - warp_sum(lt);
+    tot_eq_n = warp_sum(eq);
+  }
+
+  int eqc_before = 0, eqn_before = 0, crit_before = 0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int j0 = 0; j0 < a.Nk; j0 += 32) {
+    const int j = j0 + lane;
+    const bool in = j < a.Nk;
+    const uint64_t key = in ? keys[j] : 0;
+    const bool eqc = in && a.kc > 0 && key == Tc;
+    const bool eqn = in && a.kn > 0 && key == Tn;
+    const uint32_t bc = __ballot_sync(0xffffffffu, eqc);
+    const uint32_t bn = __ballot_sync(0xffffffffu, eqn);
+    const int rank_c = eqc_before + __popc(bc & lt_mask);
+    const int rank_n = eqn_before + __popc(bn & lt_mask);
+    const bool is_c = in && a.kc > 0 && (key > Tc || (eqc && rank_c < need_c));
+    // ties at Tn with the highest indices are the negligible ones
+    const bool is_n = in && a.kn > 0 && (key < Tn || (eqn && (tot_eq_n - rank_n - 1) < need_n));
+    const uint32_t bcrit = __ballot_sync(0xffffffffu, is_c);
+    if (in) {
+      const int8_t lab = is_c ? 2 : (is_n ? 0 : 1);
+      if (a.mask) a.mask[static_cast<size_t>(row) * a.Nk + j] = lab;
+      if (a.W) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(lab == 1 ? 1.f : 0.f);
+      if (is_c && a.crit) a.crit[static_cast<size_t>(row) * a.crit_ld + crit_before + __popc(bcrit & lt_mask)] = j;
+    }
+    eqc_before += __popc(bc);
+    eqn_before += __popc(bn);
+    crit_before += __popc(bcrit);
+  }
+  if (a.W)
+    for (int j = a.Nk + lane; j < a.w_ld; j += 32) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(0.f);
+  if (lane == 0 && a.crit_cnt) a.crit_cnt[row] = crit_before;
+}
+
+// ---------------------------------------------------------------- caller mask
+struct MaskListArgs {
+  const int8_t* mask;   // [rows, Nk]
+  int rows, Nk;
+  int32_t* crit;
+  int crit_ld;
+  int32_t* crit_cnt;
+  __nv_bfloat16* W;
+  int w_ld;
+  uint32_t* err;
+};
+
+// One warp per row: critical list (ascending), counts and marginal indicator
+// from the caller's labels. A label outside {0, 1, 2} is reported through the
+// device error word and that block is treated as negligible.
+__global__ void __launch_bounds__(256) mask_lists_kernel(MaskListArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= a.rows) return;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int crit_before = 0;
+  bool bad = false;
+  for (int j0 = 0; j0 < a.Nk; j0 += 32) {
+    const int j = j0 + lane;
+    const bool in = j < a.Nk;
+    int lab = in ? a.mask[static_cast<size_t>(row) * a.Nk + j] : 0;
+    if (lab < 0 || lab > 2) {
+      bad = true;
+      lab = 0;
+    }
+    const bool is_c = in && lab == 2;
+    const uint32_t bcrit = __ballot_sync(0xffffffffu, is_c);
+    if (in) {
+      a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(lab == 1 ? 1.f : 0.f);
+      if (is_c) a.crit[static_cast<size_t>(row) * a.crit_ld + crit_before + __popc(bcrit & lt_mask)] = j;
+    }
+    crit_before += __popc(bcrit);
+  }
+  for (int j = a.Nk + lane; j < a.w_ld; j += 32) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(0.f);
+  if (lane == 0) a.crit_cnt[row] = crit_before;
+  if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(a.err, SLA_DEVERR_BAD_MASK);
+}
+
+}  // namespace sla

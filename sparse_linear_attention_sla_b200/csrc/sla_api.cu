@@ -1,0 +1,471 @@
+// Host side of the C ABI declared in include/sla.h: argument checks, block
+// counts, workspace layout, TMA descriptors and kernel launches.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/sla.h"
+#include "aggregate.cuh"
+#include "attention.cuh"
+#include "prep.cuh"
+#include "route.cuh"
+
+namespace {
+
+using sla::AggArgs;
+using sla::AttnArgs;
+using sla::KvPrepArgs;
+using sla::MaskListArgs;
+using sla::SelectArgs;
+
+constexpr int kMaxNk = 16384;
+constexpr int kAttnStages = 3;
+thread_local std::string g_last_error;
+
+sla_status fail(sla_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+#define SLA_CUDA(call)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) return fail(SLA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+// ------------------------------------------------------------------ shape
+
+struct Shape {
+  int B, H, N, D, bq, bk, BH;
+  int Nq, Nk, kc, kn;
+  int LD;     // row length of the stacked per-block states (D*D + 128)
+  int w_ld;   // row stride of the marginal indicator (Nk rounded up to 64)
+};
+
+sla_status make_shape(const sla_problem* p, Shape* s) {
+  if (!p) return fail(SLA_ERR_INVALID_ARG, "problem is NULL");
+  if (p->B < 1 || p->H < 1 || p->N < 1) return fail(SLA_ERR_INVALID_ARG, "B, H, N must be >= 1");
+  if (p->D != 64 && p->D != 128) return fail(SLA_ERR_UNSUPPORTED, "D=%d not supported (64 or 128)", p->D);
+  if (p->block_kv != 64) return fail(SLA_ERR_UNSUPPORTED, "block_kv=%d not supported (64)", p->block_kv);
+  if (p->block_q != 64 && p->block_q != 128)
+    return fail(SLA_ERR_UNSUPPORTED, "block_q=%d not supported (64 or 128)", p->block_q);
+  if (!std::isfinite(p->kh) || !std::isfinite(p->kl)) return fail(SLA_ERR_INVALID_ARG, "kh, kl must be finite");
+  const long long kh_ppm = llround(static_cast<double>(p->kh) * 1e6);
+  const long long kl_ppm = llround(static_cast<double>(p->kl) * 1e6);
+  if (kh_ppm < 0 || kl_ppm < 0 || kh_ppm + kl_ppm > 1000000)
+    return fail(SLA_ERR_INVALID_ARG, "need 0 <= kh, kl and kh + kl <= 1 (got %g, %g)", p->kh, p->kl);
+  const long long BH = static_cast<long long>(p->B) * p->H;
+  if (BH > 65535) return fail(SLA_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", BH);
+  s->B = p->B;
+  s->H = p->H;
+  s->N = p->N;
+  s->D = p->D;
+  s->bq = p->block_q;
+  s->bk = p->block_kv;
+  s->BH = static_cast<int>(BH);
+  s->Nq = (p->N + p->block_q - 1) / p->block_q;
+  s->Nk = (p->N + p->block_kv - 1) / p->block_kv;
+  if (s->Nk > kMaxNk) return fail(SLA_ERR_UNSUPPORTED, "N=%d gives %d KV blocks (max %d)", p->N, s->Nk, kMaxNk);
+  if (static_cast<long long>(s->BH) * s->Nq * s->D >= (1ll << 31))
+    return fail(SLA_ERR_UNSUPPORTED, "B*H*Nq*D too large");
+  s->kc = static_cast<int>((kh_ppm * s->Nk + 999999) / 1000000);
+  s->kn = static_cast<int>((kl_ppm * s->Nk) / 1000000);
+  s->LD = s->D * s->D + 128;
+  s->w_ld = (s->Nk + 63) / 64 * 64;
+  return SLA_OK;
+}
+
+// ------------------------------------------------------------------ workspace
+
+struct Workspace {
+  uint32_t* err;
+  double* qbar;
+  double* kbar;
+  double* S;
+  int8_t* mask;
+  int32_t* crit;
+  int32_t* crit_cnt;
+  __nv_bfloat16* W;
+  __nv_bfloat16* hst;
+  __nv_bfloat16* Hagg;
+  float* Zagg;
+  size_t bytes;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+Workspace layout(const Shape& s, uint8_t* base) {
+  Workspace w{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  const size_t BH = s.BH;
+  w.err = reinterpret_cast<uint32_t*>(take(256));
+  w.qbar = reinterpret_cast<double*>(take(BH * s.Nq * s.D * sizeof(double)));
+  w.kbar = reinterpret_cast<double*>(take(BH * s.Nk * s.D * sizeof(double)));
+  w.S = reinterpret_cast<double*>(take(BH * s.Nq * s.Nk * sizeof(double)));
+  w.mask = reinterpret_cast<int8_t*>(take(BH * s.Nq * s.Nk));
+  w.crit = reinterpret_cast<int32_t*>(take(BH * s.Nq * s.Nk * sizeof(int32_t)));
+  w.crit_cnt = reinterpret_cast<int32_t*>(take(BH * s.Nq * sizeof(int32_t)));
+  w.W = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nq * s.w_ld * 2));
+  w.hst = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(s.LD) * 2));
+  w.Hagg = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nq * static_cast<size_t>(s.D) * s.D * 2));
+  w.Zagg = reinterpret_cast<float*>(take(BH * s.Nq * s.D * sizeof(float)));
+  w.bytes = off;
+  return w;
+}
+
+sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w) {
+  if (!ws) return fail(SLA_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(SLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  *w = layout(s, static_cast<uint8_t*>(ws));
+  if (ws_bytes < w->bytes)
+    return fail(SLA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, w->bytes);
+  return SLA_OK;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) % 16) == 0; }
+
+// ------------------------------------------------------------------ TMA descriptors
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle. dims/strides in elements (innermost first).
+sla_status make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_el,
+                    const uint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (int r = 0; r < rank; ++r) {
+    d[r] = dims[r];
+    b[r] = box[r];
+    es[r] = 1;
+  }
+  for (int r = 0; r + 1 < rank; ++r) st[r] = strides_el[r] * 2;
+  CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), d, st, b, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (res != CUDA_SUCCESS) return fail(SLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(res));
+  return SLA_OK;
+}
+
+// [BH, N, D] activation map with a box of `rows` tokens x 64 channels.
+sla_status act_map(CUtensorMap* m, const void* ptr, const Shape& s, uint32_t rows) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.N), static_cast<uint64_t>(s.BH)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.N) * s.D};
+  const uint32_t box[3] = {64, rows, 1};
+  return make_map(m, ptr, 3, dims, strides, box);
+}
+
+// ------------------------------------------------------------------ launch helpers
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <typename K>
+sla_status allow_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return fail(SLA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  return SLA_OK;
+}
+
+sla_status launched(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SLA_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return SLA_OK;
+}
+
+#define SLA_TRY(x)                 \
+  do {                             \
+    sla_status st_ = (x);          \
+    if (st_ != SLA_OK) return st_; \
+  } while (0)
+
+template <int D>
+sla_status launch_pool(const void* x, double* out, const Shape& s, int block, int nblocks, cudaStream_t st) {
+  sla::pool_mean_kernel<D><<<dim3(nblocks, s.BH), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(x), out, s.N,
+                                                                  block, nblocks);
+  return launched("pool_mean_kernel");
+}
+
+template <int D>
+sla_status launch_kv_prep(const void* k, const void* v, const Shape& s, const KvPrepArgs& args, cudaStream_t st) {
+  CUtensorMap mk, mv;
+  SLA_TRY(act_map(&mk, k, s, 64));
+  SLA_TRY(act_map(&mv, v, s, 64));
+  const int smem = 4 * 16384 + 1024;
+  SLA_TRY(allow_smem(sla::kv_prep_kernel<D>, smem));
+  const int total = s.BH * s.Nk;
+  const int grid = total < 3 * sm_count() ? total : 3 * sm_count();
+  sla::kv_prep_kernel<D><<<grid, 128, smem, st>>>(mk, mv, args);
+  return launched("kv_prep_kernel");
+}
+
+template <int D>
+sla_status launch_scores(const double* qbar, const double* kbar, double* S, const Shape& s, cudaStream_t st) {
+  dim3 grid((s.Nk + 63) / 64, (s.Nq + 63) / 64, s.BH);
+  sla::score_kernel<D><<<grid, 256, 0, st>>>(qbar, kbar, S, s.Nq, s.Nk);
+  return launched("score_kernel");
+}
+
+sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
+  const size_t per_warp = static_cast<size_t>(a.Nk) * 8;
+  int wpc = static_cast<int>((200 * 1024) / per_warp);
+  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
+  const int smem = static_cast<int>(wpc * per_warp);
+  SLA_TRY(allow_smem(sla::select_kernel, smem));
+  const int grid = (a.rows + wpc - 1) / wpc;
+  sla::select_kernel<<<grid, wpc * 32, smem, st>>>(a);
+  return launched("select_kernel");
+}
+
+template <int D>
+sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
+  CUtensorMap mw, mh;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(s.w_ld), static_cast<uint64_t>(s.Nq) * s.w_ld};
+    const uint32_t box[3] = {64, 128, 1};
+    SLA_TRY(make_map(&mw, w.W, 3, dims, strides, box));
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.LD), static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.BH)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(s.LD), static_cast<uint64_t>(s.Nk) * s.LD};
+    const uint32_t box[3] = {64, 64, 1};
+    SLA_TRY(make_map(&mh, w.hst, 3, dims, strides, box));
+  }
+  const int smem = 2 * (16384 + 32768) + 1024;
+  SLA_TRY(allow_smem(sla::agg_kernel<D>, smem));
+  AggArgs a{s.Nq, s.Nk, s.LD, w.Hagg, w.Zagg, w.err};
+  dim3 grid((s.LD + 255) / 256, (s.Nq + 127) / 128, s.BH);
+  sla::agg_kernel<D><<<grid, 128, smem, st>>>(mw, mh, a);
+  return launched("agg_kernel");
+}
+
+template <int D>
+sla_status launch_attn(const Shape& s, const void* q, const void* k, const void* v, const float* alpha, void* out,
+                       const Workspace& w, int crit_ld, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mh, mo;
+  SLA_TRY(act_map(&mq, q, s, 128));
+  SLA_TRY(act_map(&mk, k, s, 64));
+  SLA_TRY(act_map(&mv, v, s, 64));
+  SLA_TRY(act_map(&mo, out, s, static_cast<uint32_t>(s.bq)));
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.BH) * s.Nq * s.D};
+    const uint64_t strides[1] = {static_cast<uint64_t>(s.D)};
+    const uint32_t box[2] = {64, 64};
+    SLA_TRY(make_map(&mh, w.Hagg, 2, dims, strides, box));
+  }
+  constexpr int smem = sla::AttnSmem<D>::template total<kAttnStages>();
+  SLA_TRY(allow_smem(sla::attn_kernel<D, kAttnStages>, smem));
+  AttnArgs a;
+  a.H = s.H;
+  a.N = s.N;
+  a.Nq = s.Nq;
+  a.block_q = s.bq;
+  a.crit = w.crit;
+  a.crit_ld = crit_ld;
+  a.crit_cnt = w.crit_cnt;
+  a.Zagg = w.Zagg;
+  a.alpha = alpha;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  a.err = w.err;
+  sla::attn_kernel<D, kAttnStages><<<dim3(s.Nq, s.BH), 192, smem, st>>>(mq, mk, mv, mh, mo, a);
+  return launched("attn_kernel");
+}
+
+// ------------------------------------------------------------------ entry points (templated on D)
+
+template <int D>
+sla_status route_impl(const Shape& s, const void* q, const void* k, int8_t* mask_out, int32_t* crit_out,
+                      double* scores_out, const Workspace& w, cudaStream_t st) {
+  SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
+  SLA_TRY(launch_pool<D>(k, w.kbar, s, s.bk, s.Nk, st));
+  double* S = scores_out ? scores_out : w.S;
+  SLA_TRY(launch_scores<D>(w.qbar, w.kbar, S, s, st));
+  SelectArgs a{};
+  a.S = S;
+  a.rows = s.BH * s.Nq;
+  a.Nk = s.Nk;
+  a.kc = s.kc;
+  a.kn = s.kn;
+  a.mask = mask_out;
+  a.crit = crit_out ? crit_out : w.crit;
+  a.crit_ld = crit_out ? s.kc : s.Nk;
+  a.crit_cnt = w.crit_cnt;
+  a.W = nullptr;
+  a.w_ld = s.w_ld;
+  return launch_select(a, st);
+}
+
+template <int D>
+sla_status forward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
+                        const int8_t* mask, void* out, const Workspace& w, cudaStream_t st) {
+  KvPrepArgs kv{};
+  kv.BH = s.BH;
+  kv.N = s.N;
+  kv.Nk = s.Nk;
+  kv.kbar = mask ? nullptr : w.kbar;
+  kv.hst = w.hst;
+  kv.LD = s.LD;
+  kv.err = w.err;
+  if (mask) {
+    SLA_TRY(launch_kv_prep<D>(k, v, s, kv, st));
+    MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
+    sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+    SLA_TRY(launched("mask_lists_kernel"));
+  } else {
+    SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
+    SLA_TRY(launch_kv_prep<D>(k, v, s, kv, st));
+    SLA_TRY(launch_scores<D>(w.qbar, w.kbar, w.S, s, st));
+    SelectArgs a{};
+    a.S = w.S;
+    a.rows = s.BH * s.Nq;
+    a.Nk = s.Nk;
+    a.kc = s.kc;
+    a.kn = s.kn;
+    a.mask = w.mask;
+    a.crit = w.crit;
+    a.crit_ld = s.Nk;
+    a.crit_cnt = w.crit_cnt;
+    a.W = w.W;
+    a.w_ld = s.w_ld;
+    SLA_TRY(launch_select(a, st));
+  }
+  SLA_TRY(launch_agg<D>(s, w, st));
+  return launch_attn<D>(s, q, k, v, alpha, out, w, s.Nk, st);
+}
+
+bool overlaps(const void* a, const void* b, size_t bytes) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bytes && y < x + bytes;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+sla_status sla_counts(const sla_problem* p, int* Nq, int* Nk, int* kc, int* kn) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (Nq) *Nq = s.Nq;
+  if (Nk) *Nk = s.Nk;
+  if (kc) *kc = s.kc;
+  if (kn) *kn = s.kn;
+  return SLA_OK;
+}
+
+size_t sla_workspace_size(const sla_problem* p) {
+  Shape s;
+  if (make_shape(p, &s) != SLA_OK) return 0;
+  return layout(s, nullptr).bytes;
+}
+
+sla_status sla_route(const sla_problem* p, const void* q, const void* k, int8_t* mask_out, int32_t* crit_idx_out,
+                     double* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(q) || !aligned16(k)) return fail(SLA_ERR_INVALID_ARG, "q and k must be non-NULL and 16-byte aligned");
+  if (!mask_out) return fail(SLA_ERR_INVALID_ARG, "mask_out is NULL");
+  if (crit_idx_out && (reinterpret_cast<uintptr_t>(crit_idx_out) % 4))
+    return fail(SLA_ERR_INVALID_ARG, "crit_idx_out must be 4-byte aligned");
+  if (scores_out && (reinterpret_cast<uintptr_t>(scores_out) % 8))
+    return fail(SLA_ERR_INVALID_ARG, "scores_out must be 8-byte aligned");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) return route_impl<64>(s, q, k, mask_out, crit_idx_out, scores_out, w, st);
+  return route_impl<128>(s, q, k, mask_out, crit_idx_out, scores_out, w, st);
+}
+
+sla_status sla_kv_states(const sla_problem* p, const void* k, const void* v, float* h_out, float* z_out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(k) || !aligned16(v)) return fail(SLA_ERR_INVALID_ARG, "k and v must be non-NULL and 16-byte aligned");
+  if (!aligned16(h_out) || !aligned16(z_out))
+    return fail(SLA_ERR_INVALID_ARG, "h_out and z_out must be non-NULL and 16-byte aligned");
+  uint32_t* err = nullptr;
+  if (ws) {
+    if (reinterpret_cast<uintptr_t>(ws) % 256 || ws_bytes < 256)
+      return fail(SLA_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold at least 256 bytes");
+    err = static_cast<uint32_t*>(ws);
+  }
+  KvPrepArgs kv{};
+  kv.BH = s.BH;
+  kv.N = s.N;
+  kv.Nk = s.Nk;
+  kv.h32 = h_out;
+  kv.z32 = z_out;
+  kv.LD = s.LD;
+  kv.err = err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) return launch_kv_prep<64>(k, v, s, kv, st);
+  return launch_kv_prep<128>(k, v, s, kv, st);
+}
+
+sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                       const int8_t* mask, void* out, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SLA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
+  if (!alpha || reinterpret_cast<uintptr_t>(alpha) % 4) return fail(SLA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
+  const size_t act = static_cast<size_t>(s.BH) * s.N * s.D * 2;
+  if (overlaps(out, q, act) || overlaps(out, k, act) || overlaps(out, v, act))
+    return fail(SLA_ERR_INVALID_ARG, "out must not alias q, k or v");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) return forward_impl<64>(s, q, k, v, alpha, mask, out, w, st);
+  return forward_impl<128>(s, q, k, v, alpha, mask, out, w, st);
+}
+
+sla_status sla_check(void* ws, void* stream) {
+  if (!ws) return fail(SLA_ERR_WORKSPACE, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  SLA_CUDA(cudaStreamSynchronize(st));
+  uint32_t word = 0;
+  SLA_CUDA(cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost));
+  if (word == 0) return SLA_OK;
+  const uint32_t zero = 0;
+  SLA_CUDA(cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice));
+  if (word & sla::SLA_DEVERR_TIMEOUT) return fail(SLA_ERR_TIMEOUT, "a device-side wait timed out (error word %u)", word);
+  return fail(SLA_ERR_BAD_MASK, "caller mask held a label outside {0,1,2} (error word %u)", word);
+}
+
+const char* sla_last_error(void) { return g_last_error.c_str(); }
+
+const char* sla_version(void) { return "sla-b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/sla.h declares, and its host logic (counts, argument
+checks, workspace sizing) behaves as documented."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from sparse_linear_attention_sla_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load_library()
+
+
+def _declared_symbols():
+    names = set()
+    for path in os.listdir(os.path.join(ROOT, "include")):
+        if path.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", path)).read()
+            names |= set(re.findall(r"^\s*(?:sla_status|size_t|const char\*)\s+(sla_\w+)\s*\(", text, re.M))
+    return names
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared_symbols() == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert lib.sla_version().decode().startswith("sla-b200")
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 2, 1024, 64, 64, 64, 0.25, 0.25),
+    (1, 12, 8192, 128, 128, 64, 0.10, 0.40),
+    (1, 12, 32760, 128, 128, 64, 0.05, 0.10),
+    (2, 40, 75600, 128, 128, 64, 0.05, 0.15),
+    (1, 12, 32700, 128, 128, 64, 0.05, 0.0),
+    (1, 12, 32760, 128, 128, 64, 1.0, 0.0),
+    (1, 1, 130 * 64, 64, 64, 64, 0.0, 0.1),
+    (1, 1, 1, 64, 64, 64, 0.5, 0.5),
+    (3, 5, 777, 128, 64, 64, 0.33, 0.33),
+])
+def test_counts_match_oracle(lib, shape):
+    B, H, N, D, bq, bk, kh, kl = shape
+    p = binding.problem(B, H, N, D, bq, bk, kh, kl)
+    # kh, kl pass through a C float: compare with the oracle at the same float value
+    f32 = lambda x: ctypes.c_float(x).value
+    assert binding.counts(p) == oracle.block_counts(N, bq, bk, f32(kh), f32(kl))
+    assert binding.workspace_size(p) > 0
+
+
+@pytest.mark.parametrize("bad, status", [
+    ((1, 1, 64, 96, 64, 64, 0.1, 0.1), 2),     # D unsupported
+    ((1, 1, 64, 64, 32, 64, 0.1, 0.1), 2),     # block_q unsupported
+    ((1, 1, 64, 64, 64, 128, 0.1, 0.1), 2),    # block_kv unsupported
+    ((0, 1, 64, 64, 64, 64, 0.1, 0.1), 1),     # B < 1
+    ((1, 1, 0, 64, 64, 64, 0.1, 0.1), 1),      # N < 1
+    ((1, 1, 64, 64, 64, 64, 0.7, 0.4), 1),     # kh + kl > 1
+    ((1, 1, 64, 64, 64, 64, -0.1, 0.0), 1),    # kh < 0
+    ((1, 1, 64, 64, 64, 64, float("nan"), 0.0), 1),
+    ((1, 1, 64 * 20000, 64, 64, 64, 0.1, 0.1), 2),  # too many KV blocks
+])
+def test_invalid_problems_rejected_on_host(lib, bad, status):
+    p = binding.problem(*bad)
+    with pytest.raises(binding.SlaError) as e:
+        binding.counts(p)
+    assert e.value.status == status
+    assert binding.workspace_size(p) == 0
+    assert lib.sla_last_error().decode()
+
+
+def test_entry_points_reject_bad_pointers_before_any_launch(lib):
+    p = binding.problem(1, 1, 128, 64, 64, 64, 0.25, 0.25)
+    null = ctypes.c_void_p(0)
+    # NULL / misaligned pointers and missing workspace are host-side errors (no CUDA call made)
+    assert lib.sla_forward(ctypes.byref(p), null, null, null, null, null, null, null, 0, null) == 1
+    assert lib.sla_route(ctypes.byref(p), null, null, null, null, null, null, 0, null) == 1
+    assert lib.sla_kv_states(ctypes.byref(p), null, null, null, null, null, 0, null) == 1
+    fake = ctypes.c_void_p(1 << 20)  # aligned but never dereferenced on the host
+    assert lib.sla_forward(ctypes.byref(p), fake, fake, fake, fake, null, ctypes.c_void_p(2 << 20), null, 0, null) == 3
+    assert lib.sla_forward(ctypes.byref(p), fake, fake, fake, fake, null, fake, ctypes.c_void_p(4 << 20), 0, null) == 1
+    small = binding.workspace_size(p) - 1
+    assert lib.sla_forward(ctypes.byref(p), fake, fake, fake, fake, null, ctypes.c_void_p(2 << 20),
+                           ctypes.c_void_p(8 << 20), small, null) == 3
+    assert lib.sla_check(null, null) == 3

@@ -1,0 +1,189 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Every input is seeded; the oracle sees exactly the bf16 tensors the kernels
+see. Labels must match bit for bit except near ties (counted and reported);
+outputs must match within max-abs 2e-2 and mean-abs 2e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_linear_attention_sla_b200 import binding
+from sparse_linear_attention_sla_b200.workloads import (SWEEP_KH, WORKLOADS, make_inputs, random_inputs,
+                                                        sweep_workload)
+from tests.parity_utils import assert_outputs_close, label_mismatches
+
+pytestmark = pytest.mark.gpu
+
+
+def _to_cpu(*ts):
+    return [t.detach().cpu() for t in ts]
+
+
+def _route_parity(q, k, bq, kh, kl, heads=None):
+    """GPU router vs oracle on the given heads: labels (near-tie rule), scores, crit lists.
+
+    Returns (gpu_mask, oracle_mask, mismatches). oracle_mask holds the oracle's
+    labels on the checked heads and the GPU's labels elsewhere.
+    """
+    mask, crit, scores = binding.route(q, k, bq, 64, kh, kl, want_scores=True, want_crit=True)
+    B, H, N, D = q.shape
+    p = binding.problem(B, H, N, D, bq, 64, kh, kl)
+    Nq, Nk, kc, kn = binding.counts(p)
+    heads = heads or [(b, h) for b in range(B) for h in range(H)]
+    gm, gs, gc = mask.cpu().numpy(), scores.cpu().numpy(), crit.cpu().numpy()
+    om = gm.copy()
+    worst_rel = 0.0
+    total = excused = 0
+    for b, h in heads:
+        rm, S = oracle.route(q[b, h].cpu(), k[b, h].cpu(), bq, 64, kh, kl)
+        om[b, h] = rm
+        rel = np.abs(gs[b, h] - S).max() / max(np.abs(S).max(), 1e-300)
+        worst_rel = max(worst_rel, rel)
+        t, e = label_mismatches(gm[b, h], rm, S, kc, kn)
+        total += t
+        excused += e
+        # the critical list is the ascending index list of the GPU's own critical labels
+        for i in range(Nq):
+            np.testing.assert_array_equal(gc[b, h, i], np.nonzero(gm[b, h, i] == 2)[0])
+        assert np.all((gm[b, h] == 2).sum(-1) == kc) and np.all((gm[b, h] == 0).sum(-1) == kn)
+    assert worst_rel < 1e-12, f"scores differ from the oracle by {worst_rel:.2e} (relative)"
+    assert total == excused, f"{total - excused} label mismatches outside near ties ({total} total)"
+    if total:
+        print(f"near-tie label mismatches (excused): {total}")
+    return mask, torch.from_numpy(om).to(q.device), total
+
+
+def _oracle_rows(q, k, v, alpha, bq, mask, heads, query_blocks=None):
+    """Oracle output for the sampled heads (NaN elsewhere), one head at a time."""
+    B, H, N, D = q.shape
+    ref = np.full((B, H, N, D), np.nan)
+    m = mask.cpu().numpy()
+    for b, h in heads:
+        o = oracle.forward(q[b, h][None, None].cpu(), k[b, h][None, None].cpu(), v[b, h][None, None].cpu(),
+                           alpha[h][None].cpu(), bq, 64, mask=m[b, h][None, None], query_blocks=query_blocks)
+        ref[b, h] = o[0, 0]
+    return ref
+
+
+CASES = [
+    # B, H, N, D, bq, kh, kl
+    (1, 2, 1024, 64, 64, 0.25, 0.25),
+    (1, 1, 200, 64, 64, 0.3, 0.2),
+    (2, 2, 333, 128, 128, 0.2, 0.3),
+    (1, 3, 4113, 128, 128, 0.1, 0.2),
+    (1, 2, 700, 128, 64, 0.25, 0.25),
+    (1, 2, 129, 64, 128, 0.5, 0.25),
+    (1, 2, 1000, 128, 128, 1.0, 0.0),   # every block critical: dense softmax attention
+    (1, 2, 1000, 128, 128, 0.0, 0.0),   # no critical, no negligible: pure linear attention
+    (1, 2, 1000, 128, 128, 0.0, 0.5),   # empty sparse branch
+    (1, 2, 1000, 128, 128, 0.5, 0.5),   # empty linear branch
+    (1, 1, 64, 128, 128, 0.5, 0.0),     # a single KV block
+    (1, 1, 1, 64, 64, 1.0, 0.0),        # a single token
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(map(str, c)))
+def test_forward_matches_oracle(cuda_device, case):
+    B, H, N, D, bq, kh, kl = case
+    q, k, v, alpha = random_inputs(B, H, N, D, seed=sum(case[:5]), device=cuda_device)
+    gmask, omask, nmis = _route_parity(q, k, bq, kh, kl)
+    ws = binding.new_workspace(binding.problem(B, H, N, D, bq, 64, kh, kl), cuda_device)
+    out = binding.forward(q, k, v, alpha, bq, 64, kh, kl, ws=ws)          # internal router
+    out_m = binding.forward(q, k, v, alpha, bq, 64, kh, kl, mask=omask, ws=ws)  # oracle's labels
+    binding.check(ws)
+    heads = [(b, h) for b in range(B) for h in range(H)]
+    ref = _oracle_rows(q, k, v, alpha, bq, omask, heads)
+    assert_outputs_close(out_m.float().cpu().numpy(), ref, f"oracle labels {case}")
+    if nmis == 0:
+        assert torch.equal(out, out_m), "router path and caller-mask path disagree on the same labels"
+
+
+def test_kv_states_match_oracle(cuda_device):
+    for (B, H, N, D) in [(1, 2, 1024, 64), (1, 2, 333, 128), (2, 1, 4096 + 7, 128)]:
+        q, k, v, _ = random_inputs(B, H, N, D, seed=N, device=cuda_device)
+        h, z = binding.kv_states(k, v)
+        kc_, vc = _to_cpu(k, v)
+        rh, rz = oracle.kv_states(kc_, vc, 64)
+        # phi(k) enters the tensor core in bf16 (relative rounding 2^-9) with fp32 accumulation
+        scale_h = np.abs(rh).max()
+        assert np.abs(h.cpu().numpy() - rh).max() <= 8e-3 * scale_h
+        np.testing.assert_allclose(z.cpu().numpy(), rz, rtol=1e-5, atol=1e-4)
+
+
+def _workload_parity(w, device, heads=None, query_blocks=None, gen_device="cpu"):
+    q, k, v, alpha = make_inputs(w, device=gen_device)
+    q, k, v, alpha = (t.to(device) for t in (q, k, v, alpha))
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    gmask, omask, nmis = _route_parity(q, k, w.block_q, w.kh, w.kl, heads=heads)
+    ws = binding.new_workspace(binding.problem(w.B, w.H, w.N, w.D, w.block_q, 64, w.kh, w.kl), device)
+    out = binding.forward(q, k, v, alpha, w.block_q, 64, w.kh, w.kl, ws=ws)
+    out_m = binding.forward(q, k, v, alpha, w.block_q, 64, w.kh, w.kl, mask=omask, ws=ws)
+    binding.check(ws)
+    ref = _oracle_rows(q, k, v, alpha, w.block_q, omask, heads, query_blocks)
+    err = assert_outputs_close(out_m.float().cpu().numpy(), ref, w.name)
+    if nmis == 0:
+        assert torch.equal(out, out_m)
+    print(f"{w.name}: max-abs {err[0]:.3e} mean-abs {err[1]:.3e} near-tie mismatches {nmis}")
+    return err, nmis
+
+
+def test_iid_b1h2_n1024_d64(cuda_device):
+    _workload_parity(WORKLOADS["iid_b1h2_n1024_d64"], cuda_device)
+
+
+def test_field1d_b1h12_n8192_d128(cuda_device):
+    _workload_parity(WORKLOADS["field1d_b1h12_n8192_d128"], cuda_device)
+
+
+def test_wan13b_b1h12_n32760_d128(cuda_device):
+    _workload_parity(WORKLOADS["wan13b_b1h12_n32760_d128"], cuda_device)
+
+
+def test_wan14b720p_sampled(cuda_device):
+    w = WORKLOADS["wan14b720p_b2h40_n75600_d128"]
+    Nq = -(-w.N // w.block_q)
+    rng = np.random.default_rng(4)
+    heads = [(0, 0), (1, 39)] + [(int(rng.integers(2)), int(rng.integers(40))) for _ in range(2)]
+    qbs = sorted({0, Nq - 1, *[int(x) for x in rng.integers(1, Nq - 1, size=6)]})
+    _workload_parity(w, cuda_device, heads=heads, query_blocks=qbs, gen_device=cuda_device)
+
+
+@pytest.mark.parametrize("kh", SWEEP_KH)
+def test_sparsity_sweep_sampled(cuda_device, kh):
+    w = sweep_workload(kh)
+    _workload_parity(w, cuda_device, heads=[(0, 0), (0, 11)], query_blocks=[0, 1, 77, 128, 200, 255])
+
+
+def test_sparsity_sweep_tail_n32700(cuda_device):
+    w = sweep_workload(0.05, N=32700)
+    _workload_parity(w, cuda_device, heads=[(0, 3)], query_blocks=[0, 100, 254, 255])
+
+
+def test_output_invariants(cuda_device):
+    q, k, v, alpha = random_inputs(1, 2, 2000, 128, seed=9, device=cuda_device)
+    o1 = binding.forward(q, k, v, alpha, 128, 64, 0.2, 0.2)
+    o2 = binding.forward(q, k, v, alpha, 128, 64, 0.2, 0.2)
+    assert torch.equal(o1, o2), "forward is not deterministic"
+    vf = v.float()
+    lo, hi = vf.amin(dim=2, keepdim=True), vf.amax(dim=2, keepdim=True)
+    o = o1.float()
+    slack = 1e-2 * (hi - lo)
+    assert bool(((o >= lo - slack) & (o <= hi + slack)).all()), "output outside the per-channel V range"
+    # V -> 2 V + 1 gives O -> 2 O + 1 (both branches are normalised averages of V rows)
+    o3 = binding.forward(q, k, (2 * vf + 1).to(torch.bfloat16), alpha, 128, 64, 0.2, 0.2).float()
+    assert (o3 - (2 * o + 1)).abs().max().item() < 6e-2
+
+
+def test_bad_caller_mask_is_reported(cuda_device):
+    q, k, v, alpha = random_inputs(1, 1, 256, 64, seed=3, device=cuda_device)
+    mask = torch.ones(1, 1, 4, 4, dtype=torch.int8, device=cuda_device)
+    mask[0, 0, 1, 2] = 3
+    ws = binding.new_workspace(binding.problem(1, 1, 256, 64, 64, 64), cuda_device)
+    binding.forward(q, k, v, alpha, 64, 64, 0.0, 0.0, mask=mask, ws=ws)
+    with pytest.raises(binding.SlaError) as e:
+        binding.check(ws)
+    assert e.value.status == 6
+    binding.check(ws)  # the error word was cleared
