@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the fused SLA forward (sla_forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one sla_forward call (router, KV states, aggregation, fused
+attention) over one batch of seeded synthetic inputs already resident in HBM.
+L2 is flushed (512 MiB write, untimed) before every call; each call is timed
+with CUDA events on the launching stream. Rank 0 prints one JSON line.
+
+With --gpus N > 1 (launched by torch.distributed.run) every rank runs its own
+replica of the workload on its own GPU (the heads of a batch are independent
+problems, so there is no data-path collective); the step time is the maximum
+over ranks and the value counts the work of all ranks ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle on the host cores instead (rank 0
+only), one head of the workload per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective attention TFLOPS and ms/call at 1 B200; fraction of roofline"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "wan13b_b1h12_n32760_d128"
+FLUSH_BYTES = 512 << 20
+LAUNCHES_PER_FORWARD = 6  # pool, kv_prep, scores, select, aggregate, attention
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+# ---------------------------------------------------------------- peaks and work accounting
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def dense_equivalent_flops(w):
+    return 4.0 * w.B * w.H * float(w.N) ** 2 * w.D
+
+
+def algorithmic_work(w, mask):
+    """Algorithmic FLOPs and bytes of one forward (no recomputation or padding credited).
+
+    mask: [B,H,Nq,Nk] int8 labels actually used. Sparse FLOPs count the valid
+    query rows and keys of every critical (query block, KV block) pair.
+    """
+    import torch
+
+    B, H, N, D = w.B, w.H, w.N, w.D
+    BH = B * H
+    Nq, Nk = mask.shape[-2], mask.shape[-1]
+    qsize = torch.clamp(N - torch.arange(Nq, device=mask.device) * w.block_q, max=w.block_q).double()
+    ksize = torch.clamp(N - torch.arange(Nk, device=mask.device) * w.block_kv, max=w.block_kv).double()
+    crit = (mask == 2).double().reshape(BH, Nq, Nk)
+    pairs = torch.einsum("i,bij,j->", qsize, crit, ksize).item()
+    marg = (mask == 1).sum(-1).double().reshape(BH, Nq)
+    nonmarg = Nk - marg
+    f_sparse = 4.0 * D * pairs
+    f_states = 2.0 * N * D * D * BH
+    f_apply = 2.0 * N * D * D * BH
+    f_agg = float(torch.minimum(marg, nonmarg).sum().item()) * D * D
+    f_router = 2.0 * (N * D + Nq * Nk * D) * BH
+    f_elem = 3.0 * N * D * BH
+    f_alg = f_sparse + f_states + f_apply + f_agg + f_router + f_elem
+    bytes_alg = 8.0 * N * D * BH + Nq * Nk * BH + H * D * 4
+    return {"flops": f_alg, "bytes": bytes_alg, "f_sparse": f_sparse, "f_attn_kernel": f_sparse + f_apply,
+            "f_states": f_states, "f_agg": f_agg, "f_router": f_router}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    for name in ("attention.cuh", "sm100.cuh"):
+        with open(os.path.join(ROOT, "sparse_linear_attention_sla_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per attention-kernel launch from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_sha") != kernel_source_sha() or t.get("workload") != workload:
+        return None
+    return float(t["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock, power and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="sla_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                                 "hw_slowdown": parts[5], "hw_thermal_slowdown": parts[6],
+                                 "sw_thermal_slowdown": parts[7], "sw_power_cap": parts[8]})
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 250.0] or rows
+        reasons = sorted({k for r in loaded for k in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                                          "sw_power_cap") if r[k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+
+def cpu_oracle_sample(w, target_s, max_heads=None):
+    """Time the fp64 oracle (as it stands) on whole heads of w until ~target_s seconds have passed.
+
+    Returns (effective TFLOP/s, seconds, heads, threads)."""
+    import torch
+
+    import oracle
+    from sparse_linear_attention_sla_b200.workloads import make_inputs
+
+    try:
+        import threadpoolctl
+
+        threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) or 1
+    except Exception:  # noqa: BLE001 - thread count is informational
+        threads = os.cpu_count() or 1
+    q, k, v, alpha = make_inputs(w, device="cpu")
+    per_head = 4.0 * float(w.N) ** 2 * w.D
+    done, spent = 0, 0.0
+    limit = max_heads or w.B * w.H
+    for bh in range(limit):
+        b, h = divmod(bh, w.H)
+        t0 = time.perf_counter()
+        oracle.forward(q[b, h][None, None], k[b, h][None, None], v[b, h][None, None], alpha[h][None],
+                       w.block_q, w.block_kv, w.kh, w.kl)
+        spent += time.perf_counter() - t0
+        done += 1
+        if spent >= target_s:
+            break
+    del torch
+    return per_head * done / spent / 1e12, spent, done, threads
+
+
+# ---------------------------------------------------------------- our arm
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from sparse_linear_attention_sla_b200 import binding
+    from sparse_linear_attention_sla_b200.workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = WORKLOADS[args.workload]
+    q, k, v, alpha = make_inputs(w, device=dev)
+    p = binding.problem(w.B, w.H, w.N, w.D, w.block_q, w.block_kv, w.kh, w.kl)
+    ws = binding.new_workspace(p, dev)
+    out = torch.empty_like(q)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step_timed():
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        _, stages = binding.forward_timed(q, k, v, alpha, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=ws)
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1), stages
+
+    for _ in range(args.warmup):
+        step_timed()
+    binding.check(ws)
+
+    barrier()
+    torch.cuda.synchronize(dev)
+    per_step, stage_sum = [], [0.0] * 4
+    with ClockSampler(local) as clocks:
+        wall0 = time.perf_counter()
+        for _ in range(args.steps):
+            ms, stages = step_timed()
+            per_step.append(ms)
+            stage_sum = [a + b for a, b in zip(stage_sum, stages)]
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    barrier()
+    binding.check(ws)
+    clock_info = clocks.summary()
+
+    ms_local = sum(per_step) / len(per_step)
+    ms_step = max_over_ranks(ms_local)
+    stage_ms = [s / args.steps for s in stage_sum]
+    attn_ms = max_over_ranks(stage_ms[3])
+
+    # labels actually used, for the work accounting
+    mask, _, _ = binding.route(q, k, w.block_q, w.block_kv, w.kh, w.kl)
+    work = algorithmic_work(w, mask)
+    del mask
+    peaks = measured_peaks()
+    eff_flops = dense_equivalent_flops(w)
+    value = world * eff_flops / (ms_step * 1e-3) / 1e12
+
+    # dominant kernel: the fused attention (stage 3)
+    achieved = work["f_attn_kernel"] / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": f"attn_kernel<{w.D},3>", "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+                else "fallback 1590 TFLOP/s", "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                "kernel_ms": round(attn_ms, 4), "kernel_flops_per_launch": work["f_attn_kernel"],
+                "traffic": recorded_traffic(w.name)}
+    t_roof = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    path_roofline = {"t_roof_us": round(t_roof * 1e6, 2), "t_us": round(ms_step * 1e3, 2),
+                     "frac": round(t_roof / (ms_step * 1e-3), 4), "flops_alg": work["flops"],
+                     "bytes_alg": work["bytes"], "executed_tflops": round(work["flops"] / (ms_step * 1e-3) / 1e12, 2)}
+
+    # end to end through the public call with host buffers (copies inside the timed region)
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ha = alpha.cpu().pin_memory()
+        hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        dq, dk, dv, da = (torch.empty_like(t) for t in (q, k, v, alpha))
+
+        def e2e_step():
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            da.copy_(ha, non_blocking=True)
+            binding.forward(dq, dk, dv, da, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=ws)
+            hout.copy_(out, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier()
+        ms_e2e = max_over_ranks(sum(e2e_step() for _ in range(args.steps)) / args.steps)
+        barrier()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha))
+        e2e = {"value": round(world * eff_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": UNIT,
+               "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+        del hq, hk, hv, ha, hout, dq, dk, dv, da
+        binding.check(ws)
+
+    # the same kernel at kh = 100%: dense-attention reference on the same inputs
+    dense = None
+    if not args.no_dense:
+        wd = w.with_(kh=1.0, kl=0.0)
+        pd = binding.problem(w.B, w.H, w.N, w.D, w.block_q, w.block_kv, 1.0, 0.0)
+        wsd = binding.new_workspace(pd, dev)
+        times, attn_d = [], []
+        for it in range(3 + 5):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            _, st_d = binding.forward_timed(q, k, v, alpha, w.block_q, w.block_kv, 1.0, 0.0, out=out, ws=wsd)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+                attn_d.append(st_d[3])
+        binding.check(wsd)
+        ms_d = max_over_ranks(sum(times) / len(times))
+        dense = {"workload": wd.name + "_kh1", "ms_per_call": round(ms_d, 4),
+                 "effective_tflops": round(eff_flops / (ms_d * 1e-3) / 1e12, 2),
+                 "attn_kernel_ms": round(sum(attn_d) / len(attn_d), 4),
+                 "speedup_of_sparse_over_dense": round(ms_d / ms_step, 3)}
+        del wsd
+
+    cpu = None
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        tf, spent, heads, threads = cpu_oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": round(tf, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"fp64 oracle on {heads} of {w.B * w.H} heads of {w.name} (all {math.ceil(w.N / w.block_q)} "
+                         f"query blocks each: router, states, both branches), {spent:.1f} s"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "block_q": w.block_q,
+                   "block_kv": w.block_kv, "kh": w.kh, "kl": w.kl, "inputs": w.kind,
+                   "l2": "flushed before every call (512 MiB write, untimed)",
+                   "parallelism": "one replica per GPU" if world > 1 else "single GPU"},
+        "stage_ms": {"precompute": round(stage_ms[0], 4), "route": round(stage_ms[1], 4),
+                     "aggregate": round(stage_ms[2], 4), "attention": round(stage_ms[3], 4)},
+        "roofline": roofline, "path_roofline": path_roofline,
+        "clocks": clock_info, "e2e": e2e, "gpu_launches": LAUNCHES_PER_FORWARD * args.steps,
+        "dense_reference": dense, "cpu_baseline": cpu,
+        "wall_s_timed": round(wall, 3),
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import torch
+
+    import oracle
+    from sparse_linear_attention_sla_b200.workloads import WORKLOADS, make_inputs
+
+    try:
+        import threadpoolctl
+
+        threads = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()) or 1
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count() or 1
+    w = WORKLOADS[args.workload]
+    q, k, v, alpha = make_inputs(w, device="cpu")
+    per_head = 4.0 * float(w.N) ** 2 * w.D
+
+    def one(step):
+        bh = step % (w.B * w.H)
+        b, h = divmod(bh, w.H)
+        t0 = time.perf_counter()
+        oracle.forward(q[b, h][None, None], k[b, h][None, None], v[b, h][None, None], alpha[h][None],
+                       w.block_q, w.block_kv, w.kh, w.kl)
+        return time.perf_counter() - t0
+
+    for s in range(args.warmup):
+        one(s)
+    times = [one(args.warmup + s) for s in range(args.steps)]
+    sec = sum(times) / len(times)
+    value = per_head / sec / 1e12
+    del torch
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D, "block_q": w.block_q,
+                   "block_kv": w.block_kv, "kh": w.kh, "kl": w.kl, "inputs": w.kind,
+                   "step": "one head, all query blocks"},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"one of {w.B * w.H} heads of {w.name} per step (router, states, both branches)"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return line
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -108,6 +108,15 @@ sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const
                        const float* alpha, const int8_t* mask, void* out, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* sla_forward plus per-stage device times. Records CUDA events on the stream
+ * between the stages, waits for the last one, and writes stage_ms[4] (host):
+ * [0] per-block precompute (pooling, KV states), [1] routing (scores and
+ * selection, or the caller-mask lists), [2] marginal-state aggregation,
+ * [3] fused attention. Synchronises the stream; meant for measurement. */
+sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k, const void* v,
+                             const float* alpha, const int8_t* mask, void* out, void* ws,
+                             size_t ws_bytes, void* stream, float* stage_ms);
+
 /* Synchronise the stream, read and clear the workspace's device error word.
  * Returns SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_BAD_MASK (or SLA_ERR_CUDA). */
 sla_status sla_check(void* ws, void* stream);

@@ -27,7 +27,7 @@ _STATUS = {
 
 # Every symbol include/sla.h declares.
 EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sla_forward",
-           "sla_check", "sla_last_error", "sla_version")
+           "sla_forward_timed", "sla_check", "sla_last_error", "sla_version")
 
 
 class SlaError(RuntimeError):
@@ -66,10 +66,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_route.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_kv_states.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_forward_timed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(ctypes.c_float)]
         lib.sla_check.argtypes = [vp, vp]
         lib.sla_last_error.restype = ctypes.c_char_p
         lib.sla_version.restype = ctypes.c_char_p
-        for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_check"):
+        for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -167,8 +168,7 @@ def kv_states(k, v, block_kv=64, ws=None):
     return h, z
 
 
-def forward(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, out=None, ws=None):
-    """Fused SLA forward: O = alpha * O_s + (1 - alpha) * O_l, bf16 [B,H,N,D]."""
+def _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws):
     B, H, N, D = q.shape
     dev = q.device
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -187,12 +187,32 @@ def forward(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=Non
         _check_act("out", out, B, H, N, D, dev)
     if ws is None:
         ws = new_workspace(p, dev)
+    return p, out, ws
+
+
+def forward(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, out=None, ws=None):
+    """Fused SLA forward: O = alpha * O_s + (1 - alpha) * O_l, bf16 [B,H,N,D]."""
+    p, out, ws = _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws)
     lib = load_library()
-    with torch.cuda.device(dev):
+    with torch.cuda.device(q.device):
         st = lib.sla_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(mask), _ptr(out),
-                             _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+                             _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(q.device))
     _raise(st)
     return out
+
+
+def forward_timed(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, out=None, ws=None):
+    """forward() plus per-stage device milliseconds (precompute, route, aggregate, attention).
+
+    Synchronises the current stream."""
+    p, out, ws = _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws)
+    ms = (ctypes.c_float * 4)()
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        st = lib.sla_forward_timed(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(mask), _ptr(out),
+                                   _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(q.device), ms)
+    _raise(st)
+    return out, [float(x) for x in ms]
 
 
 def check(ws: torch.Tensor):

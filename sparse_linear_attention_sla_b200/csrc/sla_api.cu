@@ -326,9 +326,22 @@ sla_status route_impl(const Shape& s, const void* q, const void* k, int8_t* mask
   return launch_select(a, st);
 }
 
+// Stage boundaries for sla_forward_timed: ev[0] before the per-block precompute,
+// ev[1] after it, ev[2] after routing, ev[3] after aggregation, ev[4] after attention.
+struct StageEvents {
+  cudaEvent_t ev[5];
+  bool on;
+  sla_status mark(int i, cudaStream_t st) {
+    if (!on) return SLA_OK;
+    cudaError_t e = cudaEventRecord(ev[i], st);
+    if (e != cudaSuccess) return fail(SLA_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
+    return SLA_OK;
+  }
+};
+
 template <int D>
 sla_status forward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
-                        const int8_t* mask, void* out, const Workspace& w, cudaStream_t st) {
+                        const int8_t* mask, void* out, const Workspace& w, cudaStream_t st, StageEvents& ev) {
   KvPrepArgs kv{};
   kv.BH = s.BH;
   kv.N = s.N;
@@ -337,14 +350,17 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
   kv.hst = w.hst;
   kv.LD = s.LD;
   kv.err = w.err;
+  SLA_TRY(ev.mark(0, st));
   if (mask) {
     SLA_TRY(launch_kv_prep<D>(k, v, s, kv, st));
+    SLA_TRY(ev.mark(1, st));
     MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
     sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
     SLA_TRY(launched("mask_lists_kernel"));
   } else {
     SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
     SLA_TRY(launch_kv_prep<D>(k, v, s, kv, st));
+    SLA_TRY(ev.mark(1, st));
     SLA_TRY(launch_scores<D>(w.qbar, w.kbar, w.S, s, st));
     SelectArgs a{};
     a.S = w.S;
@@ -360,13 +376,37 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
     a.w_ld = s.w_ld;
     SLA_TRY(launch_select(a, st));
   }
+  SLA_TRY(ev.mark(2, st));
   SLA_TRY(launch_agg<D>(s, w, st));
-  return launch_attn<D>(s, q, k, v, alpha, out, w, s.Nk, st);
+  SLA_TRY(ev.mark(3, st));
+  SLA_TRY(launch_attn<D>(s, q, k, v, alpha, out, w, s.Nk, st));
+  return ev.mark(4, st);
 }
+
+sla_status forward_checked(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                           const int8_t* mask, void* out, void* ws, size_t ws_bytes, cudaStream_t st,
+                           StageEvents& ev);
 
 bool overlaps(const void* a, const void* b, size_t bytes) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + bytes && y < x + bytes;
+}
+
+sla_status forward_checked(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                           const int8_t* mask, void* out, void* ws, size_t ws_bytes, cudaStream_t st,
+                           StageEvents& ev) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SLA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
+  if (!alpha || reinterpret_cast<uintptr_t>(alpha) % 4) return fail(SLA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
+  const size_t act = static_cast<size_t>(s.BH) * s.N * s.D * 2;
+  if (overlaps(out, q, act) || overlaps(out, k, act) || overlaps(out, v, act))
+    return fail(SLA_ERR_INVALID_ARG, "out must not alias q, k or v");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  if (s.D == 64) return forward_impl<64>(s, q, k, v, alpha, mask, out, w, st, ev);
+  return forward_impl<128>(s, q, k, v, alpha, mask, out, w, st, ev);
 }
 
 }  // namespace
@@ -436,19 +476,33 @@ sla_status sla_kv_states(const sla_problem* p, const void* k, const void* v, flo
 
 sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
                        const int8_t* mask, void* out, void* ws, size_t ws_bytes, void* stream) {
-  Shape s;
-  SLA_TRY(make_shape(p, &s));
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return fail(SLA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
-  if (!alpha || reinterpret_cast<uintptr_t>(alpha) % 4) return fail(SLA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
-  const size_t act = static_cast<size_t>(s.BH) * s.N * s.D * 2;
-  if (overlaps(out, q, act) || overlaps(out, k, act) || overlaps(out, v, act))
-    return fail(SLA_ERR_INVALID_ARG, "out must not alias q, k or v");
-  Workspace w;
-  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  StageEvents ev{};
+  ev.on = false;
+  return forward_checked(p, q, k, v, alpha, mask, out, ws, ws_bytes, static_cast<cudaStream_t>(stream), ev);
+}
+
+sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                             const int8_t* mask, void* out, void* ws, size_t ws_bytes, void* stream,
+                             float* stage_ms) {
+  if (!stage_ms) return fail(SLA_ERR_INVALID_ARG, "stage_ms is NULL");
+  StageEvents ev{};
+  ev.on = true;
+  for (int i = 0; i < 5; ++i) {
+    cudaError_t e = cudaEventCreate(&ev.ev[i]);
+    if (e != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev.ev[j]);
+      return fail(SLA_ERR_CUDA, "cudaEventCreate: %s", cudaGetErrorString(e));
+    }
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (s.D == 64) return forward_impl<64>(s, q, k, v, alpha, mask, out, w, st);
-  return forward_impl<128>(s, q, k, v, alpha, mask, out, w, st);
+  sla_status rc = forward_checked(p, q, k, v, alpha, mask, out, ws, ws_bytes, st, ev);
+  if (rc == SLA_OK) {
+    cudaError_t e = cudaEventSynchronize(ev.ev[4]);
+    for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&stage_ms[i], ev.ev[i], ev.ev[i + 1]);
+    if (e != cudaSuccess) rc = fail(SLA_ERR_CUDA, "timing events: %s", cudaGetErrorString(e));
+  }
+  for (int i = 0; i < 5; ++i) cudaEventDestroy(ev.ev[i]);
+  return rc;
 }
 
 sla_status sla_check(void* ws, void* stream) {
