@@ -26,9 +26,10 @@
  *   O               alpha[h, :] * O_s + (1 - alpha[h, :]) * O_l
  *
  * Conventions (all entry points):
- *   - Tensors are device pointers owned by the caller; the library allocates
- *     no device memory. Q, K, V and O are [B, H, N, D] bf16, contiguous, D
- *     fastest, 16-byte aligned. alpha is [H, D] fp32.
+ *   - Tensors are device pointers owned by the caller; no entry point allocates
+ *     device memory (the only library-owned device memory is the fixed scratch
+ *     array of sla_route_noalloc, part of the loaded module). Q, K, V and O are
+ *     [B, H, N, D] bf16, contiguous, D fastest, 16-byte aligned. alpha is [H, D] fp32.
  *   - Supported: D in {64, 128}; block_q in {64, 128}; block_kv = 64;
  *     1 <= N; Nk = ceil(N / 64) <= 16384; 0 <= kh, kl and kh + kl <= 1.
  *   - Work is enqueued on the caller's stream; calls return before it runs.
@@ -120,6 +121,31 @@ sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k,
 /* Synchronise the stream, read and clear the workspace's device error word.
  * Returns SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_BAD_MASK (or SLA_ERR_CUDA). */
 sla_status sla_check(void* ws, void* stream);
+
+/* The block router for callers that cannot allocate device memory.
+ *
+ * There is no counterpart on the pages: this is a deployment variant of
+ * sla_route. Some callers may not call cudaMalloc or hand the library an extra
+ * buffer: a plugin running inside an inference server or graph runtime that owns
+ * every byte of device memory, or a real-time loop with a fixed memory budget.
+ * This entry point takes the same inputs and outputs as sla_route but no
+ * workspace; its scratch is a 32 MiB array compiled into the library, which every
+ * GPU that loads the library holds until the process exits.
+ *   q, k, mask_out, crit_idx_out, scores_out   as for sla_route
+ *   stream                                     cudaStream_t
+ * Limits and behaviour:
+ *   - The scratch holds the pooled means, plus the scores when scores_out is NULL
+ *     and the critical lists when crit_idx_out is NULL. A problem that needs more
+ *     than 32 MiB is rejected with SLA_ERR_WORKSPACE before anything is enqueued
+ *     (the Wan2.1-1.3B shape B=1, H=12, N=32760, D=128 fits with both outputs NULL).
+ *   - The library allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *     routine). The first call on each device looks up the array's device address
+ *     with that device current; make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents. Calls
+ *     whose work overlaps on the GPU (other streams, other host threads) race on it
+ *     and must be ordered by the caller. */
+sla_status sla_route_noalloc(const sla_problem* p, const void* q, const void* k, int8_t* mask_out,
+                             int32_t* crit_idx_out, double* scores_out, void* stream);
 
 /* Message for the calling thread's most recent failed call ("" if none). */
 const char* sla_last_error(void);

@@ -27,7 +27,7 @@ _STATUS = {
 
 # Every symbol include/sla.h declares.
 EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sla_forward",
-           "sla_forward_timed", "sla_check", "sla_last_error", "sla_version")
+           "sla_forward_timed", "sla_check", "sla_last_error", "sla_version", "sla_route_noalloc")
 
 
 class SlaError(RuntimeError):

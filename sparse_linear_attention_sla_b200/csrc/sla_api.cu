@@ -523,3 +523,78 @@ const char* sla_last_error(void) { return g_last_error.c_str(); }
 const char* sla_version(void) { return "sla-b200 0.1.0 (sm_100a)"; }
 
 }  // extern "C"
+
+// ====================================================================== router without caller scratch
+//
+// sla_route_noalloc: the router for callers that cannot allocate device memory
+// themselves. Its scratch (pooled means, and the scores and critical lists when
+// the caller does not ask for them) lives in the file-scope array below instead
+// of a caller workspace. Every GPU that loads this library holds the array
+// until the process exits.
+
+namespace {
+
+constexpr size_t kRouteScratchBytes = size_t(32) << 20;  // 32 MiB
+__device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_route_scratch_mu;
+void* g_route_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_route_scratch on the current device. Looked up once per
+// device (with that device current) on its first use; host code must never
+// pass the array's name itself to a kernel, only this address.
+sla_status route_scratch_address(void** out) {
+  int dev = 0;
+  SLA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
+  if (!g_route_scratch_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(SLA_ERR_CUDA, "cudaGetSymbolAddress(route scratch): %s", cudaGetErrorString(e));
+    g_route_scratch_addr[dev] = p;
+  }
+  *out = g_route_scratch_addr[dev];
+  return SLA_OK;
+}
+
+}  // namespace
+
+extern "C" sla_status sla_route_noalloc(const sla_problem* p, const void* q, const void* k, int8_t* mask_out,
+                                         int32_t* crit_idx_out, double* scores_out, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(q) || !aligned16(k)) return fail(SLA_ERR_INVALID_ARG, "q and k must be non-NULL and 16-byte aligned");
+  if (!mask_out) return fail(SLA_ERR_INVALID_ARG, "mask_out is NULL");
+  if (crit_idx_out && (reinterpret_cast<uintptr_t>(crit_idx_out) % 4))
+    return fail(SLA_ERR_INVALID_ARG, "crit_idx_out must be 4-byte aligned");
+  if (scores_out && (reinterpret_cast<uintptr_t>(scores_out) % 8))
+    return fail(SLA_ERR_INVALID_ARG, "scores_out must be 8-byte aligned");
+  // Scratch layout inside the static array (256-byte aligned pieces).
+  const size_t BH = s.BH;
+  const size_t qbar_b = align256(BH * s.Nq * s.D * sizeof(double));
+  const size_t kbar_b = align256(BH * s.Nk * s.D * sizeof(double));
+  const size_t S_b = scores_out ? 0 : align256(BH * s.Nq * s.Nk * sizeof(double));
+  const size_t crit_b = crit_idx_out ? 0 : align256(BH * s.Nq * s.Nk * sizeof(int32_t));
+  const size_t cnt_b = align256(BH * s.Nq * sizeof(int32_t));
+  const size_t need = qbar_b + kbar_b + S_b + crit_b + cnt_b;
+  if (need > kRouteScratchBytes)
+    return fail(SLA_ERR_WORKSPACE,
+                "sla_route_noalloc: this problem needs %zu bytes of scratch, above the built-in maximum of %zu "
+                "bytes; pass scores_out/crit_idx_out or use sla_route with a workspace",
+                need, kRouteScratchBytes);
+  void* base = nullptr;
+  SLA_TRY(route_scratch_address(&base));
+  uint8_t* b = static_cast<uint8_t*>(base);
+  Workspace w{};
+  w.qbar = reinterpret_cast<double*>(b);
+  w.kbar = reinterpret_cast<double*>(b + qbar_b);
+  w.S = S_b ? reinterpret_cast<double*>(b + qbar_b + kbar_b) : nullptr;
+  w.crit = crit_b ? reinterpret_cast<int32_t*>(b + qbar_b + kbar_b + S_b) : nullptr;
+  w.crit_cnt = reinterpret_cast<int32_t*>(b + qbar_b + kbar_b + S_b + crit_b);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) return route_impl<64>(s, q, k, mask_out, crit_idx_out, scores_out, w, st);
+  return route_impl<128>(s, q, k, mask_out, crit_idx_out, scores_out, w, st);
+}
