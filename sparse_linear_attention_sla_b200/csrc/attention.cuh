@@ -14,17 +14,22 @@
 // item 1 (the sparse branch renormalises over its keys) and §2.A
 // (O = alpha * O_s + (1 - alpha) * O_l).
 //
+// Two CTAs share an SM (<= 98 KB shared memory, 256 TMEM columns and <= 168
+// registers per thread each), so one CTA's softmax overlaps the other's MMAs.
 // Warp roles (192 threads):
-//   warp 0      TMA producer: Q tile, H_i tile, then K_j / V_j of every
-//               critical block j through an NS-stage ring.
-//   warp 1      TMEM owner and single-thread tcgen05 MMA issuer:
-//               S = Q K_j^T (M=128, N=64), O_s += P V_j (M=128, N=D),
+//   warp 0      TMA producer: Q tile, then K_j / V_j of every critical block j
+//               through a 2-slot ring, then H_i into the next free slot.
+//   warp 1      TMEM owner and single-thread tcgen05 issuer:
+//               S = Q K_j^T (M=128, N=64, both operands in shared memory),
+//               O_s += P V_j (M=128, N=D, P read from TMEM),
 //               O_l = phi(Q) H_i (M=128, N=D).
 //   warps 2..5  softmax / epilogue warpgroup: thread <-> query row <-> TMEM lane.
 //
-// TMEM columns: S ping-pong [0,64) [64,128), O_s [128,128+D), O_l [128+D,128+2D).
-// An empty critical set gives O_s = 0; an empty marginal set gives Z_i = 0 and
-// O_l = 0.
+// TMEM columns: S ping-pong [0,64) [64,128) (P, bf16, is written back over the
+// first 32 columns of its S), O_s [128,128+D); after the sparse loop O_l
+// reuses [0,D). tcgen05 MMAs issued by one thread run in order, so S_{n+2}
+// never overwrites P_n before PV_n has read it.
+// An empty critical set gives O_s = 0; an empty marginal set gives Z_i = 0 and O_l = 0.
 #pragma once
 
 #include "sm100.cuh"
@@ -53,33 +58,30 @@ __device__ __forceinline__ void wg_barrier() { asm volatile("bar.sync 1, 128;" :
 template <int D>
 struct AttnSmem {
   static constexpr uint32_t Q = 128 * D * 2;       // Q tile (later phi(Q), then the output staging)
-  static constexpr uint32_t KV = 64 * D * 2;       // one K or V stage
-  static constexpr uint32_t P = 128 * 64 * 2;      // one P buffer
+  static constexpr uint32_t KV = 64 * D * 2;       // one K or one V tile
+  static constexpr uint32_t SLOT = 2 * KV;         // one ring slot: K then V (or the H_i tile)
   static constexpr uint32_t HT = D * D * 2;        // H_i tile
-  template <int NS>
-  static constexpr uint32_t total() { return Q + 2 * NS * KV + 2 * P + HT + 1024; }
+  static_assert(HT <= SLOT, "H_i tile must fit in a ring slot");
+  static constexpr uint32_t total() { return Q + 2 * SLOT + 1024; }
 };
 
-template <int D, int NS>
-__global__ void __launch_bounds__(192, 1)
+template <int D>
+__global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
                 const __grid_constant__ CUtensorMap map_o, AttnArgs a) {
   using L = AttnSmem<D>;
-  constexpr int DB = D / 64;                    // 64-column boxes per row
-  constexpr uint32_t TMEM_COLS = (128 + 2 * D) <= 256 ? 256 : 512;
-  constexpr uint32_t OS = 128, OL = 128 + D;
+  constexpr int DB = D / 64;  // 64-column boxes per row
+  constexpr uint32_t TMEM_COLS = 256;
+  constexpr uint32_t OS = 128, OL = 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
-  uint8_t* sK = sQ + L::Q;
-  uint8_t* sV = sK + NS * L::KV;
-  uint8_t* sP = sV + NS * L::KV;
-  uint8_t* sH = sP + 2 * L::P;
+  uint8_t* sRing = sQ + L::Q;  // slot s at sRing + s * SLOT: K at +0, V at +KV
 
   __shared__ uint64_t q_full, h_full, phiq_full, ol_done, drain;
-  __shared__ uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-  __shared__ uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  __shared__ uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   __shared__ float sZ[D], sAlpha[D];
@@ -89,6 +91,7 @@ __global__ void __launch_bounds__(192, 1)
   const int row_id = bh * a.Nq + i;
   const int kc = a.crit_cnt[row_id];
   const int32_t* clist = a.crit + static_cast<size_t>(row_id) * a.crit_ld;
+  const int hslot = kc & 1;  // ring slot that receives H_i after the last K/V block
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
@@ -96,17 +99,14 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(&phiq_full, 128);
     mbar_init(&ol_done, 1);
     mbar_init(&drain, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_free[b], 128);
-      mbar_init(&p_full[b], 128);
-      mbar_init(&pv_done[b], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&pv_done[s], 1);
     }
     abort_flag = 0;
     fence_mbar_init();
@@ -128,36 +128,42 @@ __global__ void __launch_bounds__(192, 1)
       prefetch_tmap(&map_h);
       mbar_arrive_expect_tx(&q_full, L::Q);
       for (int b = 0; b < DB; ++b) tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * a.block_q, bh);
-      mbar_arrive_expect_tx(&h_full, L::HT);
-      for (int dh = 0; dh < DB; ++dh)
-        for (int eh = 0; eh < DB; ++eh)
-          tma_load_2d(sH + (dh * DB + eh) * 8192, &map_h, &h_full, eh * 64, row_id * D + dh * 64);
-      int last_round[NS];
-      for (int s = 0; s < NS; ++s) last_round[s] = -1;
-      for (int n = 0; n < kc; ++n) {
-        const int s = n % NS, r = n / NS;
+      int k_round[2] = {-1, -1}, v_round[2] = {-1, -1};
+      bool h_issued = false;
+      bool ok = true;
+      for (int n = 0; n < kc && ok; ++n) {
+        const int s = n & 1, r = n >> 1;
         const int j = clist[n];
-        if (r > 0 && !mbar_wait(&k_empty[s], (r - 1) & 1, a.err, &abort_flag)) break;
+        uint8_t* slot = sRing + s * L::SLOT;
+        if (r > 0 && !(ok = mbar_wait(&k_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
         mbar_arrive_expect_tx(&k_full[s], L::KV);
-        for (int b = 0; b < DB; ++b) tma_load_3d(sK + s * L::KV + b * 8192, &map_k, &k_full[s], b * 64, j * 64, bh);
-        if (r > 0 && !mbar_wait(&v_empty[s], (r - 1) & 1, a.err, &abort_flag)) {
-          last_round[s] = r;  // the K half of this stage is in flight
-          mbar_wait(&k_full[s], r & 1, nullptr, nullptr);
-          last_round[s] = -1;
-          break;
-        }
+        for (int b = 0; b < DB; ++b) tma_load_3d(slot + b * 8192, &map_k, &k_full[s], b * 64, j * 64, bh);
+        k_round[s] = r;
+        if (r > 0 && !(ok = mbar_wait(&v_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
         mbar_arrive_expect_tx(&v_full[s], L::KV);
-        for (int b = 0; b < DB; ++b) tma_load_3d(sV + s * L::KV + b * 8192, &map_v, &v_full[s], b * 64, j * 64, bh);
-        last_round[s] = r;
+        for (int b = 0; b < DB; ++b) tma_load_3d(slot + L::KV + b * 8192, &map_v, &v_full[s], b * 64, j * 64, bh);
+        v_round[s] = r;
+      }
+      if (ok) {  // H_i goes into the slot the next block would have used
+        const int r = kc >> 1;
+        if (r > 0) ok = mbar_wait(&k_empty[hslot], (r - 1) & 1, a.err, &abort_flag) &&
+                        mbar_wait(&v_empty[hslot], (r - 1) & 1, a.err, &abort_flag);
+        if (ok) {
+          uint8_t* slot = sRing + hslot * L::SLOT;
+          mbar_arrive_expect_tx(&h_full, L::HT);
+          for (int dh = 0; dh < DB; ++dh)
+            for (int eh = 0; eh < DB; ++eh)
+              tma_load_2d(slot + (dh * DB + eh) * 8192, &map_h, &h_full, eh * 64, row_id * D + dh * 64);
+          h_issued = true;
+        }
       }
       if (abort_flag) {  // let every load still in flight land before the CTA retires
         mbar_wait(&q_full, 0, nullptr, nullptr);
-        mbar_wait(&h_full, 0, nullptr, nullptr);
-        for (int s = 0; s < NS; ++s)
-          if (last_round[s] >= 0) {
-            mbar_wait(&k_full[s], last_round[s] & 1, nullptr, nullptr);
-            mbar_wait(&v_full[s], last_round[s] & 1, nullptr, nullptr);
-          }
+        if (h_issued) mbar_wait(&h_full, 0, nullptr, nullptr);
+        for (int s = 0; s < 2; ++s) {
+          if (k_round[s] >= 0) mbar_wait(&k_full[s], k_round[s] & 1, nullptr, nullptr);
+          if (v_round[s] >= 0) mbar_wait(&v_full[s], v_round[s] & 1, nullptr, nullptr);
+        }
       }
     }
     __syncwarp();
@@ -166,35 +172,35 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV), p0 = smem_u32(sP), h0 = smem_u32(sH);
+      const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing);
       bool ok = mbar_wait(&q_full, 0, a.err, &abort_flag);
       auto issue_pv = [&](int m) -> bool {
-        const int b = m & 1, s = m % NS;
-        if (!mbar_wait(&p_full[b], (m >> 1) & 1, a.err, &abort_flag)) return false;
-        if (!mbar_wait(&v_full[s], (m / NS) & 1, a.err, &abort_flag)) return false;
+        const int s = m & 1;
+        if (!mbar_wait(&p_full[s], (m >> 1) & 1, a.err, &abort_flag)) return false;
+        if (!mbar_wait(&v_full[s], (m >> 1) & 1, a.err, &abort_flag)) return false;
         tc_fence_after();
+        const uint32_t vb = ring0 + s * L::SLOT + L::KV;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = smem_desc_sw128(p0 + b * L::P + kk * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(v0 + s * L::KV + kk * 2048, 8192, 1024);
-          umma_bf16_ss(tmem + OS, ad, bd, id_o, (m > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(vb + kk * 2048, 8192, 1024);
+          umma_bf16_ts(tmem + OS, tmem + s * 64 + kk * 8, bd, id_o, (m > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&pv_done[b]);
+        umma_commit(&pv_done[s]);
         umma_commit(&v_empty[s]);
         return true;
       };
       for (int n = 0; ok && n < kc; ++n) {
-        const int s = n % NS, b = n & 1;
-        if (!mbar_wait(&k_full[s], (n / NS) & 1, a.err, &abort_flag)) { ok = false; break; }
-        if (n >= 2 && !mbar_wait(&s_free[b], ((n >> 1) - 1) & 1, a.err, &abort_flag)) { ok = false; break; }
+        const int s = n & 1;
+        if (!mbar_wait(&k_full[s], (n >> 1) & 1, a.err, &abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t kb = ring0 + s * L::SLOT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(k0 + s * L::KV + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(tmem + b * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          umma_bf16_ss(tmem + s * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[b]);
+        umma_commit(&s_full[s]);
         umma_commit(&k_empty[s]);
         if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
       }
@@ -204,10 +210,11 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) ok = mbar_wait(&phiq_full, 0, a.err, &abort_flag);
       if (ok) {
         tc_fence_after();
+        const uint32_t hb = ring0 + hslot * L::SLOT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(h0 + (kk >> 2) * DB * 8192 + (kk & 3) * 2048, 8192, 1024);
+          const uint64_t bd = smem_desc_sw128(hb + (kk >> 2) * DB * 8192 + (kk & 3) * 2048, 8192, 1024);
           umma_bf16_ss(tmem + OL, ad, bd, id_o, kk > 0 ? 1u : 0u);
         }
         umma_commit(&ol_done);
@@ -228,7 +235,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     wg_barrier();
 
-    float m_run = -INFINITY, l_run = 0.f;
+    const float sc = a.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and row sum
     bool ok = true;
     for (int n = 0; n < kc; ++n) {
       const int b = n & 1;
@@ -239,18 +247,16 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(lane_addr + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&s_free[b]);
-
-      const int j = clist[n];
-      const int valid = min(64, a.N - j * 64);
-      float x[64];
-      float mx = -INFINITY;
+      const int valid = min(64, a.N - clist[n] * 64);
+      if (valid < 64) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        x[c] = c < valid ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+        for (int c = 0; c < 64; ++c)
+          if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
       }
+      float mx = __uint_as_float(sv[0]);
+#pragma unroll
+      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+      mx *= sc;
       if (n == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
@@ -273,29 +279,24 @@ __global__ void __launch_bounds__(192, 1)
         l_run *= f;
         m_run = m_new;
       }
-      float ps = 0.f;
+      // p = 2^(s * scale - m): one FMA and one exponential per element
+      float ps0 = 0.f, ps1 = 0.f;
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        const float e0 = fast_exp2(x[c] - m_run), e1 = fast_exp2(x[c + 1] - m_run);
-        ps += e0 + e1;
+        const float e0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sc, -m_run));
+        const float e1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sc, -m_run));
+        ps0 += e0;
+        ps1 += e1;
         pk[c >> 1] = pack_bf16x2(e0, e1);
       }
-      l_run += ps;
-      if (n >= 2) {  // P buffer b is free once PV_{n-2} has finished
-        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[b], ((n - 2) >> 1) & 1, a.err, &abort_flag));
-        if (!ok) break;
-      }
-      uint8_t* prow = sP + b * L::P;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        *reinterpret_cast<uint4*>(prow + sw128_offset(r, c8 * 16)) =
-            make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-      fence_proxy_async_smem();
+      l_run += ps0 + ps1;
+      tmem_st32(lane_addr + b * 64, pk);  // P_n over the first 32 columns of S_n
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
     }
-    // Every MMA that reads Q has finished once the last PV has (commits complete in order).
+    // Every MMA that reads Q (or the S/P columns) has finished once the last PV has.
     if (ok && kc > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(kc - 1) & 1], ((kc - 1) >> 1) & 1, a.err, &abort_flag));
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, a.err, &abort_flag));
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(192, 1)
     // same rounded phi(q) the MMA sees.
     float den = 0.f;
     if (ok) {
-#pragma unroll
+#pragma unroll 4
       for (int c8 = 0; c8 < D / 8; ++c8) {
         uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
         uint4 u = *p;
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const float inv_d = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t os[32], ol[32];
         tmem_ld32(lane_addr + OS + c0, os);

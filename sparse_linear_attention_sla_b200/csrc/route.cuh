@@ -183,6 +183,139 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   if (lane == 0 && a.crit_cnt) a.crit_cnt[row] = crit_before;
 }
 
+// Register-resident selection for rows of up to 32 * KPL blocks.
+//
+// Exactness argument: rounding a double to float is monotone, so with
+// key32 = order key of (float)S, every block whose key32 is above the
+// kc-th largest key32 (T) is above every block whose key32 is <= T in the
+// fp64 order too. The blocks with key32 == T are the only ones whose fp64
+// order matters; they are resolved by their fp64 key and then their index.
+// The result is the same set as the fp64 total order (S desc, j asc).
+__device__ __forceinline__ uint32_t order_key32(double s) {
+  const float f = static_cast<float>(s) + 0.0f;  // -0.0 folds onto +0.0
+  const uint32_t u = __float_as_uint(f);
+  return (u >> 31) ? ~u : (u | 0x80000000u);
+}
+
+// k-th largest of the (optionally complemented) 32-bit keys of the valid slots, k >= 1.
+template <int KPL>
+__device__ __forceinline__ uint32_t kth_largest32(const uint32_t (&key)[KPL], int nvalid_lane, int k, bool flip) {
+  uint32_t T = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    uint32_t c = 0;
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) {
+      const uint32_t kk = flip ? ~key[t] : key[t];
+      c += (t < nvalid_lane && kk >= cand) ? 1u : 0u;
+    }
+    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= k) T = cand;
+  }
+  return T;
+}
+
+// Among the slots flagged in `group` (bit t of each lane), pick `need` of them in the
+// order (fp64 key descending, index ascending) when best_high, or (fp64 key ascending,
+// index descending) otherwise; returns this lane's picks as a bit mask.
+template <int KPL>
+__device__ __forceinline__ uint64_t pick_from_group(const double* srow, uint64_t group, int need, bool best_high) {
+  const int lane = threadIdx.x & 31;
+  uint64_t picked = 0;
+  for (int it = 0; it < need; ++it) {
+    // this lane's best candidate
+    uint64_t bk = 0;
+    int bj = -1;
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) {
+      if (!((group & ~picked) >> t & 1ull)) continue;
+      const int j = lane + 32 * t;
+      const uint64_t k64 = best_high ? order_key(srow[j]) : ~order_key(srow[j]);
+      // higher k64 wins; on equal keys the lower index wins (best_high) or the higher one (otherwise)
+      if (bj < 0 || k64 > bk || (k64 == bk && (best_high ? j < bj : j > bj))) {
+        bk = k64;
+        bj = j;
+      }
+    }
+    // warp arg-best
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      const bool take = oj >= 0 && (bj < 0 || ok > bk || (ok == bk && (best_high ? oj < bj : oj > bj)));
+      if (take) {
+        bk = ok;
+        bj = oj;
+      }
+    }
+    if (bj >= 0 && (bj & 31) == lane) picked |= 1ull << (bj >> 5);
+  }
+  return picked;
+}
+
+template <int KPL>
+__global__ void __launch_bounds__(256) select_reg_kernel(SelectArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= a.rows) return;  // whole warp leaves; nothing below synchronises the CTA
+  const double* srow = a.S + static_cast<size_t>(row) * a.Nk;
+  const int nvalid_lane = (a.Nk - lane + 31) / 32;  // slots t < nvalid_lane hold j = lane + 32 t < Nk
+  uint32_t key[KPL];
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) key[t] = t < nvalid_lane ? order_key32(srow[lane + 32 * t]) : 0u;
+
+  uint32_t Tc = 0, Tn = 0;
+  uint64_t eqc = 0, eqn = 0, pick_c = 0, pick_n = 0;
+  if (a.kc > 0) {
+    Tc = kth_largest32<KPL>(key, nvalid_lane, a.kc, false);
+    uint32_t gt = 0;
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) {
+      const bool v = t < nvalid_lane;
+      gt += (v && key[t] > Tc) ? 1u : 0u;
+      if (v && key[t] == Tc) eqc |= 1ull << t;
+    }
+    const int need = a.kc - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    const int neq = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popcll(eqc))));
+    pick_c = need >= neq ? eqc : pick_from_group<KPL>(srow, eqc, need, true);
+  }
+  if (a.kn > 0) {
+    Tn = ~kth_largest32<KPL>(key, nvalid_lane, a.kn, true);
+    uint32_t lt = 0;
+#pragma unroll
+    for (int t = 0; t < KPL; ++t) {
+      const bool v = t < nvalid_lane;
+      lt += (v && key[t] < Tn) ? 1u : 0u;
+      if (v && key[t] == Tn) eqn |= 1ull << t;
+    }
+    const int need = a.kn - static_cast<int>(__reduce_add_sync(0xffffffffu, lt));
+    const int neq = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popcll(eqn))));
+    pick_n = need >= neq ? eqn : pick_from_group<KPL>(srow, eqn, need, false);
+  }
+
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int crit_before = 0;
+#pragma unroll
+  for (int t = 0; t < KPL; ++t) {
+    if (32 * t >= a.Nk) break;
+    const int j = lane + 32 * t;
+    const bool in = t < nvalid_lane;
+    const bool is_c = in && a.kc > 0 && (key[t] > Tc || (pick_c >> t & 1ull));
+    const bool is_n = in && a.kn > 0 && !is_c && (key[t] < Tn || (pick_n >> t & 1ull));
+    const uint32_t bcrit = __ballot_sync(0xffffffffu, is_c);
+    if (in) {
+      const int8_t lab = is_c ? 2 : (is_n ? 0 : 1);
+      if (a.mask) a.mask[static_cast<size_t>(row) * a.Nk + j] = lab;
+      if (a.W) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(lab == 1 ? 1.f : 0.f);
+      if (is_c && a.crit) a.crit[static_cast<size_t>(row) * a.crit_ld + crit_before + __popc(bcrit & lt_mask)] = j;
+    }
+    crit_before += __popc(bcrit);
+  }
+  if (a.W)
+    for (int j = a.Nk + lane; j < a.w_ld; j += 32) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(0.f);
+  if (lane == 0 && a.crit_cnt) a.crit_cnt[row] = crit_before;
+}
+
 // ---------------------------------------------------------------- caller mask
 struct MaskListArgs {
   const int8_t* mask;   // [rows, Nk]

@@ -24,7 +24,6 @@ using sla::MaskListArgs;
 using sla::SelectArgs;
 
 constexpr int kMaxNk = 16384;
-constexpr int kAttnStages = 3;
 thread_local std::string g_last_error;
 
 sla_status fail(sla_status st, const char* fmt, ...) {
@@ -236,7 +235,19 @@ sla_status launch_scores(const double* qbar, const double* kbar, double* S, cons
   return launched("score_kernel");
 }
 
+template <int KPL>
+sla_status launch_select_reg(const SelectArgs& a, cudaStream_t st) {
+  const int wpc = 8;
+  sla::select_reg_kernel<KPL><<<(a.rows + wpc - 1) / wpc, wpc * 32, 0, st>>>(a);
+  return launched("select_reg_kernel");
+}
+
 sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
+  // Rows of up to 2048 blocks keep their keys in registers; longer rows use shared memory.
+  if (a.Nk <= 32 * 8) return launch_select_reg<8>(a, st);
+  if (a.Nk <= 32 * 16) return launch_select_reg<16>(a, st);
+  if (a.Nk <= 32 * 32) return launch_select_reg<32>(a, st);
+  if (a.Nk <= 32 * 64) return launch_select_reg<64>(a, st);
   const size_t per_warp = static_cast<size_t>(a.Nk) * 8;
   int wpc = static_cast<int>((200 * 1024) / per_warp);
   wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
@@ -284,8 +295,8 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
     const uint32_t box[2] = {64, 64};
     SLA_TRY(make_map(&mh, w.Hagg, 2, dims, strides, box));
   }
-  constexpr int smem = sla::AttnSmem<D>::template total<kAttnStages>();
-  SLA_TRY(allow_smem(sla::attn_kernel<D, kAttnStages>, smem));
+  constexpr int smem = sla::AttnSmem<D>::total();
+  SLA_TRY(allow_smem(sla::attn_kernel<D>, smem));
   AttnArgs a;
   a.H = s.H;
   a.N = s.N;
@@ -298,7 +309,7 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.alpha = alpha;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   a.err = w.err;
-  sla::attn_kernel<D, kAttnStages><<<dim3(s.Nq, s.BH), 192, smem, st>>>(mq, mk, mv, mh, mo, a);
+  sla::attn_kernel<D><<<dim3(s.Nq, s.BH), 192, smem, st>>>(mq, mk, mv, mh, mo, a);
   return launched("attn_kernel");
 }
 
