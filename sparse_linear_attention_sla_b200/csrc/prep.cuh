@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(128) pool_mean_kernel(const __nv_bfloat16* __r
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float2 f = unpack_bf16x2(w[e]);
+      const float2 f = unpack_bf16x2(w[e]);
       acc[2 * e] += static_cast<double>(f.x);
       acc[2 * e + 1] += static_cast<double>(f.y);
     }
@@ -67,29 +67,45 @@ struct KvPrepArgs {
   uint32_t* err;
 };
 
-// One CTA walks over KV blocks g = blockIdx.x, blockIdx.x + gridDim.x, ...
-// with a two-stage TMA ring. 128 threads. Dynamic smem: 2 stages x (K 16 KB + V 16 KB).
-// For D = 64 the K stage keeps a zeroed second half so the M = 128 MMA reads
-// zeros for rows 64..127 of phi(K)^T.
 template <int D>
-__global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CUtensorMap map_k,
-                                                      const __grid_constant__ CUtensorMap map_v, KvPrepArgs a) {
+struct KvPrepSmem {
+  static constexpr uint32_t SLOT = 32768;               // K (16 KB, zero upper half when D = 64) + V (16 KB)
+  static constexpr uint32_t STAGE = D * 128 * (D / 64); // bf16 h_j staging for the TMA store
+  static constexpr uint32_t total() { return 2 * SLOT + STAGE + 1024; }
+};
+
+// One CTA walks over KV blocks g = blockIdx.x, blockIdx.x + gridDim.x, ... with a
+// two-slot TMA ring; two CTAs share an SM. 128 threads.
+//   column pass  16-byte vectors: sum k (fp64) and phi(k) (fp32) per column, and
+//                rewrite the K tile in place as phi(k) (zero past the sequence end)
+//   MMA          h_j = phi(K_j)^T V_j on tcgen05 (M=128, N=D, K=64 tokens; both
+//                operands MN-major); for D = 64 rows 64..127 of phi(K)^T read zeros
+//   epilogue     bf16 h_j staged in shared memory and written by one TMA store
+//                (forward), or fp32 straight from registers (state export).
+template <int D>
+__global__ void __launch_bounds__(128, 2) kv_prep_kernel(const __grid_constant__ CUtensorMap map_k,
+                                                         const __grid_constant__ CUtensorMap map_v,
+                                                         const __grid_constant__ CUtensorMap map_hout, KvPrepArgs a) {
+  using L = KvPrepSmem<D>;
   constexpr int BK = 64;
   constexpr int KBOX = D / 64;              // 64-column boxes per row
-  constexpr uint32_t TILE = 16384;           // bytes reserved per K (or V) stage
-  constexpr uint32_t TX = BK * D * 2 * 2;    // K + V bytes per block
+  constexpr uint32_t TX = BK * D * 2 * 2;   // K + V bytes per block
+  constexpr int CPR = D / 8;                // 16-byte chunks per row
+  constexpr int RG = 128 / CPR;             // row groups
+  constexpr int RPT = BK / RG;              // rows per thread
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK[2] = {smem, smem + 2 * TILE};
-  uint8_t* sV[2] = {smem + TILE, smem + 3 * TILE};
+  uint8_t* slot[2] = {smem, smem + L::SLOT};
+  uint8_t* stage = smem + 2 * L::SLOT;
   __shared__ uint64_t bar_full[2], bar_mma;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ double ksum_part[2][D];
-  __shared__ float zsum_part[2][D];
+  __shared__ double ksum_part[RG][D];
+  __shared__ float zsum_part[RG][D];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int total = a.BH * a.Nk;
+  const bool bf16_out = a.hst != nullptr;
   if (tid == 0) {
     mbar_init(&bar_full[0], 1);
     mbar_init(&bar_full[1], 1);
@@ -98,10 +114,11 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     fence_mbar_init();
     prefetch_tmap(&map_k);
     prefetch_tmap(&map_v);
+    if (bf16_out) prefetch_tmap(&map_hout);
   }
-  if (D == 64) {  // zero the upper halves of both K stages once
+  if (D == 64) {  // zero the upper halves of both K areas once (TMA never writes them)
     for (int s = 0; s < 2; ++s)
-      for (int o = tid * 16; o < 8192; o += 128 * 16) *reinterpret_cast<uint4*>(sK[s] + 8192 + o) = make_uint4(0, 0, 0, 0);
+      for (int o = tid * 16; o < 8192; o += 128 * 16) *reinterpret_cast<uint4*>(slot[s] + 8192 + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (warp == 0) {
@@ -112,7 +129,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  // Thread 0 tracks which stages have a load in flight (parity of its phase, or -1)
+  // Thread 0 tracks which slots have a load in flight (parity of its phase, or -1)
   // so that an aborted CTA can let them land before it retires.
   int inflight[2] = {-1, -1};
   int mma_parity = -1;
@@ -121,8 +138,8 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     mbar_arrive_expect_tx(&bar_full[s], TX);
 #pragma unroll
     for (int b = 0; b < KBOX; ++b) {
-      tma_load_3d(sK[s] + b * 8192, &map_k, &bar_full[s], b * 64, j * BK, bh);
-      tma_load_3d(sV[s] + b * 8192, &map_v, &bar_full[s], b * 64, j * BK, bh);
+      tma_load_3d(slot[s] + b * 8192, &map_k, &bar_full[s], b * 64, j * BK, bh);
+      tma_load_3d(slot[s] + 16384 + b * 8192, &map_v, &bar_full[s], b * 64, j * BK, bh);
     }
     inflight[s] = round & 1;
   };
@@ -131,6 +148,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     if (blockIdx.x + gridDim.x < total) issue_load(blockIdx.x + gridDim.x, 1, 0);
   }
   const uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
+  const int cc = tid % CPR, rg = tid / CPR;
 
   int n = 0;
   for (int g = blockIdx.x; g < total; g += gridDim.x, ++n) {
@@ -141,30 +159,45 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     if (__syncthreads_or(!ok)) break;
     if (tid == 0) inflight[s] = -1;
 
-    // Column pass: a thread owns column c over all rows (D = 128) or half of them (D = 64);
-    // it sums k in fp64 and phi(k) in fp32, and rewrites the tile in place as phi(k)
-    // (zero on rows past the end of the sequence, which TMA filled with zeros).
+    // Column pass over 16-byte chunks: thread (cc, rg) owns columns 8cc..8cc+7 of rows rg + RG*k.
     {
-      constexpr int HALVES = 128 / D;
-      const int c = tid % D, half = tid / D;
-      const int rbeg = half * (BK / HALVES), rend = rbeg + BK / HALVES;
-      uint8_t* tile = sK[s] + (c / 64) * 8192;
-      const uint32_t cb = (c % 64) * 2;
-      double ks = 0.0;
-      float zs = 0.f;
-      for (int r = rbeg; r < rend; ++r) {
-        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(tile + sw128_offset(r, cb));
-        float kv = __bfloat162float(*p);
-        float f = 0.f;
-        if (r < valid) {
-          ks += static_cast<double>(kv);
-          f = phi_f(kv);
-          zs += f;
-        }
-        *p = __float2bfloat16_rn(f);
+      uint8_t* tile = slot[s] + (cc / 8) * 8192;
+      const uint32_t cb = (cc % 8) * 16;
+      double ks[8];
+      float zs[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ks[e] = 0.0;
+        zs[e] = 0.f;
       }
-      ksum_part[half][c] = ks;
-      zsum_part[half][c] = zs;
+#pragma unroll
+      for (int k = 0; k < RPT; ++k) {
+        const int r = rg + RG * k;
+        uint4* p = reinterpret_cast<uint4*>(tile + sw128_offset(r, cb));
+        const uint4 u = *p;
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const bool in = r < valid;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 kv = unpack_bf16x2(w[e]);
+          float f0 = 0.f, f1 = 0.f;
+          if (in) {
+            ks[2 * e] += static_cast<double>(kv.x);
+            ks[2 * e + 1] += static_cast<double>(kv.y);
+            f0 = phi_f(kv.x);
+            f1 = phi_f(kv.y);
+            zs[2 * e] += f0;
+            zs[2 * e + 1] += f1;
+          }
+          w[e] = pack_bf16x2(f0, f1);
+        }
+        *p = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ksum_part[rg][cc * 8 + e] = ks[e];
+        zsum_part[rg][cc * 8 + e] = zs[e];
+      }
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -172,8 +205,8 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk) {
-        uint64_t ad = smem_desc_sw128(smem_u32(sK[s]) + kk * 2048, 8192, 1024);
-        uint64_t bd = smem_desc_sw128(smem_u32(sV[s]) + kk * 2048, 8192, 1024);
+        uint64_t ad = smem_desc_sw128(smem_u32(slot[s]) + kk * 2048, 8192, 1024);
+        uint64_t bd = smem_desc_sw128(smem_u32(slot[s]) + 16384 + kk * 2048, 8192, 1024);
         umma_bf16_ss(tmem, ad, bd, idesc, kk > 0);
       }
       umma_commit(&bar_mma);
@@ -181,15 +214,16 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     }
     // kbar and z while the MMA runs
     if (tid < D) {
-      double ks = ksum_part[0][tid];
-      float zs = zsum_part[0][tid];
-      if (D == 64) {
-        ks += ksum_part[1][tid];
-        zs += zsum_part[1][tid];
+      double ks = 0.0;
+      float zs = 0.f;
+#pragma unroll
+      for (int q = 0; q < RG; ++q) {
+        ks += ksum_part[q][tid];
+        zs += zsum_part[q][tid];
       }
       const size_t row = static_cast<size_t>(bh) * a.Nk + j;
       if (a.kbar) a.kbar[row * D + tid] = ks / static_cast<double>(valid);
-      if (a.hst) {
+      if (bf16_out) {
         __nv_bfloat16* zr = a.hst + row * a.LD + D * D;
         zr[tid] = __float2bfloat16_rn(zs);
         if (D == 64) zr[64 + tid] = __float2bfloat16_rn(0.f);
@@ -198,10 +232,11 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       }
     }
     ok = mbar_wait(&bar_mma, n & 1, a.err, &abort_flag);
+    if (tid == 0 && bf16_out) tma_store_wait_read();  // the previous block's store has left the staging tile
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
     if (tid == 0) mma_parity = -1;
-    // The MMA has consumed stage s: refill it with the block two steps ahead.
+    // The MMA has consumed slot s: refill it with the block two steps ahead.
     if (tid == 0 && g + 2 * gridDim.x < total) issue_load(g + 2 * gridDim.x, s, (n >> 1) + 1);
     // Epilogue: warp w holds rows d = 32 w .. 32 w + 31 of h_j.
     if (warp * 32 < D) {
@@ -212,8 +247,8 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         uint32_t r[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, r);
         tmem_wait_ld();
-        if (a.hst) {
-          uint4* dst = reinterpret_cast<uint4*>(a.hst + row * a.LD + static_cast<size_t>(d) * D + c0);
+        if (bf16_out) {
+          uint8_t* box = stage + (c0 >> 6) * (D * 128);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 u;
@@ -221,7 +256,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
             u.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
             u.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
             u.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-            dst[q] = u;
+            *reinterpret_cast<uint4*>(box + sw128_offset(d, ((c0 & 63) >> 3) * 16 + q * 16)) = u;
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(a.h32 + (row * D + d) * D + c0);
@@ -232,14 +267,20 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         }
       }
     }
+    if (bf16_out) fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && bf16_out) {
+      for (int b = 0; b < KBOX; ++b) tma_store_3d(&map_hout, stage + b * (D * 128), b * 64, 0, bh * a.Nk + j);
+      tma_store_commit();
+    }
   }
   // After an abort: let loads and the MMA still in flight finish before the CTA retires.
   if (tid == 0) {
     for (int s = 0; s < 2; ++s)
       if (inflight[s] >= 0) mbar_wait(&bar_full[s], inflight[s], nullptr, nullptr);
     if (mma_parity >= 0) mbar_wait(&bar_mma, mma_parity, nullptr, nullptr);
+    if (bf16_out) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();

@@ -23,53 +23,66 @@
 namespace sla {
 
 // ---------------------------------------------------------------- scores
-// grid: (ceil(Nk/64), ceil(Nq/64), BH); block 256. Each thread computes a 4 x 4 patch.
+// D(8x8) += A(8x4) * B(4x8) in fp64 on the tensor cores (one warp). Fragments:
+// a = A[lane/4][lane%4], b = B[lane%4][lane/4], d = D[lane/4][2*(lane%4) + {0,1}].
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
+// grid: (ceil(Nk/64), ceil(Nq/64), BH); block 128 = 2 x 2 warps, each warp a 32 x 32 patch
+// of S as 4 x 4 tiles of 8 x 8. D is walked in chunks of 32 staged in shared memory.
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
+__global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar,
                                                     double* __restrict__ S, int Nq, int Nk) {
-  constexpr int T = 64, DC = 32;
-  __shared__ double sq[DC][T + 1];
-  __shared__ double sk[DC][T + 1];
+  constexpr int T = 64, DC = 32, LDS = DC + 1;
+  __shared__ double sq[T * LDS];
+  __shared__ double sk[T * LDS];
   const int bh = blockIdx.z, i0 = blockIdx.y * T, j0 = blockIdx.x * T;
-  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wy = warp >> 1, wx = warp & 1;
+  const int fr = lane >> 2, fc = lane & 3;
   const double* qb = qbar + static_cast<size_t>(bh) * Nq * D;
   const double* kb = kbar + static_cast<size_t>(bh) * Nk * D;
-  double acc[4][4];
+  double acc[4][4][2];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    for (int b = 0; b < 4; ++b) acc[a][b][0] = acc[a][b][1] = 0.0;
   for (int d0 = 0; d0 < D; d0 += DC) {
-    for (int e = tid; e < T * DC; e += 256) {
+    for (int e = tid; e < T * DC; e += 128) {
       const int r = e / DC, d = e % DC;
-      sq[d][r] = (i0 + r < Nq) ? qb[static_cast<size_t>(i0 + r) * D + d0 + d] : 0.0;
-      sk[d][r] = (j0 + r < Nk) ? kb[static_cast<size_t>(j0 + r) * D + d0 + d] : 0.0;
+      sq[r * LDS + d] = (i0 + r < Nq) ? qb[static_cast<size_t>(i0 + r) * D + d0 + d] : 0.0;
+      sk[r * LDS + d] = (j0 + r < Nk) ? kb[static_cast<size_t>(j0 + r) * D + d0 + d] : 0.0;
     }
     __syncthreads();
-#pragma unroll 8
-    for (int d = 0; d < DC; ++d) {
-      double qa[4], kb4[4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qa[a] = sq[d][ty + 16 * a];
+    for (int kk = 0; kk < DC; kk += 4) {
+      double af[4], bf[4];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) kb4[b] = sk[d][tx + 16 * b];
+      for (int a = 0; a < 4; ++a) af[a] = sq[(wy * 32 + a * 8 + fr) * LDS + kk + fc];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) bf[b] = sk[(wx * 32 + b * 8 + fr) * LDS + kk + fc];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fma(qa[a], kb4[b], acc[a][b]);
+        for (int b = 0; b < 4; ++b) dmma_8x8x4(acc[a][b], af[a], bf[b]);
     }
     __syncthreads();
   }
   const double rs = sqrt(static_cast<double>(D));
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
-    const int i = i0 + ty + 16 * a;
+    const int i = i0 + wy * 32 + a * 8 + fr;
     if (i >= Nq) continue;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int j = j0 + tx + 16 * b;
-      if (j < Nk) S[(static_cast<size_t>(bh) * Nq + i) * Nk + j] = acc[a][b] / rs;
-    }
+    for (int b = 0; b < 4; ++b)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = j0 + wx * 32 + b * 8 + 2 * fc + h;
+        if (j < Nk) S[(static_cast<size_t>(bh) * Nq + i) * Nk + j] = acc[a][b][h] / rs;
+      }
   }
 }
 
@@ -197,7 +210,10 @@ __device__ __forceinline__ uint32_t order_key32(double s) {
   return (u >> 31) ? ~u : (u | 0x80000000u);
 }
 
-// k-th largest of the (optionally complemented) 32-bit keys of the valid slots, k >= 1.
+// A threshold T on the (optionally complemented) 32-bit keys of the valid slots with
+// #{key >= T} >= k whose top-k set is fixed: either T is the k-th largest key, or
+// exactly k keys are >= T (then they are the top k and no key equals a smaller
+// candidate). k >= 1. Bisection on the bits, stopping as soon as the count is exactly k.
 template <int KPL>
 __device__ __forceinline__ uint32_t kth_largest32(const uint32_t (&key)[KPL], int nvalid_lane, int k, bool flip) {
   uint32_t T = 0;
@@ -210,7 +226,9 @@ __device__ __forceinline__ uint32_t kth_largest32(const uint32_t (&key)[KPL], in
       const uint32_t kk = flip ? ~key[t] : key[t];
       c += (t < nvalid_lane && kk >= cand) ? 1u : 0u;
     }
-    if (static_cast<int>(__reduce_add_sync(0xffffffffu, c)) >= k) T = cand;
+    const int cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, c));
+    if (cnt >= k) T = cand;
+    if (cnt == k) break;  // the k keys >= cand are exactly the top k
   }
   return T;
 }

@@ -217,21 +217,30 @@ sla_status launch_pool(const void* x, double* out, const Shape& s, int block, in
 
 template <int D>
 sla_status launch_kv_prep(const void* k, const void* v, const Shape& s, const KvPrepArgs& args, cudaStream_t st) {
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mv, mh;
   SLA_TRY(act_map(&mk, k, s, 64));
   SLA_TRY(act_map(&mv, v, s, 64));
-  const int smem = 4 * 16384 + 1024;
+  std::memset(&mh, 0, sizeof(mh));
+  if (args.hst) {
+    // h_j tiles inside the stacked-state rows: (e, d, block) -> row * LD + d * D + e
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.D),
+                              static_cast<uint64_t>(s.BH) * s.Nk};
+    const uint64_t strides[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.LD)};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(s.D), 1};
+    SLA_TRY(make_map(&mh, args.hst, 3, dims, strides, box));
+  }
+  constexpr int smem = sla::KvPrepSmem<D>::total();
   SLA_TRY(allow_smem(sla::kv_prep_kernel<D>, smem));
   const int total = s.BH * s.Nk;
-  const int grid = total < 3 * sm_count() ? total : 3 * sm_count();
-  sla::kv_prep_kernel<D><<<grid, 128, smem, st>>>(mk, mv, args);
+  const int grid = total < 2 * sm_count() ? total : 2 * sm_count();
+  sla::kv_prep_kernel<D><<<grid, 128, smem, st>>>(mk, mv, mh, args);
   return launched("kv_prep_kernel");
 }
 
 template <int D>
 sla_status launch_scores(const double* qbar, const double* kbar, double* S, const Shape& s, cudaStream_t st) {
   dim3 grid((s.Nk + 63) / 64, (s.Nq + 63) / 64, s.BH);
-  sla::score_kernel<D><<<grid, 256, 0, st>>>(qbar, kbar, S, s.Nq, s.Nk);
+  sla::score_kernel<D><<<grid, 128, 0, st>>>(qbar, kbar, S, s.Nq, s.Nk);
   return launched("score_kernel");
 }
 
@@ -260,7 +269,7 @@ sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
 
 template <int D>
 sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
-  CUtensorMap mw, mh;
+  CUtensorMap mw, mh, mo;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
     const uint64_t strides[2] = {static_cast<uint64_t>(s.w_ld), static_cast<uint64_t>(s.Nq) * s.w_ld};
@@ -273,11 +282,18 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
     const uint32_t box[3] = {64, 64, 1};
     SLA_TRY(make_map(&mh, w.hst, 3, dims, strides, box));
   }
-  const int smem = 2 * (16384 + 32768) + 1024;
+  {
+    const uint64_t DD = static_cast<uint64_t>(s.D) * s.D;
+    const uint64_t dims[3] = {DD, static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
+    const uint64_t strides[2] = {DD, static_cast<uint64_t>(s.Nq) * DD};
+    const uint32_t box[3] = {64, 128, 1};
+    SLA_TRY(make_map(&mo, w.Hagg, 3, dims, strides, box));
+  }
+  const int smem = 2 * sla::kAggStageBytes + 1024;
   SLA_TRY(allow_smem(sla::agg_kernel<D>, smem));
   AggArgs a{s.Nq, s.Nk, s.LD, w.Hagg, w.Zagg, w.err};
-  dim3 grid((s.LD + 255) / 256, (s.Nq + 127) / 128, s.BH);
-  sla::agg_kernel<D><<<grid, 128, smem, st>>>(mw, mh, a);
+  dim3 grid(s.LD / 128, (s.Nq + 255) / 256, s.BH);
+  sla::agg_kernel<D><<<grid, 128, smem, st>>>(mw, mh, mo, a);
   return launched("agg_kernel");
 }
 
