@@ -14,16 +14,18 @@
 // item 1 (the sparse branch renormalises over its keys) and §2.A
 // (O = alpha * O_s + (1 - alpha) * O_l).
 //
-// Two CTAs share an SM (<= 98 KB shared memory, 256 TMEM columns and <= 168
+// Two CTAs share an SM (<= 98 KB shared memory, 256 TMEM columns and <= 96
 // registers per thread each), so one CTA's softmax overlaps the other's MMAs.
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer: Q tile, then K_j / V_j of every critical block j
 //               through a 2-slot ring, then H_i into the next free slot.
 //   warp 1      TMEM owner and single-thread tcgen05 issuer:
 //               S = Q K_j^T (M=128, N=64, both operands in shared memory),
 //               O_s += P V_j (M=128, N=D, P read from TMEM),
 //               O_l = phi(Q) H_i (M=128, N=D).
-//   warps 2..5  softmax / epilogue warpgroup: thread <-> query row <-> TMEM lane.
+//   warps 2..9  two softmax / epilogue warpgroups: a thread owns one query row
+//               (= TMEM lane) and one half of the columns; the two threads of a
+//               row exchange their block maxima through shared memory.
 //
 // TMEM columns: S ping-pong [0,64) [64,128) (P, bf16, is written back over the
 // first 32 columns of its S), O_s [128,128+D); after the sparse loop O_l
@@ -53,7 +55,8 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void wg_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barrier over the two softmax warpgroups (256 threads).
+__device__ __forceinline__ void wg_barrier() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 template <int D>
 struct AttnSmem {
@@ -66,7 +69,7 @@ struct AttnSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(320, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
                 const __grid_constant__ CUtensorMap map_o, AttnArgs a) {
@@ -85,6 +88,8 @@ __global__ void __launch_bounds__(192, 2)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   __shared__ float sZ[D], sAlpha[D];
+  __shared__ float red_max[2][2][128];  // [block parity][half][row]
+  __shared__ float red_l[2][128], red_den[2][128];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(192, 2)
   if (tid == 0) {
     mbar_init(&q_full, 1);
     mbar_init(&h_full, 1);
-    mbar_init(&phiq_full, 128);
+    mbar_init(&phiq_full, 256);
     mbar_init(&ol_done, 1);
     mbar_init(&drain, 1);
     for (int s = 0; s < 2; ++s) {
@@ -105,7 +110,7 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+      mbar_init(&p_full[s], 256);
       mbar_init(&pv_done[s], 1);
     }
     abort_flag = 0;
@@ -224,56 +229,68 @@ __global__ void __launch_bounds__(192, 2)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax / epilogue warpgroup
-    const int wt = tid - 64;                    // 0..127
+    // ------------------------------------------------------------ softmax / epilogue warpgroups
+    const int wt = tid - 64;                    // 0..255
+    const int g = wt >> 7;                      // column half owned by this warpgroup
     const int quarter = warp & 3;               // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;          // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    for (int c = wt; c < D; c += 128) {
+    for (int c = wt; c < D; c += 256) {
       sZ[c] = a.Zagg[static_cast<size_t>(row_id) * D + c];
       sAlpha[c] = a.alpha[h * D + c];
     }
     wg_barrier();
 
     const float sc = a.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and row sum
+    float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and this half's row sum
     bool ok = true;
+    int j_next = kc > 0 ? clist[0] : 0;  // critical-block index, read one iteration ahead
+    // Every warp of both warpgroups runs every iteration and reaches every named barrier,
+    // also after a failed wait (then the work is skipped), so a barrier can never wait for a
+    // warp that has left the loop.
     for (int n = 0; n < kc; ++n) {
       const int b = n & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (n >> 1) & 1, a.err, &abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld32(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(lane_addr + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_wait_ld();
-      const int valid = min(64, a.N - clist[n] * 64);
-      if (valid < 64) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (n >> 1) & 1, a.err, &abort_flag));
+      uint32_t sv[32];
+      float mx = -INFINITY;
+      const int j_cur = j_next;
+      if (n + 1 < kc) j_next = clist[n + 1];
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(lane_addr + b * 64 + g * 32, sv);
+        tmem_wait_ld();
+        const int valid = min(64, a.N - j_cur * 64) - g * 32;  // valid columns in this half
+        if (valid < 32) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
+          for (int c = 0; c < 32; ++c)
+            if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
+        }
+        mx = __uint_as_float(sv[0]);
+#pragma unroll
+        for (int c = 1; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
       }
-      float mx = __uint_as_float(sv[0]);
-#pragma unroll
-      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
-      mx *= sc;
+      red_max[b][g][r] = mx;
+      wg_barrier();
+      if (!ok) continue;
+      mx = fmaxf(mx, red_max[b][g ^ 1][r]) * sc;
       if (n == 0) {
         m_run = mx;
       } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
-        // The running maximum grew by more than 2^8: rescale O_s (needs PV_{n-1} finished).
+        // The running maximum grew by more than 2^8: rescale this half of O_s (needs PV_{n-1}
+        // finished). The partner thread of the row takes the same decision from the same values.
         ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, &abort_flag));
-        if (!ok) break;
+        if (!ok) continue;
         tc_fence_after();
         const float m_new = fmaxf(m_run, mx);
         const float f = fast_exp2(m_run - m_new);
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + OS + c0, o);
+        for (int c0 = 0; c0 < D / 2; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(lane_addr + OS + g * (D / 2) + c0, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-          tmem_st32(lane_addr + OS + c0, o);
+          for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+          tmem_st16(lane_addr + OS + g * (D / 2) + c0, o);
         }
         tmem_wait_st();
         l_run *= f;
@@ -281,9 +298,9 @@ __global__ void __launch_bounds__(192, 2)
       }
       // p = 2^(s * scale - m): one FMA and one exponential per element
       float ps0 = 0.f, ps1 = 0.f;
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
+      for (int c = 0; c < 32; c += 2) {
         const float e0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sc, -m_run));
         const float e1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sc, -m_run));
         ps0 += e0;
@@ -291,7 +308,7 @@ __global__ void __launch_bounds__(192, 2)
         pk[c >> 1] = pack_bf16x2(e0, e1);
       }
       l_run += ps0 + ps1;
-      tmem_st32(lane_addr + b * 64, pk);  // P_n over the first 32 columns of S_n
+      tmem_st16(lane_addr + b * 64 + g * 16, pk);  // this half of P_n over the S_n columns
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
@@ -301,12 +318,12 @@ __global__ void __launch_bounds__(192, 2)
       ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(kc - 1) & 1], ((kc - 1) >> 1) & 1, a.err, &abort_flag));
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, a.err, &abort_flag));
 
-    // phi(Q) in place (bf16), and the linear-branch denominator phi(q) . Z_i with the
-    // same rounded phi(q) the MMA sees.
+    // phi(Q) in place (bf16) over this half of the row, and this half of the linear-branch
+    // denominator phi(q) . Z_i with the same rounded phi(q) the MMA sees.
     float den = 0.f;
     if (ok) {
-#pragma unroll 4
-      for (int c8 = 0; c8 < D / 8; ++c8) {
+#pragma unroll 2
+      for (int c8 = g * (D / 16); c8 < (g + 1) * (D / 16); ++c8) {
         uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
         uint4 u = *p;
         uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -324,25 +341,30 @@ __global__ void __launch_bounds__(192, 2)
       }
       fence_proxy_async_smem();
     }
+    red_l[g][r] = l_run;
+    red_den[g][r] = den;
     tc_fence_before();
     mbar_arrive(&phiq_full);
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, 0, a.err, &abort_flag));
+    wg_barrier();  // both halves' row sums and denominators are in shared memory
+    const float l_tot = red_l[0][r] + red_l[1][r];
+    const float den_tot = red_den[0][r] + red_den[1][r];
 
     // Epilogue: O = alpha * O_s / l + (1 - alpha) * O_l / den -> bf16 staging (reuses sQ) -> TMA store.
     const uint32_t box_bytes = static_cast<uint32_t>(a.block_q) * 128u;
     if (ok) {
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      const float inv_d = den > 0.f ? 1.f / den : 0.f;
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float inv_d = den_tot > 0.f ? 1.f / den_tot : 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t os[32], ol[32];
-        tmem_ld32(lane_addr + OS + c0, os);
-        tmem_ld32(lane_addr + OL + c0, ol);
+      for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 16) {
+        uint32_t os[16], ol[16];
+        tmem_ld16(lane_addr + OS + c0, os);
+        tmem_ld16(lane_addr + OL + c0, ol);
         tmem_wait_ld();
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
+        for (int c = 0; c < 16; c += 2) {
           const float al0 = sAlpha[c0 + c], al1 = sAlpha[c0 + c + 1];
           const float y0 = al0 * (kc > 0 ? __uint_as_float(os[c]) * inv_l : 0.f) +
                            (1.f - al0) * (__uint_as_float(ol[c]) * inv_d);
@@ -353,7 +375,7 @@ __global__ void __launch_bounds__(192, 2)
         if (r < a.block_q) {
           uint8_t* box = sQ + (c0 >> 6) * box_bytes;
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+          for (int q = 0; q < 2; ++q)
             *reinterpret_cast<uint4*>(box + sw128_offset(r, ((c0 & 63) >> 3) * 16 + q * 16)) =
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
         }
@@ -364,7 +386,7 @@ __global__ void __launch_bounds__(192, 2)
     if (wt == 0 && !abort_flag) {
       for (int bcol = 0; bcol < DB; ++bcol) tma_store_3d(&map_o, sQ + bcol * box_bytes, bcol * 64, i * a.block_q, bh);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();  // shared memory may be released once the store has read it
     }
   }
   tc_fence_before();

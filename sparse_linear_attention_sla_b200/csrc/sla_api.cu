@@ -325,7 +325,7 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.alpha = alpha;
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   a.err = w.err;
-  sla::attn_kernel<D><<<dim3(s.Nq, s.BH), 192, smem, st>>>(mq, mk, mv, mh, mo, a);
+  sla::attn_kernel<D><<<dim3(s.Nq, s.BH), 320, smem, st>>>(mq, mk, mv, mh, mo, a);
   return launched("attn_kernel");
 }
 
