@@ -1,5 +1,5 @@
-// Fused SLA attention tile: one CTA computes the output of one query block
-// (128 query rows) of one (batch, head):
+// Fused SLA attention: each output tile is one query block (128 query rows) of
+// one (batch, head):
 //
 //   sparse branch  O_s = softmax over the keys of the critical KV blocks only
 //                        (online softmax, renormalised over that set)
@@ -14,23 +14,24 @@
 // item 1 (the sparse branch renormalises over its keys) and §2.A
 // (O = alpha * O_s + (1 - alpha) * O_l).
 //
-// Two CTAs share an SM (<= 98 KB shared memory, 256 TMEM columns and <= 96
-// registers per thread each), so one CTA's softmax overlaps the other's MMAs.
-// Warp roles (320 threads):
-//   warp 0      TMA producer: Q tile, then K_j / V_j of every critical block j
-//               through a 2-slot ring, then H_i into the next free slot.
+// Persistent: two CTAs per SM (<= 98 KB shared memory, 256 TMEM columns, <= 96
+// registers per thread each) walk the tiles t = blockIdx.x, blockIdx.x +
+// gridDim.x, ... in head-major order, so a head's K/V stay in L2 and the next
+// tile's loads overlap the current tile's epilogue. Warp roles (320 threads):
+//   warp 0      TMA producer: per tile Q, then K_j / V_j of every critical block
+//               through a 2-slot ring, then H_i into the next slot (a pseudo-block
+//               of the ring: its two halves complete the slot's K and V barriers).
 //   warp 1      TMEM owner and single-thread tcgen05 issuer:
-//               S = Q K_j^T (M=128, N=64, both operands in shared memory),
-//               O_s += P V_j (M=128, N=D, P read from TMEM),
-//               O_l = phi(Q) H_i (M=128, N=D).
+//               S = Q K_j^T (M=128, N=64), O_s += P V_j (M=128, N=D, P read from
+//               TMEM), O_l = phi(Q) H_i (M=128, N=D).
 //   warps 2..9  two softmax / epilogue warpgroups: a thread owns one query row
 //               (= TMEM lane) and one half of the columns; the two threads of a
 //               row exchange their block maxima through shared memory.
 //
 // TMEM columns: S ping-pong [0,64) [64,128) (P, bf16, is written back over the
-// first 32 columns of its S), O_s [128,128+D); after the sparse loop O_l
-// reuses [0,D). tcgen05 MMAs issued by one thread run in order, so S_{n+2}
-// never overwrites P_n before PV_n has read it.
+// first 32 columns of its S), O_s [128,128+D); after a tile's sparse loop O_l
+// reuses [0,D) until the epilogue has read it. tcgen05 MMAs issued by one thread
+// run in order, so S_{n+2} never overwrites P_n before PV_n has read it.
 // An empty critical set gives O_s = 0; an empty marginal set gives Z_i = 0 and O_l = 0.
 #pragma once
 
@@ -39,12 +40,13 @@
 namespace sla {
 
 struct AttnArgs {
-  int H, N, Nq, block_q;
+  int H, N, Nq, block_q, n_tiles;
   const int32_t* crit;      // [BH*Nq, crit_ld] critical KV block indices, ascending
   int crit_ld;
   const int32_t* crit_cnt;  // [BH*Nq]
   const float* Zagg;        // [BH*Nq, D]
   const float* alpha;       // [H, D]
+  __nv_bfloat16* out;       // [BH, N, D]
   float scale_log2;         // log2(e) / sqrt(D)
   uint32_t* err;
 };
@@ -55,12 +57,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Named barrier over the two softmax warpgroups (256 threads).
-__device__ __forceinline__ void wg_barrier() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
 template <int D>
 struct AttnSmem {
-  static constexpr uint32_t Q = 128 * D * 2;       // Q tile (later phi(Q), then the output staging)
+  static constexpr uint32_t Q = 128 * D * 2;       // Q tile (rewritten as phi(Q) at the end of a tile)
   static constexpr uint32_t KV = 64 * D * 2;       // one K or one V tile
   static constexpr uint32_t SLOT = 2 * KV;         // one ring slot: K then V (or the H_i tile)
   static constexpr uint32_t HT = D * D * 2;        // H_i tile
@@ -71,8 +70,7 @@ struct AttnSmem {
 template <int D>
 __global__ void __launch_bounds__(320, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
-                const __grid_constant__ CUtensorMap map_o, AttnArgs a) {
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h, AttnArgs a) {
   using L = AttnSmem<D>;
   constexpr int DB = D / 64;  // 64-column boxes per row
   constexpr uint32_t TMEM_COLS = 256;
@@ -82,7 +80,7 @@ __global__ void __launch_bounds__(320, 2)
   uint8_t* sQ = base;
   uint8_t* sRing = sQ + L::Q;  // slot s at sRing + s * SLOT: K at +0, V at +KV
 
-  __shared__ uint64_t q_full, h_full, phiq_full, ol_done, drain;
+  __shared__ uint64_t q_full, q_free, phiq_full, ol_done, tmem_free, drain;
   __shared__ uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base_sh;
@@ -92,17 +90,13 @@ __global__ void __launch_bounds__(320, 2)
   __shared__ float red_l[2][128], red_den[2][128];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i = blockIdx.x, bh = blockIdx.y, h = bh % a.H;
-  const int row_id = bh * a.Nq + i;
-  const int kc = a.crit_cnt[row_id];
-  const int32_t* clist = a.crit + static_cast<size_t>(row_id) * a.crit_ld;
-  const int hslot = kc & 1;  // ring slot that receives H_i after the last K/V block
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
-    mbar_init(&h_full, 1);
+    mbar_init(&q_free, 1);
     mbar_init(&phiq_full, 256);
     mbar_init(&ol_done, 1);
+    mbar_init(&tmem_free, 256);
     mbar_init(&drain, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
@@ -131,40 +125,53 @@ __global__ void __launch_bounds__(320, 2)
       prefetch_tmap(&map_k);
       prefetch_tmap(&map_v);
       prefetch_tmap(&map_h);
-      mbar_arrive_expect_tx(&q_full, L::Q);
-      for (int b = 0; b < DB; ++b) tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * a.block_q, bh);
       int k_round[2] = {-1, -1}, v_round[2] = {-1, -1};
-      bool h_issued = false;
+      int q_loads = 0;
+      uint32_t nb = 0;  // ring uses so far (K/V blocks and H_i pseudo-blocks)
       bool ok = true;
-      for (int n = 0; n < kc && ok; ++n) {
-        const int s = n & 1, r = n >> 1;
-        const int j = clist[n];
-        uint8_t* slot = sRing + s * L::SLOT;
-        if (r > 0 && !(ok = mbar_wait(&k_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
-        mbar_arrive_expect_tx(&k_full[s], L::KV);
-        for (int b = 0; b < DB; ++b) tma_load_3d(slot + b * 8192, &map_k, &k_full[s], b * 64, j * 64, bh);
-        k_round[s] = r;
-        if (r > 0 && !(ok = mbar_wait(&v_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
-        mbar_arrive_expect_tx(&v_full[s], L::KV);
-        for (int b = 0; b < DB; ++b) tma_load_3d(slot + L::KV + b * 8192, &map_v, &v_full[s], b * 64, j * 64, bh);
-        v_round[s] = r;
-      }
-      if (ok) {  // H_i goes into the slot the next block would have used
-        const int r = kc >> 1;
-        if (r > 0) ok = mbar_wait(&k_empty[hslot], (r - 1) & 1, a.err, &abort_flag) &&
-                        mbar_wait(&v_empty[hslot], (r - 1) & 1, a.err, &abort_flag);
-        if (ok) {
-          uint8_t* slot = sRing + hslot * L::SLOT;
-          mbar_arrive_expect_tx(&h_full, L::HT);
-          for (int dh = 0; dh < DB; ++dh)
-            for (int eh = 0; eh < DB; ++eh)
-              tma_load_2d(slot + (dh * DB + eh) * 8192, &map_h, &h_full, eh * 64, row_id * D + dh * 64);
-          h_issued = true;
+      int k = 0;
+      for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
+        const int bh = t / a.Nq, i = t % a.Nq;
+        const int kc = a.crit_cnt[t];
+        const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
+        if (k > 0 && !(ok = mbar_wait(&q_free, (k - 1) & 1, a.err, &abort_flag))) break;
+        mbar_arrive_expect_tx(&q_full, L::Q);
+        for (int b = 0; b < DB; ++b) tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * a.block_q, bh);
+        ++q_loads;
+        for (int n = 0; n <= kc; ++n, ++nb) {  // n == kc is the H_i pseudo-block
+          const int s = nb & 1, r = nb >> 1;
+          uint8_t* slot = sRing + s * L::SLOT;
+          // The K half is refilled as soon as S of its previous block is done, the V half
+          // once P*V of its previous block is done.
+          if (r > 0 && !(ok = mbar_wait(&k_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
+          const int j = n < kc ? clist[n] : 0;
+          if (n < kc) {
+            mbar_arrive_expect_tx(&k_full[s], L::KV);
+            for (int b = 0; b < DB; ++b) tma_load_3d(slot + b * 8192, &map_k, &k_full[s], b * 64, j * 64, bh);
+          } else if (D == 128) {  // H_i rows 0..63 land in the K half, rows 64..127 in the V half
+            mbar_arrive_expect_tx(&k_full[s], L::KV);
+            for (int eh = 0; eh < 2; ++eh) tma_load_2d(slot + eh * 8192, &map_h, &k_full[s], eh * 64, t * D);
+          } else {
+            mbar_arrive_expect_tx(&k_full[s], L::HT);
+            tma_load_2d(slot, &map_h, &k_full[s], 0, t * D);
+          }
+          k_round[s] = r;
+          if (r > 0 && !(ok = mbar_wait(&v_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
+          if (n < kc) {
+            mbar_arrive_expect_tx(&v_full[s], L::KV);
+            for (int b = 0; b < DB; ++b) tma_load_3d(slot + L::KV + b * 8192, &map_v, &v_full[s], b * 64, j * 64, bh);
+          } else if (D == 128) {
+            mbar_arrive_expect_tx(&v_full[s], L::KV);
+            for (int eh = 0; eh < 2; ++eh)
+              tma_load_2d(slot + L::KV + eh * 8192, &map_h, &v_full[s], eh * 64, t * D + 64);
+          } else {
+            mbar_arrive(&v_full[s]);
+          }
+          v_round[s] = r;
         }
       }
       if (abort_flag) {  // let every load still in flight land before the CTA retires
-        mbar_wait(&q_full, 0, nullptr, nullptr);
-        if (h_issued) mbar_wait(&h_full, 0, nullptr, nullptr);
+        if (q_loads > 0) mbar_wait(&q_full, (q_loads - 1) & 1, nullptr, nullptr);
         for (int s = 0; s < 2; ++s) {
           if (k_round[s] >= 0) mbar_wait(&k_full[s], k_round[s] & 1, nullptr, nullptr);
           if (v_round[s] >= 0) mbar_wait(&v_full[s], v_round[s] & 1, nullptr, nullptr);
@@ -178,44 +185,54 @@ __global__ void __launch_bounds__(320, 2)
       const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);
       const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing);
-      bool ok = mbar_wait(&q_full, 0, a.err, &abort_flag);
-      auto issue_pv = [&](int m) -> bool {
-        const int s = m & 1;
-        if (!mbar_wait(&p_full[s], (m >> 1) & 1, a.err, &abort_flag)) return false;
-        if (!mbar_wait(&v_full[s], (m >> 1) & 1, a.err, &abort_flag)) return false;
+      uint32_t nb = 0, ns = 0;  // ring uses, S/P blocks
+      bool ok = true;
+      // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites O_s.
+      auto issue_pv = [&](uint32_t nbm, uint32_t nsm, bool first) -> bool {
+        const int s = nbm & 1, b = nsm & 1;
+        if (!mbar_wait(&p_full[b], (nsm >> 1) & 1, a.err, &abort_flag)) return false;
+        if (!mbar_wait(&v_full[s], (nbm >> 1) & 1, a.err, &abort_flag)) return false;
         tc_fence_after();
         const uint32_t vb = ring0 + s * L::SLOT + L::KV;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = smem_desc_sw128(vb + kk * 2048, 8192, 1024);
-          umma_bf16_ts(tmem + OS, tmem + s * 64 + kk * 8, bd, id_o, (m > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + OS, tmem + b * 64 + kk * 8, bd, id_o, (first && kk == 0) ? 0u : 1u);
         }
-        umma_commit(&pv_done[s]);
+        umma_commit(&pv_done[b]);
         umma_commit(&v_empty[s]);
         return true;
       };
-      for (int n = 0; ok && n < kc; ++n) {
-        const int s = n & 1;
-        if (!mbar_wait(&k_full[s], (n >> 1) & 1, a.err, &abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = ring0 + s * L::SLOT;
+      int k = 0;
+      for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
+        const int kc = a.crit_cnt[t];
+        if (!(ok = mbar_wait(&q_full, k & 1, a.err, &abort_flag))) break;
+        // the epilogue of the previous tile has read O_s and O_l out of TMEM
+        if (k > 0 && !(ok = mbar_wait(&tmem_free, (k - 1) & 1, a.err, &abort_flag))) break;
+        for (int n = 0; n < kc; ++n, ++nb, ++ns) {
+          const int s = nb & 1, b = ns & 1;
+          if (!(ok = mbar_wait(&k_full[s], (nb >> 1) & 1, a.err, &abort_flag))) break;
+          tc_fence_after();
+          const uint32_t kb = ring0 + s * L::SLOT;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(tmem + s * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+            umma_bf16_ss(tmem + b * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[b]);
+          umma_commit(&k_empty[s]);
+          if (n >= 1 && !(ok = issue_pv(nb - 1, ns - 1, n == 1))) break;
         }
-        umma_commit(&s_full[s]);
-        umma_commit(&k_empty[s]);
-        if (n >= 1 && !issue_pv(n - 1)) { ok = false; break; }
-      }
-      if (ok && kc > 0) ok = issue_pv(kc - 1);
-      // linear branch: O_l = phi(Q) H_i once the warpgroup has rewritten Q as phi(Q)
-      if (ok) ok = mbar_wait(&h_full, 0, a.err, &abort_flag);
-      if (ok) ok = mbar_wait(&phiq_full, 0, a.err, &abort_flag);
-      if (ok) {
+        if (!ok) break;
+        if (kc > 0 && !(ok = issue_pv(nb - 1, ns - 1, kc == 1))) break;
+        // linear branch: O_l = phi(Q) H_i once H_i has landed and the warpgroups rewrote Q as phi(Q)
+        const int s = nb & 1;
+        if (!(ok = mbar_wait(&k_full[s], (nb >> 1) & 1, a.err, &abort_flag))) break;
+        if (!(ok = mbar_wait(&v_full[s], (nb >> 1) & 1, a.err, &abort_flag))) break;
+        if (!(ok = mbar_wait(&phiq_full, k & 1, a.err, &abort_flag))) break;
         tc_fence_after();
-        const uint32_t hb = ring0 + hslot * L::SLOT;
+        const uint32_t hb = ring0 + s * L::SLOT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
@@ -223,6 +240,10 @@ __global__ void __launch_bounds__(320, 2)
           umma_bf16_ss(tmem + OL, ad, bd, id_o, kk > 0 ? 1u : 0u);
         }
         umma_commit(&ol_done);
+        umma_commit(&q_free);
+        umma_commit(&k_empty[s]);
+        umma_commit(&v_empty[s]);
+        ++nb;
       }
       umma_commit(&drain);  // every MMA issued above has finished once this arrives
       mbar_wait(&drain, 0, nullptr, nullptr);
@@ -235,127 +256,132 @@ __global__ void __launch_bounds__(320, 2)
     const int quarter = warp & 3;               // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;          // query row within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    for (int c = wt; c < D; c += 256) {
-      sZ[c] = a.Zagg[static_cast<size_t>(row_id) * D + c];
-      sAlpha[c] = a.alpha[h * D + c];
-    }
-    wg_barrier();
-
     const float sc = a.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and this half's row sum
+    uint32_t ns = 0;  // S/P blocks so far
     bool ok = true;
-    int j_next = kc > 0 ? clist[0] : 0;  // critical-block index, read one iteration ahead
-    // Every warp of both warpgroups runs every iteration and reaches every named barrier,
-    // also after a failed wait (then the work is skipped), so a barrier can never wait for a
-    // warp that has left the loop.
-    for (int n = 0; n < kc; ++n) {
-      const int b = n & 1;
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (n >> 1) & 1, a.err, &abort_flag));
-      uint32_t sv[32];
-      float mx = -INFINITY;
-      const int j_cur = j_next;
-      if (n + 1 < kc) j_next = clist[n + 1];
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32(lane_addr + b * 64 + g * 32, sv);
-        tmem_wait_ld();
-        const int valid = min(64, a.N - j_cur * 64) - g * 32;  // valid columns in this half
-        if (valid < 32) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
-        }
-        mx = __uint_as_float(sv[0]);
-#pragma unroll
-        for (int c = 1; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+    int k = 0;
+    // Every barrier between the two warpgroups ANDs the threads' status, so a failed
+    // wait makes all 256 threads leave together.
+    for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++k) {
+      const int bh = t / a.Nq, i = t % a.Nq, h = bh % a.H;
+      const int kc = a.crit_cnt[t];
+      const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
+      if (!named_barrier_and(1, 256, ok)) break;  // the previous tile's epilogue is done with sZ / sAlpha
+      for (int c = wt; c < D; c += 256) {
+        sZ[c] = a.Zagg[static_cast<size_t>(t) * D + c];
+        sAlpha[c] = a.alpha[h * D + c];
       }
-      red_max[b][g][r] = mx;
-      wg_barrier();
-      if (!ok) continue;
-      mx = fmaxf(mx, red_max[b][g ^ 1][r]) * sc;
-      if (n == 0) {
-        m_run = mx;
-      } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
-        // The running maximum grew by more than 2^8: rescale this half of O_s (needs PV_{n-1}
-        // finished). The partner thread of the row takes the same decision from the same values.
-        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, a.err, &abort_flag));
-        if (!ok) continue;
-        tc_fence_after();
-        const float m_new = fmaxf(m_run, mx);
-        const float f = fast_exp2(m_run - m_new);
-#pragma unroll
-        for (int c0 = 0; c0 < D / 2; c0 += 16) {
-          uint32_t o[16];
-          tmem_ld16(lane_addr + OS + g * (D / 2) + c0, o);
+      if (!named_barrier_and(1, 256, ok)) break;  // sZ / sAlpha of this tile are visible
+      float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and this half's row sum
+      int j_next = kc > 0 ? clist[0] : 0;   // critical-block index, read one iteration ahead
+      for (int n = 0; n < kc; ++n, ++ns) {
+        const int b = ns & 1;
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[b], (ns >> 1) & 1, a.err, &abort_flag));
+        uint32_t sv[32];
+        float mx = -INFINITY;
+        const int j_cur = j_next;
+        if (n + 1 < kc) j_next = clist[n + 1];
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32(lane_addr + b * 64 + g * 32, sv);
           tmem_wait_ld();
+          const int valid = min(64, a.N - j_cur * 64) - g * 32;  // valid columns in this half
+          if (valid < 32) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-          tmem_st16(lane_addr + OS + g * (D / 2) + c0, o);
+            for (int c = 0; c < 32; ++c)
+              if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
+          }
+          mx = __uint_as_float(sv[0]);
+#pragma unroll
+          for (int c = 1; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
         }
+        red_max[b][g][r] = mx;
+        if (!(ok = named_barrier_and(1, 256, ok))) break;
+        mx = fmaxf(mx, red_max[b][g ^ 1][r]) * sc;
+        if (n == 0) {
+          m_run = mx;
+        } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
+          // The running maximum grew by more than 2^8: rescale this half of O_s (needs PV of
+          // the previous block finished). The partner thread of the row decides identically.
+          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
+          if (!ok) continue;  // the next barrier takes every thread out
+          tc_fence_after();
+          const float m_new = fmaxf(m_run, mx);
+          const float f = fast_exp2(m_run - m_new);
+#pragma unroll
+          for (int c0 = 0; c0 < D / 2; c0 += 16) {
+            uint32_t o[16];
+            tmem_ld16(lane_addr + OS + g * (D / 2) + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+            tmem_st16(lane_addr + OS + g * (D / 2) + c0, o);
+          }
+          tmem_wait_st();
+          l_run *= f;
+          m_run = m_new;
+        }
+        // p = 2^(s * scale - m): one FMA and one exponential per element
+        float ps0 = 0.f, ps1 = 0.f;
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float e0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sc, -m_run));
+          const float e1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sc, -m_run));
+          ps0 += e0;
+          ps1 += e1;
+          pk[c >> 1] = pack_bf16x2(e0, e1);
+        }
+        l_run += ps0 + ps1;
+        tmem_st16(lane_addr + b * 64 + g * 16, pk);  // this half of P over the S columns
         tmem_wait_st();
-        l_run *= f;
-        m_run = m_new;
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
       }
-      // p = 2^(s * scale - m): one FMA and one exponential per element
-      float ps0 = 0.f, ps1 = 0.f;
-      uint32_t pk[16];
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float e0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sc, -m_run));
-        const float e1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sc, -m_run));
-        ps0 += e0;
-        ps1 += e1;
-        pk[c >> 1] = pack_bf16x2(e0, e1);
-      }
-      l_run += ps0 + ps1;
-      tmem_st16(lane_addr + b * 64 + g * 16, pk);  // this half of P_n over the S_n columns
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[b]);
-    }
-    // Every MMA that reads Q (or the S/P columns) has finished once the last PV has.
-    if (ok && kc > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(kc - 1) & 1], ((kc - 1) >> 1) & 1, a.err, &abort_flag));
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, 0, a.err, &abort_flag));
+      // Every MMA that reads Q (or the S/P columns) has finished once the last PV has.
+      if (ok && kc > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, k & 1, a.err, &abort_flag));
 
-    // phi(Q) in place (bf16) over this half of the row, and this half of the linear-branch
-    // denominator phi(q) . Z_i with the same rounded phi(q) the MMA sees.
-    float den = 0.f;
-    if (ok) {
+      // phi(Q) in place (bf16) over this half of the row, and this half of the linear-branch
+      // denominator phi(q) . Z_i with the same rounded phi(q) the MMA sees.
+      float den = 0.f;
+      if (ok) {
 #pragma unroll 2
-      for (int c8 = g * (D / 16); c8 < (g + 1) * (D / 16); ++c8) {
-        uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
-        uint4 u = *p;
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        for (int c8 = g * (D / 16); c8 < (g + 1) * (D / 16); ++c8) {
+          uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
+          uint4 u = *p;
+          uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float2 f = unpack_bf16x2(w[e]);
-          const float g0 = f.x > 0.f ? f.x + 1.f : __expf(f.x);
-          const float g1 = f.y > 0.f ? f.y + 1.f : __expf(f.y);
-          w[e] = pack_bf16x2(g0, g1);
-          const float2 gr = unpack_bf16x2(w[e]);
-          den = fmaf(gr.x, sZ[c8 * 8 + 2 * e], den);
-          den = fmaf(gr.y, sZ[c8 * 8 + 2 * e + 1], den);
+          for (int e = 0; e < 4; ++e) {
+            float2 f = unpack_bf16x2(w[e]);
+            const float g0 = f.x > 0.f ? f.x + 1.f : __expf(f.x);
+            const float g1 = f.y > 0.f ? f.y + 1.f : __expf(f.y);
+            w[e] = pack_bf16x2(g0, g1);
+            const float2 gr = unpack_bf16x2(w[e]);
+            den = fmaf(gr.x, sZ[c8 * 8 + 2 * e], den);
+            den = fmaf(gr.y, sZ[c8 * 8 + 2 * e + 1], den);
+          }
+          *p = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        *p = make_uint4(w[0], w[1], w[2], w[3]);
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-    }
-    red_l[g][r] = l_run;
-    red_den[g][r] = den;
-    tc_fence_before();
-    mbar_arrive(&phiq_full);
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, 0, a.err, &abort_flag));
-    wg_barrier();  // both halves' row sums and denominators are in shared memory
-    const float l_tot = red_l[0][r] + red_l[1][r];
-    const float den_tot = red_den[0][r] + red_den[1][r];
+      red_l[g][r] = l_run;
+      red_den[g][r] = den;
+      tc_fence_before();
+      mbar_arrive(&phiq_full);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, k & 1, a.err, &abort_flag));
+      if (!(ok = named_barrier_and(1, 256, ok))) break;  // both halves' sums are in shared memory
+      const float l_tot = red_l[0][r] + red_l[1][r];
+      const float den_tot = red_den[0][r] + red_den[1][r];
 
-    // Epilogue: O = alpha * O_s / l + (1 - alpha) * O_l / den -> bf16 staging (reuses sQ) -> TMA store.
-    const uint32_t box_bytes = static_cast<uint32_t>(a.block_q) * 128u;
-    if (ok) {
+      // Epilogue: O = alpha * O_s / l + (1 - alpha) * O_l / den, bf16, straight to global memory.
       tc_fence_after();
       const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
       const float inv_d = den_tot > 0.f ? 1.f / den_tot : 0.f;
+      const int tok = i * a.block_q + r;
+      const bool store = r < a.block_q && tok < a.N;
+      __nv_bfloat16* orow = a.out + (static_cast<size_t>(bh) * a.N + tok) * D;
 #pragma unroll 1
       for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 16) {
         uint32_t os[16], ol[16];
@@ -372,21 +398,14 @@ __global__ void __launch_bounds__(320, 2)
                            (1.f - al1) * (__uint_as_float(ol[c + 1]) * inv_d);
           pk[c >> 1] = pack_bf16x2(y0, y1);
         }
-        if (r < a.block_q) {
-          uint8_t* box = sQ + (c0 >> 6) * box_bytes;
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-            *reinterpret_cast<uint4*>(box + sw128_offset(r, ((c0 & 63) >> 3) * 16 + q * 16)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      fence_proxy_async_smem();
-    }
-    wg_barrier();
-    if (wt == 0 && !abort_flag) {
-      for (int bcol = 0; bcol < DB; ++bcol) tma_store_3d(&map_o, sQ + bcol * box_bytes, bcol * 64, i * a.block_q, bh);
-      tma_store_commit();
-      tma_store_wait_read();  // shared memory may be released once the store has read it
+      tc_fence_before();
+      mbar_arrive(&tmem_free);  // O_s and O_l have left TMEM: the next tile may overwrite them
     }
   }
   tc_fence_before();

@@ -300,11 +300,10 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
 template <int D>
 sla_status launch_attn(const Shape& s, const void* q, const void* k, const void* v, const float* alpha, void* out,
                        const Workspace& w, int crit_ld, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mh, mo;
+  CUtensorMap mq, mk, mv, mh;
   SLA_TRY(act_map(&mq, q, s, 128));
   SLA_TRY(act_map(&mk, k, s, 64));
   SLA_TRY(act_map(&mv, v, s, 64));
-  SLA_TRY(act_map(&mo, out, s, static_cast<uint32_t>(s.bq)));
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.BH) * s.Nq * s.D};
     const uint64_t strides[1] = {static_cast<uint64_t>(s.D)};
@@ -318,14 +317,18 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.N = s.N;
   a.Nq = s.Nq;
   a.block_q = s.bq;
+  a.n_tiles = s.BH * s.Nq;
   a.crit = w.crit;
   a.crit_ld = crit_ld;
   a.crit_cnt = w.crit_cnt;
   a.Zagg = w.Zagg;
   a.alpha = alpha;
+  a.out = static_cast<__nv_bfloat16*>(out);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   a.err = w.err;
-  sla::attn_kernel<D><<<dim3(s.Nq, s.BH), 320, smem, st>>>(mq, mk, mv, mh, mo, a);
+  // persistent: two CTAs per SM walk the tiles
+  const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
+  sla::attn_kernel<D><<<grid, 320, smem, st>>>(mq, mk, mv, mh, a);
   return launched("attn_kernel");
 }
 
