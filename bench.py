@@ -38,7 +38,7 @@ METRIC = "effective attention TFLOPS and ms/call at 1 B200; fraction of roofline
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "wan13b_b1h12_n32760_d128"
 FLUSH_BYTES = 512 << 20
-LAUNCHES_PER_FORWARD = 6  # pool, kv_prep, scores, select, aggregate, attention
+LAUNCHES_PER_FORWARD = 5  # precompute, scores, select, aggregate, attention
 
 
 def parse_args(argv=None):

@@ -56,10 +56,11 @@ __global__ void __launch_bounds__(128) pool_mean_kernel(const __nv_bfloat16* __r
   }
 }
 
-// ---------------------------------------------------------------- KV states
-struct KvPrepArgs {
-  int BH, N, Nk;
-  double* kbar;            // [BH, Nk, D] (nullable)
+// ---------------------------------------------------------------- fused precompute
+struct PrepArgs {
+  int BH, N, Nq, Nk, block_q;
+  double* qbar;            // [BH, Nq, D] query-block means (nullable: no query pooling)
+  double* kbar;            // [BH, Nk, D] KV-block means (nullable)
   __nv_bfloat16* hst;      // [BH, Nk, LD] bf16: h_j row-major (D*D) then z_j (D) then zero pad (forward)
   float* h32;              // [BH, Nk, D, D] fp32 (state export), used when hst == nullptr
   float* z32;              // [BH, Nk, D] fp32 (state export)
@@ -68,225 +69,314 @@ struct KvPrepArgs {
 };
 
 template <int D>
-struct KvPrepSmem {
-  static constexpr uint32_t SLOT = 32768;               // K (16 KB, zero upper half when D = 64) + V (16 KB)
-  static constexpr uint32_t STAGE = D * 128 * (D / 64); // bf16 h_j staging for the TMA store
-  static constexpr uint32_t total() { return 2 * SLOT + STAGE + 1024; }
+struct PrepSmem {
+  static constexpr int NSLOT = 4;
+  static constexpr uint32_t SLOT = 32768;                // K (16 KB) then V (16 KB), or one query block
+  static constexpr uint32_t STAGE = D * 128 * (D / 64);  // bf16 h_j tile for the TMA store
+  static constexpr uint32_t ZERO = D == 64 ? 8192 : 0;   // zero rows 64..127 of phi(K)^T when D = 64
+  static constexpr uint32_t total() { return NSLOT * SLOT + 2 * STAGE + ZERO + 1024; }
 };
 
-// One CTA walks over KV blocks g = blockIdx.x, blockIdx.x + gridDim.x, ... with a
-// two-slot TMA ring; two CTAs share an SM. 128 threads.
-//   column pass  16-byte vectors: sum k (fp64) and phi(k) (fp32) per column, and
-//                rewrite the K tile in place as phi(k) (zero past the sequence end)
-//   MMA          h_j = phi(K_j)^T V_j on tcgen05 (M=128, N=D, K=64 tokens; both
-//                operands MN-major); for D = 64 rows 64..127 of phi(K)^T read zeros
-//   epilogue     bf16 h_j staged in shared memory and written by one TMA store
-//                (forward), or fp32 straight from registers (state export).
+// Column pass of one warpgroup over a ROWS x D tile (16-byte chunks, 128-byte swizzle):
+// thread (cc, rg) owns columns 8cc..8cc+7 of rows rg, rg + RG, ...; it sums the valid
+// rows in fp64 and, for a K tile (PHI), sums phi(k) in fp32 and rewrites the tile in
+// place as phi(k) (zero past the sequence end). Partial sums go to part_d / part_f[rg].
+template <int D, int ROWS, bool PHI>
+__device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int valid, double (*part_d)[D],
+                                            float (*part_f)[D]) {
+  constexpr int RG = 128 / (D / 8);
+  uint8_t* tile = tile0 + (cc / 8) * (ROWS * 128);
+  const uint32_t cb = (cc % 8) * 16;
+  double ks[8];
+  float zs[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    ks[e] = 0.0;
+    zs[e] = 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < ROWS / RG; ++k) {
+    const int rr = rg + RG * k;
+    uint4* p = reinterpret_cast<uint4*>(tile + sw128_offset(rr, cb));
+    const uint4 u = *p;
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    const bool in = rr < valid;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = unpack_bf16x2(w[e]);
+      float f0 = 0.f, f1 = 0.f;
+      if (in) {
+        ks[2 * e] += static_cast<double>(x.x);
+        ks[2 * e + 1] += static_cast<double>(x.y);
+        if (PHI) {
+          f0 = phi_f(x.x);
+          f1 = phi_f(x.y);
+          zs[2 * e] += f0;
+          zs[2 * e + 1] += f1;
+        }
+      }
+      w[e] = pack_bf16x2(f0, f1);
+    }
+    if (PHI) *p = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    part_d[rg][cc * 8 + e] = ks[e];
+    part_f[rg][cc * 8 + e] = zs[e];
+  }
+}
+
+// Persistent, warp-specialised precompute; one CTA per SM, 448 threads.
+// A CTA walks the items g = blockIdx.x, blockIdx.x + gridDim.x, ... of the list
+// [KV blocks of every head | query blocks of every head (when qbar is set)].
+//   warp 0      TMA producer: K_j and V_j (or a query block) into a 4-slot ring
+//   warps 2..5 and 10..13
+//               two column-pass warpgroups taking alternate items: over 16-byte
+//               chunks, the sum of the valid rows in fp64 (block means), and for KV
+//               blocks the sum of phi(k) (z_j) while the K tile is rewritten in
+//               place as phi(k) (zero past the sequence end)
+//   warp 1      tcgen05 issuer: h_j = phi(K_j)^T V_j (M=128, N=D, K=64 tokens; both
+//               operands MN-major) into one of two TMEM accumulators
+//   warps 6..9  epilogue: TMEM -> bf16 -> one of two staging tiles -> TMA store (forward),
+//               or TMEM -> fp32 straight to global memory (state export)
+// For D = 64 the second half of phi(K)^T (rows 64..127 of the M=128 MMA) points
+// at a zero tile, so the result rows 64..127 are zero and ignored.
 template <int D>
-__global__ void __launch_bounds__(128, 2) kv_prep_kernel(const __grid_constant__ CUtensorMap map_k,
-                                                         const __grid_constant__ CUtensorMap map_v,
-                                                         const __grid_constant__ CUtensorMap map_hout, KvPrepArgs a) {
-  using L = KvPrepSmem<D>;
-  constexpr int BK = 64;
-  constexpr int KBOX = D / 64;              // 64-column boxes per row
-  constexpr uint32_t TX = BK * D * 2 * 2;   // K + V bytes per block
-  constexpr int CPR = D / 8;                // 16-byte chunks per row
-  constexpr int RG = 128 / CPR;             // row groups
-  constexpr int RPT = BK / RG;              // rows per thread
+__global__ void __launch_bounds__(448, 1)
+    prep_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_hout, PrepArgs a) {
+  using L = PrepSmem<D>;
+  constexpr int NS = L::NSLOT;
+  constexpr int KBOX = D / 64;  // 64-column boxes per row
+  constexpr int CPR = D / 8;    // 16-byte chunks per row
+  constexpr int RG = 128 / CPR; // row groups of the column pass
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* slot[2] = {smem, smem + L::SLOT};
-  uint8_t* stage = smem + 2 * L::SLOT;
-  __shared__ uint64_t bar_full[2], bar_mma;
+  uint8_t* stage0 = smem + NS * L::SLOT;
+  uint8_t* zero = stage0 + 2 * L::STAGE;
+  __shared__ uint64_t full[NS], phi_done[NS], empty[NS], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ double ksum_part[RG][D];
-  __shared__ float zsum_part[RG][D];
+  __shared__ double part_d[2][RG][D];
+  __shared__ float part_f[2][RG][D];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int total = a.BH * a.Nk;
+  const int n_kv = a.BH * a.Nk;
+  const int n_items = n_kv + (a.qbar ? a.BH * a.Nq : 0);
   const bool bf16_out = a.hst != nullptr;
   if (tid == 0) {
-    mbar_init(&bar_full[0], 1);
-    mbar_init(&bar_full[1], 1);
-    mbar_init(&bar_mma, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&phi_done[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&map_k);
-    prefetch_tmap(&map_v);
-    if (bf16_out) prefetch_tmap(&map_hout);
   }
-  if (D == 64) {  // zero the upper halves of both K areas once (TMA never writes them)
-    for (int s = 0; s < 2; ++s)
-      for (int o = tid * 16; o < 8192; o += 128 * 16) *reinterpret_cast<uint4*>(slot[s] + 8192 + o) = make_uint4(0, 0, 0, 0);
+  if (D == 64) {
+    for (uint32_t o = tid * 16; o < L::ZERO; o += 448 * 16) *reinterpret_cast<uint4*>(zero + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
-  if (warp == 0) {
-    tmem_alloc(&tmem_base_sh, 128);
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 256);
     tmem_relinquish();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  // Thread 0 tracks which slots have a load in flight (parity of its phase, or -1)
-  // so that an aborted CTA can let them land before it retires.
-  int inflight[2] = {-1, -1};
-  int mma_parity = -1;
-  auto issue_load = [&](int g, int s, int round) {
-    const int bh = g / a.Nk, j = g % a.Nk;
-    mbar_arrive_expect_tx(&bar_full[s], TX);
-#pragma unroll
-    for (int b = 0; b < KBOX; ++b) {
-      tma_load_3d(slot[s] + b * 8192, &map_k, &bar_full[s], b * 64, j * BK, bh);
-      tma_load_3d(slot[s] + 16384 + b * 8192, &map_v, &bar_full[s], b * 64, j * BK, bh);
-    }
-    inflight[s] = round & 1;
-  };
-  if (tid == 0) {
-    if (blockIdx.x < total) issue_load(blockIdx.x, 0, 0);
-    if (blockIdx.x + gridDim.x < total) issue_load(blockIdx.x + gridDim.x, 1, 0);
-  }
-  const uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
-  const int cc = tid % CPR, rg = tid / CPR;
-
-  int n = 0;
-  for (int g = blockIdx.x; g < total; g += gridDim.x, ++n) {
-    const int s = n & 1;
-    const int bh = g / a.Nk, j = g % a.Nk;
-    const int valid = min(BK, a.N - j * BK);
-    bool ok = mbar_wait(&bar_full[s], (n >> 1) & 1, a.err, &abort_flag);
-    if (__syncthreads_or(!ok)) break;
-    if (tid == 0) inflight[s] = -1;
-
-    // Column pass over 16-byte chunks: thread (cc, rg) owns columns 8cc..8cc+7 of rows rg + RG*k.
-    {
-      uint8_t* tile = slot[s] + (cc / 8) * 8192;
-      const uint32_t cb = (cc % 8) * 16;
-      double ks[8];
-      float zs[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        ks[e] = 0.0;
-        zs[e] = 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < RPT; ++k) {
-        const int r = rg + RG * k;
-        uint4* p = reinterpret_cast<uint4*>(tile + sw128_offset(r, cb));
-        const uint4 u = *p;
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        const bool in = r < valid;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 kv = unpack_bf16x2(w[e]);
-          float f0 = 0.f, f1 = 0.f;
-          if (in) {
-            ks[2 * e] += static_cast<double>(kv.x);
-            ks[2 * e + 1] += static_cast<double>(kv.y);
-            f0 = phi_f(kv.x);
-            f1 = phi_f(kv.y);
-            zs[2 * e] += f0;
-            zs[2 * e + 1] += f1;
-          }
-          w[e] = pack_bf16x2(f0, f1);
-        }
-        *p = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        ksum_part[rg][cc * 8 + e] = ks[e];
-        zsum_part[rg][cc * 8 + e] = zs[e];
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        uint64_t ad = smem_desc_sw128(smem_u32(slot[s]) + kk * 2048, 8192, 1024);
-        uint64_t bd = smem_desc_sw128(smem_u32(slot[s]) + 16384 + kk * 2048, 8192, 1024);
-        umma_bf16_ss(tmem, ad, bd, idesc, kk > 0);
-      }
-      umma_commit(&bar_mma);
-      mma_parity = n & 1;
-    }
-    // kbar and z while the MMA runs
-    if (tid < D) {
-      double ks = 0.0;
-      float zs = 0.f;
-#pragma unroll
-      for (int q = 0; q < RG; ++q) {
-        ks += ksum_part[q][tid];
-        zs += zsum_part[q][tid];
-      }
-      const size_t row = static_cast<size_t>(bh) * a.Nk + j;
-      if (a.kbar) a.kbar[row * D + tid] = ks / static_cast<double>(valid);
-      if (bf16_out) {
-        __nv_bfloat16* zr = a.hst + row * a.LD + D * D;
-        zr[tid] = __float2bfloat16_rn(zs);
-        if (D == 64) zr[64 + tid] = __float2bfloat16_rn(0.f);
-      } else if (a.z32) {
-        a.z32[row * D + tid] = zs;
-      }
-    }
-    ok = mbar_wait(&bar_mma, n & 1, a.err, &abort_flag);
-    if (tid == 0 && bf16_out) tma_store_wait_read();  // the previous block's store has left the staging tile
-    if (__syncthreads_or(!ok)) break;
-    tc_fence_after();
-    if (tid == 0) mma_parity = -1;
-    // The MMA has consumed slot s: refill it with the block two steps ahead.
-    if (tid == 0 && g + 2 * gridDim.x < total) issue_load(g + 2 * gridDim.x, s, (n >> 1) + 1);
-    // Epilogue: warp w holds rows d = 32 w .. 32 w + 31 of h_j.
-    if (warp * 32 < D) {
-      const int d = warp * 32 + lane;
-      const size_t row = static_cast<size_t>(bh) * a.Nk + j;
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c0, r);
-        tmem_wait_ld();
-        if (bf16_out) {
-          uint8_t* box = stage + (c0 >> 6) * (D * 128);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-            u.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-            u.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-            u.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-            *reinterpret_cast<uint4*>(box + sw128_offset(d, ((c0 & 63) >> 3) * 16 + q * 16)) = u;
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&map_k);
+      prefetch_tmap(&map_v);
+      if (a.qbar) prefetch_tmap(&map_q);
+      if (bf16_out) prefetch_tmap(&map_hout);
+      int last_round[NS];
+      for (int s = 0; s < NS; ++s) last_round[s] = -1;
+      int k = 0;
+      for (int g = blockIdx.x; g < n_items; g += gridDim.x, ++k) {
+        const int s = k % NS, r = k / NS;
+        if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, a.err, &abort_flag)) break;
+        uint8_t* slot = smem + s * L::SLOT;
+        if (g < n_kv) {
+          const int bh = g / a.Nk, j = g % a.Nk;
+          mbar_arrive_expect_tx(&full[s], 64 * D * 2 * 2);
+          for (int b = 0; b < KBOX; ++b) {
+            tma_load_3d(slot + b * 8192, &map_k, &full[s], b * 64, j * 64, bh);
+            tma_load_3d(slot + 16384 + b * 8192, &map_v, &full[s], b * 64, j * 64, bh);
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(a.h32 + (row * D + d) * D + c0);
+          const int q = g - n_kv, bh = q / a.Nq, i = q % a.Nq;
+          mbar_arrive_expect_tx(&full[s], a.block_q * D * 2);
+          for (int b = 0; b < KBOX; ++b)
+            tma_load_3d(slot + b * (a.block_q * 128), &map_q, &full[s], b * 64, i * a.block_q, bh);
+        }
+        last_round[s] = r;
+      }
+      if (abort_flag)
+        for (int s = 0; s < NS; ++s)
+          if (last_round[s] >= 0) mbar_wait(&full[s], last_round[s] & 1, nullptr, nullptr);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
+      int k = 0, m = 0;
+      for (int g = blockIdx.x; g < n_items; g += gridDim.x, ++k) {
+        const int s = k % NS, r = k / NS;
+        if (!mbar_wait(&phi_done[s], r & 1, a.err, &abort_flag)) break;
+        if (g >= n_kv) {  // a query block: nothing to multiply, the slot is free again
+          mbar_arrive(&empty[s]);
+          continue;
+        }
+        const int acc = m & 1;
+        if (m >= 2 && !mbar_wait(&acc_empty[acc], ((m >> 1) - 1) & 1, a.err, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * L::SLOT);
+        const uint32_t lbo_a = D == 64 ? smem_u32(zero) - sa : 8192u;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                 __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sa + kk * 2048, lbo_a, 1024);
+          const uint64_t bd = smem_desc_sw128(sa + 16384 + kk * 2048, 8192, 1024);
+          umma_bf16_ss(tmem + acc * 128, ad, bd, idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+        umma_commit(&acc_full[acc]);
+        ++m;
+      }
+      umma_commit(&drain);
+      mbar_wait(&drain, 0, nullptr, nullptr);
+    }
+    __syncwarp();
+  } else if (warp < 6 || warp >= 10) {
+    // ------------------------------------------------------------ column passes (2 x 128 threads)
+    const int cw = warp < 6 ? 0 : 1;         // this warpgroup takes the items with k % 2 == cw
+    const int wt = warp < 6 ? tid - 64 : tid - 320;
+    const int bar_id = cw == 0 ? 1 : 3;
+    const int cc = wt % CPR, rg = wt / CPR;
+    int k = cw;
+    for (int g = blockIdx.x + cw * gridDim.x; g < n_items; g += 2 * gridDim.x, k += 2) {
+      const int s = k % NS, r = k / NS;
+      bool ok = mbar_wait(&full[s], r & 1, a.err, &abort_flag);
+      if (!named_barrier_and(bar_id, 128, ok)) break;
+      const bool isq = g >= n_kv;
+      int bh, idx, rows;
+      if (isq) {
+        const int q = g - n_kv;
+        bh = q / a.Nq;
+        idx = q % a.Nq;
+        rows = a.block_q;
+      } else {
+        bh = g / a.Nk;
+        idx = g % a.Nk;
+        rows = 64;
+      }
+      const int valid = min(rows, a.N - idx * rows);
+      uint8_t* slotp = smem + s * L::SLOT;
+      if (isq) {
+        if (a.block_q == 128)
+          column_pass<D, 128, false>(slotp, cc, rg, valid, part_d[cw], part_f[cw]);
+        else
+          column_pass<D, 64, false>(slotp, cc, rg, valid, part_d[cw], part_f[cw]);
+      } else {
+        column_pass<D, 64, true>(slotp, cc, rg, valid, part_d[cw], part_f[cw]);
+      }
+      if (!isq) fence_proxy_async_smem();
+      named_barrier(bar_id, 128);
+      if (wt < D) {
+        double sum = 0.0;
+        float zsum = 0.f;
+#pragma unroll
+        for (int q = 0; q < RG; ++q) {
+          sum += part_d[cw][q][wt];
+          zsum += part_f[cw][q][wt];
+        }
+        if (isq) {
+          a.qbar[(static_cast<size_t>(bh) * a.Nq + idx) * D + wt] = sum / static_cast<double>(valid);
+        } else {
+          const size_t row = static_cast<size_t>(bh) * a.Nk + idx;
+          if (a.kbar) a.kbar[row * D + wt] = sum / static_cast<double>(valid);
+          if (bf16_out) {
+            __nv_bfloat16* zr = a.hst + row * a.LD + D * D;
+            zr[wt] = __float2bfloat16_rn(zsum);
+            if (D == 64) zr[64 + wt] = __float2bfloat16_rn(0.f);
+          } else if (a.z32) {
+            a.z32[row * D + wt] = zsum;
+          }
+        }
+      }
+      named_barrier(bar_id, 128);  // partial sums consumed; the next item may overwrite them
+      mbar_arrive(&phi_done[s]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 6..9, 128 threads)
+    const int et = tid - 192;
+    const int quarter = warp & 3;
+    const int d = quarter * 32 + lane;  // row of h_j held in this thread's TMEM lane
+    int m = 0;
+    for (int g = blockIdx.x; g < n_kv; g += gridDim.x, ++m) {
+      const int bh = g / a.Nk, j = g % a.Nk;
+      const int acc = m & 1;
+      bool ok = mbar_wait(&acc_full[acc], (m >> 1) & 1, a.err, &abort_flag);
+      if (!named_barrier_and(2, 128, ok)) break;
+      tc_fence_after();
+      uint8_t* stg = stage0 + acc * L::STAGE;
+      if (bf16_out) {
+        if (et == 0) tma_store_wait_read_all_but_one();  // the store that last used this staging tile is done reading
+        named_barrier(2, 128);
+      }
+      if (quarter * 32 < D) {
+        const size_t row = static_cast<size_t>(bh) * a.Nk + j;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t rv[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + acc * 128 + c0, rv);
+          tmem_wait_ld();
+          if (bf16_out) {
+            uint8_t* box = stg + (c0 >> 6) * (D * 128);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(rv[8 * q + 0]), __uint_as_float(rv[8 * q + 1]));
+              u.y = pack_bf16x2(__uint_as_float(rv[8 * q + 2]), __uint_as_float(rv[8 * q + 3]));
+              u.z = pack_bf16x2(__uint_as_float(rv[8 * q + 4]), __uint_as_float(rv[8 * q + 5]));
+              u.w = pack_bf16x2(__uint_as_float(rv[8 * q + 6]), __uint_as_float(rv[8 * q + 7]));
+              *reinterpret_cast<uint4*>(box + sw128_offset(d, ((c0 & 63) >> 3) * 16 + q * 16)) = u;
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(a.h32 + (row * D + d) * D + c0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(rv[4 * q]), __uint_as_float(rv[4 * q + 1]),
+                                   __uint_as_float(rv[4 * q + 2]), __uint_as_float(rv[4 * q + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      if (bf16_out) {
+        fence_proxy_async_smem();
+        named_barrier(2, 128);
+        if (et == 0) {
+          for (int b = 0; b < KBOX; ++b) tma_store_3d(&map_hout, stg + b * (D * 128), b * 64, 0, bh * a.Nk + j);
+          tma_store_commit();
         }
       }
     }
-    if (bf16_out) fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && bf16_out) {
-      for (int b = 0; b < KBOX; ++b) tma_store_3d(&map_hout, stage + b * (D * 128), b * 64, 0, bh * a.Nk + j);
-      tma_store_commit();
-    }
-  }
-  // After an abort: let loads and the MMA still in flight finish before the CTA retires.
-  if (tid == 0) {
-    for (int s = 0; s < 2; ++s)
-      if (inflight[s] >= 0) mbar_wait(&bar_full[s], inflight[s], nullptr, nullptr);
-    if (mma_parity >= 0) mbar_wait(&bar_mma, mma_parity, nullptr, nullptr);
-    if (bf16_out) tma_store_wait_all();
+    if (et == 0 && bf16_out) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 

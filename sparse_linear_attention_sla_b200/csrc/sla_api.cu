@@ -19,7 +19,6 @@ namespace {
 
 using sla::AggArgs;
 using sla::AttnArgs;
-using sla::KvPrepArgs;
 using sla::MaskListArgs;
 using sla::SelectArgs;
 
@@ -215,12 +214,16 @@ sla_status launch_pool(const void* x, double* out, const Shape& s, int block, in
   return launched("pool_mean_kernel");
 }
 
+// Fused precompute: query-block means (when qbar is set), KV-block means, z_j and h_j.
 template <int D>
-sla_status launch_kv_prep(const void* k, const void* v, const Shape& s, const KvPrepArgs& args, cudaStream_t st) {
-  CUtensorMap mk, mv, mh;
+sla_status launch_prep(const void* q, const void* k, const void* v, const Shape& s, const sla::PrepArgs& args,
+                       cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mh;
+  std::memset(&mq, 0, sizeof(mq));
+  std::memset(&mh, 0, sizeof(mh));
+  if (args.qbar) SLA_TRY(act_map(&mq, q, s, static_cast<uint32_t>(s.bq)));
   SLA_TRY(act_map(&mk, k, s, 64));
   SLA_TRY(act_map(&mv, v, s, 64));
-  std::memset(&mh, 0, sizeof(mh));
   if (args.hst) {
     // h_j tiles inside the stacked-state rows: (e, d, block) -> row * LD + d * D + e
     const uint64_t dims[3] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.D),
@@ -229,12 +232,12 @@ sla_status launch_kv_prep(const void* k, const void* v, const Shape& s, const Kv
     const uint32_t box[3] = {64, static_cast<uint32_t>(s.D), 1};
     SLA_TRY(make_map(&mh, args.hst, 3, dims, strides, box));
   }
-  constexpr int smem = sla::KvPrepSmem<D>::total();
-  SLA_TRY(allow_smem(sla::kv_prep_kernel<D>, smem));
-  const int total = s.BH * s.Nk;
-  const int grid = total < 2 * sm_count() ? total : 2 * sm_count();
-  sla::kv_prep_kernel<D><<<grid, 128, smem, st>>>(mk, mv, mh, args);
-  return launched("kv_prep_kernel");
+  constexpr int smem = sla::PrepSmem<D>::total();
+  SLA_TRY(allow_smem(sla::prep_kernel<D>, smem));
+  const long long items = static_cast<long long>(s.BH) * s.Nk + (args.qbar ? static_cast<long long>(s.BH) * s.Nq : 0);
+  const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
+  sla::prep_kernel<D><<<grid, 448, smem, st>>>(mq, mk, mv, mh, args);
+  return launched("prep_kernel");
 }
 
 template <int D>
@@ -372,24 +375,26 @@ struct StageEvents {
 template <int D>
 sla_status forward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
                         const int8_t* mask, void* out, const Workspace& w, cudaStream_t st, StageEvents& ev) {
-  KvPrepArgs kv{};
-  kv.BH = s.BH;
-  kv.N = s.N;
-  kv.Nk = s.Nk;
-  kv.kbar = mask ? nullptr : w.kbar;
-  kv.hst = w.hst;
-  kv.LD = s.LD;
-  kv.err = w.err;
+  sla::PrepArgs pa{};
+  pa.BH = s.BH;
+  pa.N = s.N;
+  pa.Nq = s.Nq;
+  pa.Nk = s.Nk;
+  pa.block_q = s.bq;
+  pa.qbar = mask ? nullptr : w.qbar;
+  pa.kbar = mask ? nullptr : w.kbar;
+  pa.hst = w.hst;
+  pa.LD = s.LD;
+  pa.err = w.err;
   SLA_TRY(ev.mark(0, st));
   if (mask) {
-    SLA_TRY(launch_kv_prep<D>(k, v, s, kv, st));
+    SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
     SLA_TRY(ev.mark(1, st));
     MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
     sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
     SLA_TRY(launched("mask_lists_kernel"));
   } else {
-    SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
-    SLA_TRY(launch_kv_prep<D>(k, v, s, kv, st));
+    SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
     SLA_TRY(ev.mark(1, st));
     SLA_TRY(launch_scores<D>(w.qbar, w.kbar, w.S, s, st));
     SelectArgs a{};
@@ -491,17 +496,19 @@ sla_status sla_kv_states(const sla_problem* p, const void* k, const void* v, flo
       return fail(SLA_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold at least 256 bytes");
     err = static_cast<uint32_t*>(ws);
   }
-  KvPrepArgs kv{};
-  kv.BH = s.BH;
-  kv.N = s.N;
-  kv.Nk = s.Nk;
-  kv.h32 = h_out;
-  kv.z32 = z_out;
-  kv.LD = s.LD;
-  kv.err = err;
+  sla::PrepArgs pa{};
+  pa.BH = s.BH;
+  pa.N = s.N;
+  pa.Nq = s.Nq;
+  pa.Nk = s.Nk;
+  pa.block_q = s.bq;
+  pa.h32 = h_out;
+  pa.z32 = z_out;
+  pa.LD = s.LD;
+  pa.err = err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (s.D == 64) return launch_kv_prep<64>(k, v, s, kv, st);
-  return launch_kv_prep<128>(k, v, s, kv, st);
+  if (s.D == 64) return launch_prep<64>(nullptr, k, v, s, pa, st);
+  return launch_prep<128>(nullptr, k, v, s, pa, st);
 }
 
 sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
