@@ -106,6 +106,22 @@ def algorithmic_work(w, mask):
             "f_states": f_states, "f_agg": f_agg, "f_router": f_router}
 
 
+def max_over_ranks(x, dist=None, device="cpu"):
+    """Largest value of x over all ranks (x itself without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world, flops_per_rank, ms_step):
+    """Aggregate throughput of `world` replicas that each did flops_per_rank in ms_step (the slowest rank)."""
+    return world * flops_per_rank / (ms_step * 1e-3) / 1e12
+
+
 def kernel_source_sha():
     h = hashlib.sha256()
     for name in ("attention.cuh", "sm100.cuh"):
@@ -248,12 +264,8 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x):
+        return max_over_ranks(x, dist if world > 1 else None, dev)
 
     w = WORKLOADS[args.workload]
     q, k, v, alpha = make_inputs(w, device=dev)
@@ -292,9 +304,9 @@ def run_ours(args):
     clock_info = clocks.summary()
 
     ms_local = sum(per_step) / len(per_step)
-    ms_step = max_over_ranks(ms_local)
+    ms_step = rank_max(ms_local)
     stage_ms = [s / args.steps for s in stage_sum]
-    attn_ms = max_over_ranks(stage_ms[3])
+    attn_ms = rank_max(stage_ms[3])
 
     # labels actually used, for the work accounting
     mask, _, _ = binding.route(q, k, w.block_q, w.block_kv, w.kh, w.kl)
@@ -302,7 +314,7 @@ def run_ours(args):
     del mask
     peaks = measured_peaks()
     eff_flops = dense_equivalent_flops(w)
-    value = world * eff_flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, eff_flops, ms_step)
 
     # dominant kernel: the fused attention (stage 3)
     achieved = work["f_attn_kernel"] / (attn_ms * 1e-3) / 1e12
@@ -342,10 +354,10 @@ def run_ours(args):
         for _ in range(args.warmup):
             e2e_step()
         barrier()
-        ms_e2e = max_over_ranks(sum(e2e_step() for _ in range(args.steps)) / args.steps)
+        ms_e2e = rank_max(sum(e2e_step() for _ in range(args.steps)) / args.steps)
         barrier()
         h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, ha))
-        e2e = {"value": round(world * eff_flops / (ms_e2e * 1e-3) / 1e12, 3), "unit": UNIT,
+        e2e = {"value": round(whole_job_tflops(world, eff_flops, ms_e2e), 3), "unit": UNIT,
                "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": hout.numel() * hout.element_size()}
         del hq, hk, hv, ha, hout, dq, dk, dv, da
@@ -369,7 +381,7 @@ def run_ours(args):
                 times.append(e0.elapsed_time(e1))
                 attn_d.append(st_d[3])
         binding.check(wsd)
-        ms_d = max_over_ranks(sum(times) / len(times))
+        ms_d = rank_max(sum(times) / len(times))
         dense = {"workload": wd.name + "_kh1", "ms_per_call": round(ms_d, 4),
                  "effective_tflops": round(eff_flops / (ms_d * 1e-3) / 1e12, 2),
                  "attn_kernel_ms": round(sum(attn_d) / len(attn_d), 4),

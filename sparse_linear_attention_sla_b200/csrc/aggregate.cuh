@@ -19,144 +19,189 @@
 namespace sla {
 
 struct AggArgs {
-  int Nq, Nk, LD;
+  int Nq, Nk, LD, BH;
   __nv_bfloat16* Hagg;   // [BH, Nq, D*D]
   float* Zagg;           // [BH, Nq, D]
   uint32_t* err;
 };
 
+constexpr int kAggStages = 3;
 constexpr uint32_t kAggStageBytes = 3 * 16384;  // A for two M-tiles + one B tile (64 x 128)
+constexpr uint32_t kAggStagingBytes = 65536;    // bf16 output tile: 2 M-tiles x 128 rows x 128 columns
 
-// grid: (LD/128, ceil(Nq/256), BH); block 128 (warp 0: TMA, warp 1: MMA, all: epilogue).
-// One CTA owns 128 state columns for up to two 128-row M-tiles of query blocks, so each
-// stacked-state tile is read once per head. Two CTAs share an SM: 2 stages x 48 KB of
-// shared memory, 256 TMEM columns (M-tile t accumulates in columns [128 t, 128 t + 128)).
+// Persistent, one CTA per SM, 192 threads: warp 0 TMA producer, warp 1 tcgen05 issuer,
+// warps 2..5 epilogue (TMEM -> bf16 -> shared-memory staging -> TMA store). A tile is 128 state columns x up to two 128-row M-tiles of query
+// blocks of one head (so each stacked-state tile is read once per head); tiles are walked
+// columns-fastest. Accumulators are double-buffered in TMEM (2 x 256 columns, M-tile t of
+// buffer b at column 256 b + 128 t) so the epilogue of a tile overlaps the next mainloop.
 template <int D>
-__global__ void __launch_bounds__(128, 2) agg_kernel(const __grid_constant__ CUtensorMap map_w,
+__global__ void __launch_bounds__(192, 1) agg_kernel(const __grid_constant__ CUtensorMap map_w,
                                                      const __grid_constant__ CUtensorMap map_h,
                                                      const __grid_constant__ CUtensorMap map_out, AggArgs a) {
-  constexpr int NSTAGE = 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[NSTAGE], empty[NSTAGE], acc_full, drain;
+  __shared__ uint64_t full[kAggStages], empty[kAggStages], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * 128, m0 = blockIdx.y * 256, bh = blockIdx.z;
-  const int nm = (m0 + 128 < a.Nq) ? 2 : 1;  // M-tiles this CTA owns
+  const int n_nt = a.LD / 128, n_mp = (a.Nq + 255) / 256;
+  const int n_tiles = n_nt * n_mp * a.BH;
   const int nk = (a.Nk + 63) / 64;
   if (tid == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
+    for (int s = 0; s < kAggStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, 256);
+    tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
+  auto decode = [&](int t, int& n0, int& m0, int& bh, int& nm) {
+    const int nt = t % n_nt, rest = t / n_nt;
+    n0 = nt * 128;
+    m0 = (rest % n_mp) * 256;
+    bh = rest / n_mp;
+    nm = (m0 + 128 < a.Nq) ? 2 : 1;
+  };
+
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&map_w);
       prefetch_tmap(&map_h);
       prefetch_tmap(&map_out);
-      int last_round[NSTAGE] = {-1, -1};
-      for (int k = 0; k < nk; ++k) {
-        const int s = k % NSTAGE, r = k / NSTAGE;
-        if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, a.err, &abort_flag)) break;
-        uint8_t* st = smem + s * kAggStageBytes;
-        mbar_arrive_expect_tx(&full[s], (nm + 1) * 16384);
-        for (int t = 0; t < nm; ++t) tma_load_3d(st + t * 16384, &map_w, &full[s], k * 64, m0 + 128 * t, bh);
-        for (int b = 0; b < 2; ++b) tma_load_3d(st + 32768 + b * 8192, &map_h, &full[s], n0 + 64 * b, k * 64, bh);
-        last_round[s] = r;
+      int last_round[kAggStages];
+      for (int s = 0; s < kAggStages; ++s) last_round[s] = -1;
+      uint32_t sc = 0;  // stages filled so far
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        int n0, m0, bh, nm;
+        decode(t, n0, m0, bh, nm);
+        for (int k = 0; k < nk; ++k, ++sc) {
+          const int s = sc % kAggStages, r = sc / kAggStages;
+          if (r > 0 && !(ok = mbar_wait(&empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
+          uint8_t* st = smem + s * kAggStageBytes;
+          mbar_arrive_expect_tx(&full[s], (nm + 1) * 16384);
+          for (int tt = 0; tt < nm; ++tt) tma_load_3d(st + tt * 16384, &map_w, &full[s], k * 64, m0 + 128 * tt, bh);
+          for (int b = 0; b < 2; ++b) tma_load_3d(st + 32768 + b * 8192, &map_h, &full[s], n0 + 64 * b, k * 64, bh);
+          last_round[s] = r;
+        }
       }
       if (abort_flag)
-        for (int s = 0; s < NSTAGE; ++s)
+        for (int s = 0; s < kAggStages; ++s)
           if (last_round[s] >= 0) mbar_wait(&full[s], last_round[s] & 1, nullptr, nullptr);
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);
-      for (int k = 0; k < nk; ++k) {
-        const int s = k % NSTAGE;
-        if (!mbar_wait(&full[s], (k / NSTAGE) & 1, a.err, &abort_flag)) break;
-        tc_fence_after();
-        const uint32_t st = smem_u32(smem + s * kAggStageBytes);
+      uint32_t sc = 0;
+      int tc = 0;  // tiles issued
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tc) {
+        int n0, m0, bh, nm;
+        decode(t, n0, m0, bh, nm);
+        const int ab = tc & 1;
+        if (tc >= 2 && !(ok = mbar_wait(&acc_empty[ab], ((tc >> 1) - 1) & 1, a.err, &abort_flag))) break;
+        for (int k = 0; k < nk; ++k, ++sc) {
+          const int s = sc % kAggStages;
+          if (!(ok = mbar_wait(&full[s], (sc / kAggStages) & 1, a.err, &abort_flag))) break;
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * kAggStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc_sw128(st + 32768 + kk * 2048, 8192, 1024);
-          for (int t = 0; t < nm; ++t) {
-            const uint64_t ad = smem_desc_sw128(st + t * 16384 + kk * 32, 16, 1024);
-            umma_bf16_ss(tmem + 128 * t, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = smem_desc_sw128(st + 32768 + kk * 2048, 8192, 1024);
+            for (int tt = 0; tt < nm; ++tt) {
+              const uint64_t ad = smem_desc_sw128(st + tt * 16384 + kk * 32, 16, 1024);
+              umma_bf16_ss(tmem + ab * 256 + 128 * tt, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+            }
           }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        if (!ok) break;
+        umma_commit(&acc_full[ab]);
       }
-      umma_commit(&acc_full);
       umma_commit(&drain);
       mbar_wait(&drain, 0, nullptr, nullptr);
     }
     __syncwarp();
-  }
-
-  // Epilogue: warp w holds rows m0 + 128 t + 32 w + lane of M-tile t.
-  const bool ok = mbar_wait(&acc_full, 0, a.err, &abort_flag);
-  const bool go = __syncthreads_and(ok) && !abort_flag;
-  const bool z_tile = n0 >= D * D;
-  if (go) {
-    tc_fence_after();
-    for (int t = 0; t < nm; ++t) {
-      const int rloc = warp * 32 + lane;
-      const int m = m0 + 128 * t + rloc;
-      uint8_t* stg = smem + t * 32768;  // two 16 KB boxes per M-tile; the stages are free now
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        __syncwarp();
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + 128 * t + c0, r);
+  } else {
+    // Epilogue: warp w (quarter w & 3) holds rows m0 + 128 t + 32 (w & 3) + lane of M-tile t.
+    const int et = tid - 64;
+    const int quarter = warp & 3;
+    const int rloc = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint8_t* stg = smem + kAggStages * kAggStageBytes;
+    int tc = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
+      int n0, m0, bh, nm;
+      decode(t, n0, m0, bh, nm);
+      const int ab = tc & 1;
+      const bool ok = mbar_wait(&acc_full[ab], (tc >> 1) & 1, a.err, &abort_flag);
+      if (et == 0) tma_store_wait_read();  // the previous tile's store has left the staging tile
+      if (!named_barrier_and(1, 128, ok)) break;
+      tc_fence_after();
+      const bool z_tile = n0 >= D * D;
+      for (int tt = 0; tt < nm; ++tt) {
+        const int m = m0 + 128 * tt + rloc;
+        uint32_t r[4][32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(lane_addr + ab * 256 + 128 * tt + 32 * q, r[q]);
         tmem_wait_ld();
         if (!z_tile) {
-          uint8_t* box = stg + (c0 >> 6) * 16384;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-            u.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-            u.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-            u.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-            *reinterpret_cast<uint4*>(box + sw128_offset(rloc, ((c0 & 63) >> 3) * 16 + q * 16)) = u;
-          }
-        } else if (m < a.Nq && c0 < D) {
-          float4* dst = reinterpret_cast<float4*>(a.Zagg + (static_cast<size_t>(bh) * a.Nq + m) * D + c0);
+            uint8_t* box = stg + tt * 32768 + (q >> 1) * 16384;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                 __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+            for (int v = 0; v < 4; ++v)
+              *reinterpret_cast<uint4*>(box + sw128_offset(rloc, ((q & 1) * 4 + v) * 16)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(r[q][8 * v + 0]), __uint_as_float(r[q][8 * v + 1])),
+                             pack_bf16x2(__uint_as_float(r[q][8 * v + 2]), __uint_as_float(r[q][8 * v + 3])),
+                             pack_bf16x2(__uint_as_float(r[q][8 * v + 4]), __uint_as_float(r[q][8 * v + 5])),
+                             pack_bf16x2(__uint_as_float(r[q][8 * v + 6]), __uint_as_float(r[q][8 * v + 7])));
+          }
+        } else if (m < a.Nq) {
+          float4* dst = reinterpret_cast<float4*>(a.Zagg + (static_cast<size_t>(bh) * a.Nq + m) * D);
+#pragma unroll
+          for (int q = 0; q < D / 32; ++q)
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[8 * q + v] = make_float4(__uint_as_float(r[q][4 * v]), __uint_as_float(r[q][4 * v + 1]),
+                                           __uint_as_float(r[q][4 * v + 2]), __uint_as_float(r[q][4 * v + 3]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);  // the accumulator has left TMEM
+      if (!z_tile) {
+        fence_proxy_async_smem();
+        named_barrier(1, 128);
+        if (et == 0) {
+          for (int tt = 0; tt < nm; ++tt)
+            for (int b = 0; b < 2; ++b)
+              tma_store_3d(&map_out, stg + tt * 32768 + b * 16384, n0 + 64 * b, m0 + 128 * tt, bh);
+          tma_store_commit();
         }
       }
     }
-    if (!z_tile) fence_proxy_async_smem();
+    if (et == 0) tma_store_wait_all();
   }
   tc_fence_before();
   __syncthreads();
-  if (go && !z_tile && tid == 0) {
-    for (int t = 0; t < nm; ++t)
-      for (int b = 0; b < 2; ++b) tma_store_3d(&map_out, smem + t * 32768 + b * 16384, n0 + 64 * b, m0 + 128 * t, bh);
-    tma_store_commit();
-    tma_store_wait_all();
-  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -272,7 +272,7 @@ sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
 
 template <int D>
 sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
-  CUtensorMap mw, mh, mo;
+  CUtensorMap mw, mh;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
     const uint64_t strides[2] = {static_cast<uint64_t>(s.w_ld), static_cast<uint64_t>(s.Nq) * s.w_ld};
@@ -285,6 +285,7 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
     const uint32_t box[3] = {64, 64, 1};
     SLA_TRY(make_map(&mh, w.hst, 3, dims, strides, box));
   }
+  CUtensorMap mo;
   {
     const uint64_t DD = static_cast<uint64_t>(s.D) * s.D;
     const uint64_t dims[3] = {DD, static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
@@ -292,11 +293,12 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
     const uint32_t box[3] = {64, 128, 1};
     SLA_TRY(make_map(&mo, w.Hagg, 3, dims, strides, box));
   }
-  const int smem = 2 * sla::kAggStageBytes + 1024;
+  const int smem = sla::kAggStages * sla::kAggStageBytes + sla::kAggStagingBytes + 1024;
   SLA_TRY(allow_smem(sla::agg_kernel<D>, smem));
-  AggArgs a{s.Nq, s.Nk, s.LD, w.Hagg, w.Zagg, w.err};
-  dim3 grid(s.LD / 128, (s.Nq + 255) / 256, s.BH);
-  sla::agg_kernel<D><<<grid, 128, smem, st>>>(mw, mh, mo, a);
+  AggArgs a{s.Nq, s.Nk, s.LD, s.BH, w.Hagg, w.Zagg, w.err};
+  const long long tiles = static_cast<long long>(s.LD / 128) * ((s.Nq + 255) / 256) * s.BH;
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  sla::agg_kernel<D><<<grid, 192, smem, st>>>(mw, mh, mo, a);
   return launched("agg_kernel");
 }
 
