@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(192, 1) agg_kernel(const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_launch();
+  grid_dep_wait();  // the indicator and the stacked states come from earlier kernels
 
   auto decode = [&](int t, int& n0, int& m0, int& bh, int& nm) {
     const int nt = t % n_nt, rest = t / n_nt;

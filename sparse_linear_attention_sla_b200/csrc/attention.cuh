@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(320, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  grid_dep_wait();  // critical lists, H_i and Z_i come from earlier kernels
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(448, 1)
   const int n_kv = a.BH * a.Nk;
   const int n_items = n_kv + (a.qbar ? a.BH * a.Nq : 0);
   const bool bf16_out = a.hst != nullptr;
+  grid_dep_launch();
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);

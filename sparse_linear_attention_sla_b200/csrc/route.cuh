@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(128) score_kernel(const double* __restrict__ q
   const int bh = blockIdx.z, i0 = blockIdx.y * T, j0 = blockIdx.x * T;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wy = warp >> 1, wx = warp & 1;
+  grid_dep_launch();
+  grid_dep_wait();  // pooled means come from the previous kernel
   const int fr = lane >> 2, fc = lane & 3;
   const double* qb = qbar + static_cast<size_t>(bh) * Nq * D;
   const double* kb = kbar + static_cast<size_t>(bh) * Nk * D;
@@ -132,6 +134,8 @@ struct SelectArgs {
 
 // One warp per row; dynamic smem = warps_per_cta * Nk * 8 bytes of keys.
 __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
+  grid_dep_launch();
+  grid_dep_wait();  // scores come from the previous kernel
   extern __shared__ uint64_t keys_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpc = blockDim.x >> 5;
@@ -273,6 +277,8 @@ __device__ __forceinline__ uint64_t pick_from_group(const double* srow, uint64_t
 
 template <int KPL>
 __global__ void __launch_bounds__(256) select_reg_kernel(SelectArgs a) {
+  grid_dep_launch();
+  grid_dep_wait();  // scores come from the previous kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * (blockDim.x >> 5) + warp;
   if (row >= a.rows) return;  // whole warp leaves; nothing below synchronises the CTA

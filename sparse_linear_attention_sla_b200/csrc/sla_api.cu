@@ -6,6 +6,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include <cudaTypedefs.h>
 
@@ -195,6 +196,27 @@ sla_status allow_smem(K kernel, int bytes) {
   return SLA_OK;
 }
 
+// Launch `kernel` as a programmatic dependent of the previous kernel in the stream: it may
+// be scheduled while the predecessor drains and waits (griddepcontrol.wait) before
+// reading the predecessor's results.
+template <typename... KArgs, typename... Args>
+sla_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                            const char* what, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return fail(SLA_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return SLA_OK;
+}
+
 sla_status launched(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SLA_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
@@ -243,15 +265,14 @@ sla_status launch_prep(const void* q, const void* k, const void* v, const Shape&
 template <int D>
 sla_status launch_scores(const double* qbar, const double* kbar, double* S, const Shape& s, cudaStream_t st) {
   dim3 grid((s.Nk + 63) / 64, (s.Nq + 63) / 64, s.BH);
-  sla::score_kernel<D><<<grid, 128, 0, st>>>(qbar, kbar, S, s.Nq, s.Nk);
-  return launched("score_kernel");
+  return launch_dependent(sla::score_kernel<D>, grid, dim3(128), 0, st, "score_kernel", qbar, kbar, S, s.Nq, s.Nk);
 }
 
 template <int KPL>
 sla_status launch_select_reg(const SelectArgs& a, cudaStream_t st) {
   const int wpc = 8;
-  sla::select_reg_kernel<KPL><<<(a.rows + wpc - 1) / wpc, wpc * 32, 0, st>>>(a);
-  return launched("select_reg_kernel");
+  return launch_dependent(sla::select_reg_kernel<KPL>, dim3((a.rows + wpc - 1) / wpc), dim3(wpc * 32), 0, st,
+                          "select_reg_kernel", a);
 }
 
 sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
@@ -266,8 +287,7 @@ sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
   const int smem = static_cast<int>(wpc * per_warp);
   SLA_TRY(allow_smem(sla::select_kernel, smem));
   const int grid = (a.rows + wpc - 1) / wpc;
-  sla::select_kernel<<<grid, wpc * 32, smem, st>>>(a);
-  return launched("select_kernel");
+  return launch_dependent(sla::select_kernel, dim3(grid), dim3(wpc * 32), smem, st, "select_kernel", a);
 }
 
 template <int D>
@@ -298,8 +318,7 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
   AggArgs a{s.Nq, s.Nk, s.LD, s.BH, w.Hagg, w.Zagg, w.err};
   const long long tiles = static_cast<long long>(s.LD / 128) * ((s.Nq + 255) / 256) * s.BH;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  sla::agg_kernel<D><<<grid, 192, smem, st>>>(mw, mh, mo, a);
-  return launched("agg_kernel");
+  return launch_dependent(sla::agg_kernel<D>, dim3(grid), dim3(192), smem, st, "agg_kernel", mw, mh, mo, a);
 }
 
 template <int D>
@@ -333,8 +352,7 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.err = w.err;
   // persistent: two CTAs per SM walk the tiles
   const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
-  sla::attn_kernel<D><<<grid, 320, smem, st>>>(mq, mk, mv, mh, a);
-  return launched("attn_kernel");
+  return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(320), smem, st, "attn_kernel", mq, mk, mv, mh, a);
 }
 
 // ------------------------------------------------------------------ entry points (templated on D)

@@ -107,6 +107,16 @@ __device__ __forceinline__ void named_barrier(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// A kernel launched as a programmatic dependent of the previous kernel in the stream
+// may start (barrier set-up, TMEM allocation) while its predecessor drains; it must
+// wait here before reading anything the predecessor writes. A no-op otherwise.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel in the stream be scheduled as SMs free up (it still waits for this
+// grid to complete before reading its results).
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ fences
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
