@@ -21,6 +21,7 @@ namespace {
 using sla::AggArgs;
 using sla::AttnArgs;
 using sla::MaskListArgs;
+using sla::CertArgs;
 using sla::SelectArgs;
 
 constexpr int kMaxNk = 16384;
@@ -90,7 +91,10 @@ struct Workspace {
   uint32_t* err;
   double* qbar;
   double* kbar;
-  double* S;
+  double* S;    // fp64 scores (the long-row selection)
+  float* S32;   // fp32 scores (the certified selection), aliases S
+  float* nq;    // fp32 norms of the pooled queries
+  float* nk;    // fp32 norms of the pooled keys
   int8_t* mask;
   int32_t* crit;
   int32_t* crit_cnt;
@@ -116,6 +120,9 @@ Workspace layout(const Shape& s, uint8_t* base) {
   w.qbar = reinterpret_cast<double*>(take(BH * s.Nq * s.D * sizeof(double)));
   w.kbar = reinterpret_cast<double*>(take(BH * s.Nk * s.D * sizeof(double)));
   w.S = reinterpret_cast<double*>(take(BH * s.Nq * s.Nk * sizeof(double)));
+  w.S32 = reinterpret_cast<float*>(w.S);
+  w.nq = reinterpret_cast<float*>(take(BH * s.Nq * sizeof(float)));
+  w.nk = reinterpret_cast<float*>(take(BH * s.Nk * sizeof(float)));
   w.mask = reinterpret_cast<int8_t*>(take(BH * s.Nq * s.Nk));
   w.crit = reinterpret_cast<int32_t*>(take(BH * s.Nq * s.Nk * sizeof(int32_t)));
   w.crit_cnt = reinterpret_cast<int32_t*>(take(BH * s.Nq * sizeof(int32_t)));
@@ -268,19 +275,70 @@ sla_status launch_scores(const double* qbar, const double* kbar, double* S, cons
   return launch_dependent(sla::score_kernel<D>, grid, dim3(128), 0, st, "score_kernel", qbar, kbar, S, s.Nq, s.Nk);
 }
 
-template <int KPL>
-sla_status launch_select_reg(const SelectArgs& a, cudaStream_t st) {
-  const int wpc = 8;
-  return launch_dependent(sla::select_reg_kernel<KPL>, dim3((a.rows + wpc - 1) / wpc), dim3(wpc * 32), 0, st,
-                          "select_reg_kernel", a);
+template <int D>
+sla_status launch_scores32(const Shape& s, const Workspace& w, cudaStream_t st) {
+  dim3 grid((s.Nk + 63) / 64, (s.Nq + 63) / 64, s.BH);
+  constexpr int smem = sla::Score32Smem<D>::kBytes;
+  SLA_TRY(allow_smem(sla::score32_kernel<D>, smem));
+  return launch_dependent(sla::score32_kernel<D>, grid, dim3(256), smem, st, "score32_kernel", w.qbar, w.kbar, w.S32,
+                          w.nq, w.nk, s.Nq, s.Nk);
 }
 
-sla_status launch_select(const SelectArgs& a, cudaStream_t st) {
-  // Rows of up to 2048 blocks keep their keys in registers; longer rows use shared memory.
-  if (a.Nk <= 32 * 8) return launch_select_reg<8>(a, st);
-  if (a.Nk <= 32 * 16) return launch_select_reg<16>(a, st);
-  if (a.Nk <= 32 * 32) return launch_select_reg<32>(a, st);
-  if (a.Nk <= 32 * 64) return launch_select_reg<64>(a, st);
+template <int KPL, int D>
+sla_status launch_cert(const CertArgs& a, cudaStream_t st) {
+  const int wpc = 8;
+  return launch_dependent(sla::select_cert_kernel<KPL, D>, dim3((a.rows + wpc - 1) / wpc), dim3(wpc * 32), 0, st,
+                          "select_cert_kernel", a);
+}
+
+// Rows of up to kCertMaxNk blocks are selected from fp32 scores with fp64 resolution of
+// the uncertain band (keys in registers); longer rows from fp64 scores in shared memory.
+constexpr int kCertMaxNk = 32 * 64;
+
+// Labels, critical lists and the marginal indicator from the pooled means in w.qbar and
+// w.kbar. scores64 (nullable) receives the fp64 scores whenever it is given.
+template <int D>
+sla_status launch_router(const Shape& s, const Workspace& w, double* scores64, int8_t* mask, int32_t* crit,
+                         int crit_ld, __nv_bfloat16* W, cudaStream_t st) {
+  if (s.Nk <= kCertMaxNk) {
+    if (scores64) SLA_TRY(launch_scores<D>(w.qbar, w.kbar, scores64, s, st));
+    SLA_TRY(launch_scores32<D>(s, w, st));
+    CertArgs a{};
+    a.S32 = w.S32;
+    a.nq = w.nq;
+    a.nk = w.nk;
+    a.qbar = w.qbar;
+    a.kbar = w.kbar;
+    a.rows = s.BH * s.Nq;
+    a.Nq = s.Nq;
+    a.Nk = s.Nk;
+    a.kc = s.kc;
+    a.kn = s.kn;
+    a.mask = mask;
+    a.crit = crit;
+    a.crit_ld = crit_ld;
+    a.crit_cnt = w.crit_cnt;
+    a.W = W;
+    a.w_ld = s.w_ld;
+    if (s.Nk <= 32 * 8) return launch_cert<8, D>(a, st);
+    if (s.Nk <= 32 * 16) return launch_cert<16, D>(a, st);
+    if (s.Nk <= 32 * 32) return launch_cert<32, D>(a, st);
+    return launch_cert<64, D>(a, st);
+  }
+  double* S = scores64 ? scores64 : w.S;
+  SLA_TRY(launch_scores<D>(w.qbar, w.kbar, S, s, st));
+  SelectArgs a{};
+  a.S = S;
+  a.rows = s.BH * s.Nq;
+  a.Nk = s.Nk;
+  a.kc = s.kc;
+  a.kn = s.kn;
+  a.mask = mask;
+  a.crit = crit;
+  a.crit_ld = crit_ld;
+  a.crit_cnt = w.crit_cnt;
+  a.W = W;
+  a.w_ld = s.w_ld;
   const size_t per_warp = static_cast<size_t>(a.Nk) * 8;
   int wpc = static_cast<int>((200 * 1024) / per_warp);
   wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
@@ -362,21 +420,8 @@ sla_status route_impl(const Shape& s, const void* q, const void* k, int8_t* mask
                       double* scores_out, const Workspace& w, cudaStream_t st) {
   SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
   SLA_TRY(launch_pool<D>(k, w.kbar, s, s.bk, s.Nk, st));
-  double* S = scores_out ? scores_out : w.S;
-  SLA_TRY(launch_scores<D>(w.qbar, w.kbar, S, s, st));
-  SelectArgs a{};
-  a.S = S;
-  a.rows = s.BH * s.Nq;
-  a.Nk = s.Nk;
-  a.kc = s.kc;
-  a.kn = s.kn;
-  a.mask = mask_out;
-  a.crit = crit_out ? crit_out : w.crit;
-  a.crit_ld = crit_out ? s.kc : s.Nk;
-  a.crit_cnt = w.crit_cnt;
-  a.W = nullptr;
-  a.w_ld = s.w_ld;
-  return launch_select(a, st);
+  return launch_router<D>(s, w, scores_out, mask_out, crit_out ? crit_out : w.crit, crit_out ? s.kc : s.Nk, nullptr,
+                          st);
 }
 
 // Stage boundaries for sla_forward_timed: ev[0] before the per-block precompute,
@@ -416,20 +461,7 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
   } else {
     SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
     SLA_TRY(ev.mark(1, st));
-    SLA_TRY(launch_scores<D>(w.qbar, w.kbar, w.S, s, st));
-    SelectArgs a{};
-    a.S = w.S;
-    a.rows = s.BH * s.Nq;
-    a.Nk = s.Nk;
-    a.kc = s.kc;
-    a.kn = s.kn;
-    a.mask = w.mask;
-    a.crit = w.crit;
-    a.crit_ld = s.Nk;
-    a.crit_cnt = w.crit_cnt;
-    a.W = w.W;
-    a.w_ld = s.w_ld;
-    SLA_TRY(launch_select(a, st));
+    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
   }
   SLA_TRY(ev.mark(2, st));
   SLA_TRY(launch_agg<D>(s, w, st));
@@ -633,10 +665,15 @@ extern "C" sla_status sla_route_noalloc(const sla_problem* p, const void* q, con
   const size_t BH = s.BH;
   const size_t qbar_b = align256(BH * s.Nq * s.D * sizeof(double));
   const size_t kbar_b = align256(BH * s.Nk * s.D * sizeof(double));
-  const size_t S_b = scores_out ? 0 : align256(BH * s.Nq * s.Nk * sizeof(double));
+  // Scores: fp32 for the certified selection (rows of up to kCertMaxNk blocks), else
+  // fp64 unless the caller's scores_out holds them.
+  const size_t S_b = s.Nk <= kCertMaxNk ? align256(BH * s.Nq * s.Nk * sizeof(float))
+                                        : (scores_out ? 0 : align256(BH * s.Nq * s.Nk * sizeof(double)));
+  const size_t nq_b = align256(BH * s.Nq * sizeof(float));
+  const size_t nk_b = align256(BH * s.Nk * sizeof(float));
   const size_t crit_b = crit_idx_out ? 0 : align256(BH * s.Nq * s.Nk * sizeof(int32_t));
   const size_t cnt_b = align256(BH * s.Nq * sizeof(int32_t));
-  const size_t need = qbar_b + kbar_b + S_b + crit_b + cnt_b;
+  const size_t need = qbar_b + kbar_b + S_b + nq_b + nk_b + crit_b + cnt_b;
   if (need > kRouteScratchBytes)
     return fail(SLA_ERR_WORKSPACE,
                 "sla_route_noalloc: this problem needs %zu bytes of scratch, above the built-in maximum of %zu "
@@ -646,11 +683,20 @@ extern "C" sla_status sla_route_noalloc(const sla_problem* p, const void* q, con
   SLA_TRY(route_scratch_address(&base));
   uint8_t* b = static_cast<uint8_t*>(base);
   Workspace w{};
-  w.qbar = reinterpret_cast<double*>(b);
-  w.kbar = reinterpret_cast<double*>(b + qbar_b);
-  w.S = S_b ? reinterpret_cast<double*>(b + qbar_b + kbar_b) : nullptr;
-  w.crit = crit_b ? reinterpret_cast<int32_t*>(b + qbar_b + kbar_b + S_b) : nullptr;
-  w.crit_cnt = reinterpret_cast<int32_t*>(b + qbar_b + kbar_b + S_b + crit_b);
+  size_t off = 0;
+  auto piece = [&](size_t bytes) {
+    uint8_t* p = bytes ? b + off : nullptr;
+    off += bytes;
+    return p;
+  };
+  w.qbar = reinterpret_cast<double*>(piece(qbar_b));
+  w.kbar = reinterpret_cast<double*>(piece(kbar_b));
+  w.S = reinterpret_cast<double*>(piece(S_b));
+  w.S32 = reinterpret_cast<float*>(w.S);
+  w.nq = reinterpret_cast<float*>(piece(nq_b));
+  w.nk = reinterpret_cast<float*>(piece(nk_b));
+  w.crit = reinterpret_cast<int32_t*>(piece(crit_b));
+  w.crit_cnt = reinterpret_cast<int32_t*>(piece(cnt_b));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.D == 64) return route_impl<64>(s, q, k, mask_out, crit_idx_out, scores_out, w, st);
   return route_impl<128>(s, q, k, mask_out, crit_idx_out, scores_out, w, st);
