@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(320, 2)
   __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ float sZ[D], sAlpha[D];
+  __shared__ __align__(16) float sZ[D];
+  __shared__ __align__(16) float sAlpha[D];
   __shared__ float red_max[2][2][128];  // [block parity][half][row]
   __shared__ float red_l[2][128], red_den[2][128];
 
@@ -292,9 +293,15 @@ __global__ void __launch_bounds__(320, 2)
             for (int c = 0; c < 32; ++c)
               if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
           }
-          mx = __uint_as_float(sv[0]);
+          // two independent chains of 3-input maxima
+          float m0 = fmax3(__uint_as_float(sv[0]), __uint_as_float(sv[1]), __uint_as_float(sv[2]));
+          float m1 = fmax3(__uint_as_float(sv[3]), __uint_as_float(sv[4]), __uint_as_float(sv[5]));
 #pragma unroll
-          for (int c = 1; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
+          for (int c = 6; c < 30; c += 4) {
+            m0 = fmax3(m0, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+            m1 = fmax3(m1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+          }
+          mx = fmax3(m0, m1, fmaxf(__uint_as_float(sv[30]), __uint_as_float(sv[31])));
         }
         red_max[b][g][r] = mx;
         if (!(ok = named_barrier_and(1, 256, ok))) break;
@@ -314,26 +321,32 @@ __global__ void __launch_bounds__(320, 2)
             uint32_t o[16];
             tmem_ld16(lane_addr + OS + g * (D / 2) + c0, o);
             tmem_wait_ld();
+            const uint64_t f2 = f2_make(f, f);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+            for (int c = 0; c < 16; c += 2) {
+              const uint64_t y = f2_mul(static_cast<uint64_t>(o[c]) | (static_cast<uint64_t>(o[c + 1]) << 32), f2);
+              o[c] = static_cast<uint32_t>(y);
+              o[c + 1] = static_cast<uint32_t>(y >> 32);
+            }
             tmem_st16(lane_addr + OS + g * (D / 2) + c0, o);
           }
           tmem_wait_st();
           l_run *= f;
           m_run = m_new;
         }
-        // p = 2^(s * scale - m): one FMA and one exponential per element
-        float ps0 = 0.f, ps1 = 0.f;
+        // p = 2^(s * scale - m): one paired FMA per two elements and one exponential per
+        // element; the even and odd columns are summed in the two lanes of a paired add.
+        const uint64_t sc2 = f2_make(sc, sc), nm2 = f2_make(-m_run, -m_run);
+        uint64_t ps2 = 0ull;
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float e0 = fast_exp2(fmaf(__uint_as_float(sv[c]), sc, -m_run));
-          const float e1 = fast_exp2(fmaf(__uint_as_float(sv[c + 1]), sc, -m_run));
-          ps0 += e0;
-          ps1 += e1;
+          const uint64_t x2 = f2_fma(static_cast<uint64_t>(sv[c]) | (static_cast<uint64_t>(sv[c + 1]) << 32), sc2, nm2);
+          const float e0 = fast_exp2(f2_lo(x2)), e1 = fast_exp2(f2_hi(x2));
+          ps2 = f2_add(ps2, f2_make(e0, e1));
           pk[c >> 1] = pack_bf16x2(e0, e1);
         }
-        l_run += ps0 + ps1;
+        l_run += f2_lo(ps2) + f2_hi(ps2);
         tmem_st16(lane_addr + b * 64 + g * 16, pk);  // this half of P over the S columns
         tmem_wait_st();
         tc_fence_before();
@@ -346,27 +359,39 @@ __global__ void __launch_bounds__(320, 2)
 
       // phi(Q) in place (bf16) over this half of the row, and this half of the linear-branch
       // denominator phi(q) . Z_i with the same rounded phi(q) the MMA sees.
-      float den = 0.f;
+      // Column pairs in paired arithmetic: phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e);
+      // the even and odd columns' products with Z_i are summed in the two lanes.
+      uint64_t den2 = 0ull;
       if (ok) {
+        const uint64_t one2 = f2_make(1.f, 1.f), log2e2 = f2_make(1.4426950408889634f, 1.4426950408889634f);
 #pragma unroll 2
         for (int c8 = g * (D / 16); c8 < (g + 1) * (D / 16); ++c8) {
           uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
           uint4 u = *p;
           uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          const uint4 z01 = *reinterpret_cast<const uint4*>(&sZ[c8 * 8]);
+          const uint4 z23 = *reinterpret_cast<const uint4*>(&sZ[c8 * 8 + 4]);
+          const uint64_t z2[4] = {static_cast<uint64_t>(z01.x) | (static_cast<uint64_t>(z01.y) << 32),
+                                  static_cast<uint64_t>(z01.z) | (static_cast<uint64_t>(z01.w) << 32),
+                                  static_cast<uint64_t>(z23.x) | (static_cast<uint64_t>(z23.y) << 32),
+                                  static_cast<uint64_t>(z23.z) | (static_cast<uint64_t>(z23.w) << 32)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float2 f = unpack_bf16x2(w[e]);
-            const float g0 = f.x > 0.f ? f.x + 1.f : __expf(f.x);
-            const float g1 = f.y > 0.f ? f.y + 1.f : __expf(f.y);
+            // bf16 -> fp32 is a shift into the high half-word
+            const uint64_t x2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
+            const uint64_t pos2 = f2_add(x2, one2);
+            const uint64_t t2 = f2_mul(x2, log2e2);
+            const float g0 = f2_lo(x2) > 0.f ? f2_lo(pos2) : fast_exp2(f2_lo(t2));
+            const float g1 = f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
             w[e] = pack_bf16x2(g0, g1);
-            const float2 gr = unpack_bf16x2(w[e]);
-            den = fmaf(gr.x, sZ[c8 * 8 + 2 * e], den);
-            den = fmaf(gr.y, sZ[c8 * 8 + 2 * e + 1], den);
+            const uint64_t gr2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
+            den2 = f2_fma(gr2, z2[e], den2);
           }
           *p = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
       }
+      const float den = f2_lo(den2) + f2_hi(den2);
       red_l[g][r] = l_run;
       red_den[g][r] = den;
       tc_fence_before();
@@ -383,21 +408,24 @@ __global__ void __launch_bounds__(320, 2)
       const int tok = i * a.block_q + r;
       const bool store = r < a.block_q && tok < a.N;
       __nv_bfloat16* orow = a.out + (static_cast<size_t>(bh) * a.N + tok) * D;
+      // per column pair: y = (alpha inv_l) O_s + ((1 - alpha) inv_d) O_l in paired arithmetic;
+      // O_s is not read when the critical set is empty (its TMEM columns were never written)
+      const uint64_t il2 = f2_make(inv_l, inv_l), id2 = f2_make(inv_d, inv_d);
 #pragma unroll 1
       for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 16) {
         uint32_t os[16], ol[16];
-        tmem_ld16(lane_addr + OS + c0, os);
+        if (kc > 0) tmem_ld16(lane_addr + OS + c0, os);
         tmem_ld16(lane_addr + OL + c0, ol);
         tmem_wait_ld();
         uint32_t pk[8];
 #pragma unroll
         for (int c = 0; c < 16; c += 2) {
-          const float al0 = sAlpha[c0 + c], al1 = sAlpha[c0 + c + 1];
-          const float y0 = al0 * (kc > 0 ? __uint_as_float(os[c]) * inv_l : 0.f) +
-                           (1.f - al0) * (__uint_as_float(ol[c]) * inv_d);
-          const float y1 = al1 * (kc > 0 ? __uint_as_float(os[c + 1]) * inv_l : 0.f) +
-                           (1.f - al1) * (__uint_as_float(ol[c + 1]) * inv_d);
-          pk[c >> 1] = pack_bf16x2(y0, y1);
+          const uint64_t al2 = *reinterpret_cast<const uint64_t*>(&sAlpha[c0 + c]);
+          const uint64_t wl = f2_fma(al2 ^ 0x8000000080000000ull, id2, id2);  // (1 - alpha) inv_d
+          uint64_t y = f2_mul(wl, static_cast<uint64_t>(ol[c]) | (static_cast<uint64_t>(ol[c + 1]) << 32));
+          if (kc > 0)
+            y = f2_fma(f2_mul(al2, il2), static_cast<uint64_t>(os[c]) | (static_cast<uint64_t>(os[c + 1]) << 32), y);
+          pk[c >> 1] = pack_bf16x2(f2_lo(y), f2_hi(y));
         }
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c0);

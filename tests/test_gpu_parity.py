@@ -187,3 +187,63 @@ def test_bad_caller_mask_is_reported(cuda_device):
         binding.check(ws)
     assert e.value.status == 6
     binding.check(ws)  # the error word was cleared
+
+
+def _clustered_keys(N, D, seed):
+    """Inputs whose compressed scores tie in fp32 but not in fp64.
+
+    Every KV block is the same random block except in one channel d*, where the
+    block's first token carries a perturbation delta_j (exactly representable in
+    bf16) and the rest are zero; every query token has 1.0 in channel d*. So
+    S_j = S_base + delta_j / (64 sqrt(D)). A quarter of the blocks get large
+    positive deltas, a quarter large negative ones, and half get deltas of
+    m * 2^-30 with m in [-40, 40) (many exact repeats): their scores agree to
+    ~1e-12, far below fp32 resolution, so the labels inside that cluster are
+    decided by fp64 scores and then by index.
+    """
+    g = torch.Generator().manual_seed(seed)
+    Nk = N // 64
+    dstar = 5
+    base = torch.randn(64, D, generator=g)
+    base[:, dstar] = 0.0
+    k = base.repeat(Nk, 1)
+    m_small = torch.randint(-40, 40, (Nk,), generator=g).double()
+    m_big = torch.randint(1, 120, (Nk,), generator=g).double()
+    j = torch.arange(Nk)
+    delta = torch.where(j % 2 == 0, m_small * 2.0 ** -30,
+                        torch.where(j % 4 == 1, m_big * 2.0 ** -4, -m_big * 2.0 ** -4))
+    k[j * 64, dstar] = delta.float()
+    q = torch.randn(N, D, generator=g)
+    q[:, dstar] = 1.0
+    v = torch.randn(N, D, generator=g)
+    kb = k.to(torch.bfloat16)
+    assert torch.equal(kb[j * 64, dstar].double(), delta), "perturbations must be exact in bf16"
+    return q.to(torch.bfloat16), kb, v.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("N, D, bq, kh, kl", [(32768, 128, 128, 0.5, 0.375), (8192, 64, 64, 0.375, 0.375),
+                                              (32768, 128, 128, 0.3, 0.45)])
+def test_router_resolves_fp32_ties_in_fp64(cuda_device, N, D, bq, kh, kl):
+    """Labels inside a cluster of scores that fp32 cannot tell apart match the oracle exactly."""
+    q, k, v = _clustered_keys(N, D, seed=N + D)
+    rm, S = oracle.route(q, k, bq, 64, kh, kl)
+    Nk = N // 64
+    # the construction is meaningful: the boundaries fall inside the cluster, where fp32 ties
+    s32 = S.astype(np.float32)
+    clustered = np.arange(Nk) % 2 == 0
+    assert np.all(s32[:, clustered] == s32[:, clustered][:, :1]) or np.ptp(s32[:, clustered], axis=1).max() <= \
+        4 * np.spacing(np.abs(s32).max())
+    assert np.all((rm[:, clustered] == 2).any(-1)) and np.all((rm[:, clustered] == 1).any(-1))
+    qd, kd = q[None, None].to(cuda_device), k[None, None].to(cuda_device)
+    mask, crit, _ = binding.route(qd, kd, bq, 64, kh, kl, want_scores=True, want_crit=True)
+    gm = mask[0, 0].cpu().numpy()
+    assert np.array_equal(gm, rm), f"{int((gm != rm).sum())} labels differ inside an fp32 tie cluster"
+    gc = crit[0, 0].cpu().numpy()
+    for i in range(gm.shape[0]):
+        np.testing.assert_array_equal(gc[i], np.nonzero(rm[i] == 2)[0])
+    # the fused forward's own router gives the same labels (through the forward output)
+    alpha = torch.rand(1, D, generator=torch.Generator().manual_seed(1)).to(cuda_device)
+    vd = v[None, None].to(cuda_device)
+    o_int = binding.forward(qd, kd, vd, alpha, bq, 64, kh, kl)
+    o_ext = binding.forward(qd, kd, vd, alpha, bq, 64, kh, kl, mask=torch.from_numpy(rm)[None, None].to(cuda_device))
+    assert torch.equal(o_int, o_ext)
