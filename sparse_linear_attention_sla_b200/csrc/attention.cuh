@@ -14,19 +14,18 @@
 // item 1 (the sparse branch renormalises over its keys) and §2.A
 // (O = alpha * O_s + (1 - alpha) * O_l).
 //
-// Persistent: two CTAs per SM (<= 98 KB shared memory, 256 TMEM columns, <= 96
-// registers per thread each) walk the tiles t = blockIdx.x, blockIdx.x +
-// gridDim.x, ... in head-major order, so a head's K/V stay in L2 and the next
-// tile's loads overlap the current tile's epilogue. Warp roles (320 threads):
+// Persistent: two CTAs per SM (<= 98 KB shared memory, 256 TMEM columns, <= 168
+// registers per thread each) walk the tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// in head-major order, so a head's K/V stay in L2 and the next tile's loads overlap the
+// current tile's epilogue. Warp roles (192 threads):
 //   warp 0      TMA producer: per tile Q, then K_j / V_j of every critical block
 //               through a 2-slot ring, then H_i into the next slot (a pseudo-block
 //               of the ring: its two halves complete the slot's K and V barriers).
 //   warp 1      TMEM owner and single-thread tcgen05 issuer:
 //               S = Q K_j^T (M=128, N=64), O_s += P V_j (M=128, N=D, P read from
 //               TMEM), O_l = phi(Q) H_i (M=128, N=D).
-//   warps 2..9  two softmax / epilogue warpgroups: a thread owns one query row
-//               (= TMEM lane) and one half of the columns; the two threads of a
-//               row exchange their block maxima through shared memory.
+//   warps 2..5  softmax / epilogue warpgroup: a thread owns one query row (= TMEM lane)
+//               and all 64 columns of each S block; S_{n+1} is loaded while P_n is stored.
 //
 // TMEM columns: S ping-pong [0,64) [64,128) (P, bf16, is written back over the
 // first 32 columns of its S), O_s [128,128+D); after a tile's sparse loop O_l
@@ -68,7 +67,7 @@ struct AttnSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 2)
+__global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h, AttnArgs a) {
   using L = AttnSmem<D>;
@@ -87,17 +86,15 @@ __global__ void __launch_bounds__(320, 2)
   __shared__ int abort_flag;
   __shared__ __align__(16) float sZ[D];
   __shared__ __align__(16) float sAlpha[D];
-  __shared__ float red_max[2][2][128];  // [block parity][half][row]
-  __shared__ float red_l[2][128], red_den[2][128];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
     mbar_init(&q_free, 1);
-    mbar_init(&phiq_full, 256);
+    mbar_init(&phiq_full, 128);
     mbar_init(&ol_done, 1);
-    mbar_init(&tmem_free, 256);
+    mbar_init(&tmem_free, 128);
     mbar_init(&drain, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&k_full[s], 1);
@@ -105,7 +102,7 @@ __global__ void __launch_bounds__(320, 2)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 256);
+      mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
     }
     abort_flag = 0;
@@ -252,83 +249,90 @@ __global__ void __launch_bounds__(320, 2)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax / epilogue warpgroups
-    const int wt = tid - 64;                    // 0..255
-    const int g = wt >> 7;                      // column half owned by this warpgroup
+    // ------------------------------------------------------------ softmax / epilogue warpgroup
+    // Thread = query row r = TMEM lane; it owns all 64 columns of every S block. The load of
+    // S_{n+1} is issued before P_n is published, so its latency overlaps the store of P_n.
     const int quarter = warp & 3;               // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;          // query row within the tile
+    const int wt = tid - 64;                    // 0..127
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float sc = a.scale_log2;
     uint32_t ns = 0;  // S/P blocks so far
     bool ok = true;
     int k = 0;
-    // Every barrier between the two warpgroups ANDs the threads' status, so a failed
-    // wait makes all 256 threads leave together.
+    // Every barrier of the warpgroup ANDs the threads' status, so a failed wait makes all
+    // 128 threads leave together.
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++k) {
       const int bh = t / a.Nq, i = t % a.Nq, h = bh % a.H;
       const int kc = a.crit_cnt[t];
       const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
-      if (!named_barrier_and(1, 256, ok)) break;  // the previous tile's epilogue is done with sZ / sAlpha
-      for (int c = wt; c < D; c += 256) {
+      if (!named_barrier_and(1, 128, ok)) break;  // the previous tile's epilogue is done with sZ / sAlpha
+      for (int c = wt; c < D; c += 128) {
         sZ[c] = a.Zagg[static_cast<size_t>(t) * D + c];
         sAlpha[c] = a.alpha[h * D + c];
       }
-      if (!named_barrier_and(1, 256, ok)) break;  // sZ / sAlpha of this tile are visible
-      float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and this half's row sum
-      int j_next = kc > 0 ? clist[0] : 0;   // critical-block index, read one iteration ahead
-      for (int n = 0; n < kc; ++n, ++ns) {
-        const int b = ns & 1;
-        ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[b], (ns >> 1) & 1, a.err, &abort_flag));
-        uint32_t sv[32];
-        float mx = -INFINITY;
-        const int j_cur = j_next;
-        if (n + 1 < kc) j_next = clist[n + 1];
+      if (!named_barrier_and(1, 128, ok)) break;  // sZ / sAlpha of this tile are visible
+      float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and row sum
+      uint32_t sa[32], sb[32];               // S columns [0, 32) and [32, 64) of the current block
+      int j_cur = kc > 0 ? clist[0] : 0;
+      if (kc > 0) {
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[ns & 1], (ns >> 1) & 1, a.err, &abort_flag));
         if (ok) {
           tc_fence_after();
-          tmem_ld32(lane_addr + b * 64 + g * 32, sv);
+          tmem_ld32(lane_addr + (ns & 1) * 64, sa);
+          tmem_ld32(lane_addr + (ns & 1) * 64 + 32, sb);
           tmem_wait_ld();
-          const int valid = min(64, a.N - j_cur * 64) - g * 32;  // valid columns in this half
-          if (valid < 32) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (c >= valid) sv[c] = __float_as_uint(-INFINITY);
-          }
-          // two independent chains of 3-input maxima
-          float m0 = fmax3(__uint_as_float(sv[0]), __uint_as_float(sv[1]), __uint_as_float(sv[2]));
-          float m1 = fmax3(__uint_as_float(sv[3]), __uint_as_float(sv[4]), __uint_as_float(sv[5]));
-#pragma unroll
-          for (int c = 6; c < 30; c += 4) {
-            m0 = fmax3(m0, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
-            m1 = fmax3(m1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
-          }
-          mx = fmax3(m0, m1, fmaxf(__uint_as_float(sv[30]), __uint_as_float(sv[31])));
         }
-        red_max[b][g][r] = mx;
-        if (!(ok = named_barrier_and(1, 256, ok))) break;
-        mx = fmaxf(mx, red_max[b][g ^ 1][r]) * sc;
+      }
+      for (int n = 0; ok && n < kc; ++n, ++ns) {
+        const int b = ns & 1;
+        const int j_next = n + 1 < kc ? clist[n + 1] : 0;
+        const int valid = min(64, a.N - j_cur * 64);  // valid key columns of this block
+        if (valid < 64) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (c >= valid) sa[c] = __float_as_uint(-INFINITY);
+            if (c + 32 >= valid) sb[c] = __float_as_uint(-INFINITY);
+          }
+        }
+        // row maximum: four independent chains of 3-input maxima
+        float m0 = fmax3(__uint_as_float(sa[0]), __uint_as_float(sa[1]), __uint_as_float(sa[2]));
+        float m1 = fmax3(__uint_as_float(sa[3]), __uint_as_float(sa[4]), __uint_as_float(sa[5]));
+        float m2 = fmax3(__uint_as_float(sb[0]), __uint_as_float(sb[1]), __uint_as_float(sb[2]));
+        float m3 = fmax3(__uint_as_float(sb[3]), __uint_as_float(sb[4]), __uint_as_float(sb[5]));
+#pragma unroll
+        for (int c = 6; c < 30; c += 4) {
+          m0 = fmax3(m0, __uint_as_float(sa[c]), __uint_as_float(sa[c + 1]));
+          m1 = fmax3(m1, __uint_as_float(sa[c + 2]), __uint_as_float(sa[c + 3]));
+          m2 = fmax3(m2, __uint_as_float(sb[c]), __uint_as_float(sb[c + 1]));
+          m3 = fmax3(m3, __uint_as_float(sb[c + 2]), __uint_as_float(sb[c + 3]));
+        }
+        m0 = fmax3(m0, __uint_as_float(sa[30]), __uint_as_float(sa[31]));
+        m2 = fmax3(m2, __uint_as_float(sb[30]), __uint_as_float(sb[31]));
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sc;
         if (n == 0) {
           m_run = mx;
         } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
-          // The running maximum grew by more than 2^8: rescale this half of O_s (needs PV of
-          // the previous block finished). The partner thread of the row decides identically.
+          // The running maximum grew by more than 2^8: rescale the row of O_s (needs P*V of
+          // the previous block finished).
           ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
-          if (!ok) continue;  // the next barrier takes every thread out
+          if (!ok) break;
           tc_fence_after();
           const float m_new = fmaxf(m_run, mx);
           const float f = fast_exp2(m_run - m_new);
-#pragma unroll
-          for (int c0 = 0; c0 < D / 2; c0 += 16) {
+          const uint64_t f2 = f2_make(f, f);
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 16) {
             uint32_t o[16];
-            tmem_ld16(lane_addr + OS + g * (D / 2) + c0, o);
+            tmem_ld16(lane_addr + OS + c0, o);
             tmem_wait_ld();
-            const uint64_t f2 = f2_make(f, f);
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
               const uint64_t y = f2_mul(static_cast<uint64_t>(o[c]) | (static_cast<uint64_t>(o[c + 1]) << 32), f2);
               o[c] = static_cast<uint32_t>(y);
               o[c + 1] = static_cast<uint32_t>(y >> 32);
             }
-            tmem_st16(lane_addr + OS + g * (D / 2) + c0, o);
+            tmem_st16(lane_addr + OS + c0, o);
           }
           tmem_wait_st();
           l_run *= f;
@@ -337,35 +341,51 @@ __global__ void __launch_bounds__(320, 2)
         // p = 2^(s * scale - m): one paired FMA per two elements and one exponential per
         // element; the even and odd columns are summed in the two lanes of a paired add.
         const uint64_t sc2 = f2_make(sc, sc), nm2 = f2_make(-m_run, -m_run);
-        uint64_t ps2 = 0ull;
-        uint32_t pk[16];
+        uint64_t ps2 = 0ull, ps2b = 0ull;
+        uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const uint64_t x2 = f2_fma(static_cast<uint64_t>(sv[c]) | (static_cast<uint64_t>(sv[c + 1]) << 32), sc2, nm2);
+          const uint64_t x2 = f2_fma(static_cast<uint64_t>(sa[c]) | (static_cast<uint64_t>(sa[c + 1]) << 32), sc2, nm2);
+          const uint64_t y2 = f2_fma(static_cast<uint64_t>(sb[c]) | (static_cast<uint64_t>(sb[c + 1]) << 32), sc2, nm2);
           const float e0 = fast_exp2(f2_lo(x2)), e1 = fast_exp2(f2_hi(x2));
+          const float e2 = fast_exp2(f2_lo(y2)), e3 = fast_exp2(f2_hi(y2));
           ps2 = f2_add(ps2, f2_make(e0, e1));
+          ps2b = f2_add(ps2b, f2_make(e2, e3));
           pk[c >> 1] = pack_bf16x2(e0, e1);
+          pk[16 + (c >> 1)] = pack_bf16x2(e2, e3);
         }
-        l_run += f2_lo(ps2) + f2_hi(ps2);
-        tmem_st16(lane_addr + b * 64 + g * 16, pk);  // this half of P over the S columns
+        const uint64_t pst = f2_add(ps2, ps2b);
+        l_run += f2_lo(pst) + f2_hi(pst);
+        tmem_st32(lane_addr + b * 64, pk);  // P over the first 32 columns of its S
+        // the next block's S: its load overlaps the store of P
+        if (n + 1 < kc) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b ^ 1], ((ns + 1) >> 1) & 1, a.err, &abort_flag));
+          if (ok) {
+            tc_fence_after();
+            tmem_ld32(lane_addr + (b ^ 1) * 64, sa);
+            tmem_ld32(lane_addr + (b ^ 1) * 64 + 32, sb);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
+        if (n + 1 < kc) tmem_wait_ld();
+        j_cur = j_next;
       }
       // Every MMA that reads Q (or the S/P columns) has finished once the last PV has.
       if (ok && kc > 0)
         ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, k & 1, a.err, &abort_flag));
 
-      // phi(Q) in place (bf16) over this half of the row, and this half of the linear-branch
-      // denominator phi(q) . Z_i with the same rounded phi(q) the MMA sees.
-      // Column pairs in paired arithmetic: phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e);
-      // the even and odd columns' products with Z_i are summed in the two lanes.
+      // phi(Q) in place (bf16) over the row, and the linear-branch denominator phi(q) . Z_i
+      // with the same rounded phi(q) the MMA sees. Column pairs in paired arithmetic:
+      // phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e); even and odd columns' products
+      // with Z_i are summed in the two lanes.
       uint64_t den2 = 0ull;
       if (ok) {
         const uint64_t one2 = f2_make(1.f, 1.f), log2e2 = f2_make(1.4426950408889634f, 1.4426950408889634f);
 #pragma unroll 2
-        for (int c8 = g * (D / 16); c8 < (g + 1) * (D / 16); ++c8) {
+        for (int c8 = 0; c8 < D / 8; ++c8) {
           uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
           uint4 u = *p;
           uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -391,19 +411,15 @@ __global__ void __launch_bounds__(320, 2)
         }
         fence_proxy_async_smem();
       }
-      const float den = f2_lo(den2) + f2_hi(den2);
-      red_l[g][r] = l_run;
-      red_den[g][r] = den;
+      const float den_tot = f2_lo(den2) + f2_hi(den2);
       tc_fence_before();
       mbar_arrive(&phiq_full);
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, k & 1, a.err, &abort_flag));
-      if (!(ok = named_barrier_and(1, 256, ok))) break;  // both halves' sums are in shared memory
-      const float l_tot = red_l[0][r] + red_l[1][r];
-      const float den_tot = red_den[0][r] + red_den[1][r];
+      if (!(ok = named_barrier_and(1, 128, ok))) break;
 
       // Epilogue: O = alpha * O_s / l + (1 - alpha) * O_l / den, bf16, straight to global memory.
       tc_fence_after();
-      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const float inv_d = den_tot > 0.f ? 1.f / den_tot : 0.f;
       const int tok = i * a.block_q + r;
       const bool store = r < a.block_q && tok < a.N;
@@ -412,7 +428,7 @@ __global__ void __launch_bounds__(320, 2)
       // O_s is not read when the critical set is empty (its TMEM columns were never written)
       const uint64_t il2 = f2_make(inv_l, inv_l), id2 = f2_make(inv_d, inv_d);
 #pragma unroll 1
-      for (int c0 = g * (D / 2); c0 < (g + 1) * (D / 2); c0 += 16) {
+      for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t os[16], ol[16];
         if (kc > 0) tmem_ld16(lane_addr + OS + c0, os);
         tmem_ld16(lane_addr + OL + c0, ol);

@@ -410,7 +410,7 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.err = w.err;
   // persistent: two CTAs per SM walk the tiles
   const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
-  return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(320), smem, st, "attn_kernel", mq, mk, mv, mh, a);
+  return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, a);
 }
 
 // ------------------------------------------------------------------ entry points (templated on D)
