@@ -29,13 +29,14 @@ constexpr int kAggStages = 3;
 constexpr uint32_t kAggStageBytes = 3 * 16384;  // A for two M-tiles + one B tile (64 x 128)
 constexpr uint32_t kAggStagingBytes = 65536;    // bf16 output tile: 2 M-tiles x 128 rows x 128 columns
 
-// Persistent, one CTA per SM, 192 threads: warp 0 TMA producer, warp 1 tcgen05 issuer,
-// warps 2..5 epilogue (TMEM -> bf16 -> shared-memory staging -> TMA store). A tile is 128 state columns x up to two 128-row M-tiles of query
+// Persistent, one CTA per SM, 224 threads: warp 0 TMA producer, warps 1 and 6 tcgen05
+// issuers (one per M-tile), warps 2..5 epilogue (TMEM -> bf16 -> shared-memory staging ->
+// TMA store). A tile is 128 state columns x up to two 128-row M-tiles of query
 // blocks of one head (so each stacked-state tile is read once per head); tiles are walked
 // columns-fastest. Accumulators are double-buffered in TMEM (2 x 256 columns, M-tile t of
 // buffer b at column 256 b + 128 t) so the epilogue of a tile overlaps the next mainloop.
 template <int D>
-__global__ void __launch_bounds__(192, 1) agg_kernel(const __grid_constant__ CUtensorMap map_w,
+__global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUtensorMap map_w,
                                                      const __grid_constant__ CUtensorMap map_h,
                                                      const __grid_constant__ CUtensorMap map_out, AggArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -51,13 +52,13 @@ __global__ void __launch_bounds__(192, 1) agg_kernel(const __grid_constant__ CUt
   if (tid == 0) {
     for (int s = 0; s < kAggStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);  // one commit from each issuer
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_full[b], 2);
       mbar_init(&acc_empty[b], 128);
     }
-    mbar_init(&drain, 1);
+    mbar_init(&drain, 2);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -106,38 +107,42 @@ __global__ void __launch_bounds__(192, 1) agg_kernel(const __grid_constant__ CUt
           if (last_round[s] >= 0) mbar_wait(&full[s], last_round[s] & 1, nullptr, nullptr);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);
-      uint32_t sc = 0;
-      int tc = 0;  // tiles issued
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tc) {
-        int n0, m0, bh, nm;
-        decode(t, n0, m0, bh, nm);
-        const int ab = tc & 1;
-        if (tc >= 2 && !(ok = mbar_wait(&acc_empty[ab], ((tc >> 1) - 1) & 1, a.err, &abort_flag))) break;
-        for (int k = 0; k < nk; ++k, ++sc) {
-          const int s = sc % kAggStages;
-          if (!(ok = mbar_wait(&full[s], (sc / kAggStages) & 1, a.err, &abort_flag))) break;
-          tc_fence_after();
-          const uint32_t st = smem_u32(smem + s * kAggStageBytes);
+  } else if (warp == 1 || warp == 6) {
+    // Two tcgen05 issuers, one per M-tile: a warp's MMAs run one at a time, so two warps
+    // keep two accumulation chains in flight. The whole warp runs the loop; one lane issues.
+    const int tt = warp == 1 ? 0 : 1;
+    const uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);
+    uint32_t sc = 0;
+    int tc = 0;  // tiles issued
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++tc) {
+      int n0, m0, bh, nm;
+      decode(t, n0, m0, bh, nm);
+      const int ab = tc & 1;
+      if (tc >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&acc_empty[ab], ((tc >> 1) - 1) & 1, a.err, &abort_flag));
+      for (int k = 0; ok && k < nk; ++k, ++sc) {
+        const int s = sc % kAggStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (sc / kAggStages) & 1, a.err, &abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kAggStageBytes);
+        if (tt < nm) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bd = smem_desc_sw128(st + 32768 + kk * 2048, 8192, 1024);
-            for (int tt = 0; tt < nm; ++tt) {
-              const uint64_t ad = smem_desc_sw128(st + tt * 16384 + kk * 32, 16, 1024);
-              umma_bf16_ss(tmem + ab * 256 + 128 * tt, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
-            }
+            const uint64_t ad = smem_desc_sw128(st + tt * 16384 + kk * 32, 16, 1024);
+            if (elect_one()) umma_bf16_ss(tmem + ab * 256 + 128 * tt, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(&empty[s]);
         }
-        if (!ok) break;
-        umma_commit(&acc_full[ab]);
+        if (elect_one()) umma_commit(&empty[s]);  // both issuers release the stage
+        __syncwarp();
       }
-      umma_commit(&drain);
-      mbar_wait(&drain, 0, nullptr, nullptr);
+      if (!ok) break;
+      if (elect_one()) umma_commit(&acc_full[ab]);
+      __syncwarp();
     }
+    if (elect_one()) umma_commit(&drain);
+    mbar_wait(&drain, 0, nullptr, nullptr);
     __syncwarp();
   } else {
     // Epilogue: warp w (quarter w & 3) holds rows m0 + 128 t + 32 (w & 3) + lane of M-tile t.

@@ -376,7 +376,7 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
   AggArgs a{s.Nq, s.Nk, s.LD, s.BH, w.Hagg, w.Zagg, w.err};
   const long long tiles = static_cast<long long>(s.LD / 128) * ((s.Nq + 255) / 256) * s.BH;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  return launch_dependent(sla::agg_kernel<D>, dim3(grid), dim3(192), smem, st, "agg_kernel", mw, mh, mo, a);
+  return launch_dependent(sla::agg_kernel<D>, dim3(grid), dim3(224), smem, st, "agg_kernel", mw, mh, mo, a);
 }
 
 template <int D>
