@@ -80,9 +80,10 @@ struct PrepSmem {
 // Column pass of one warpgroup over a ROWS x D tile (16-byte chunks, 128-byte swizzle):
 // thread (cc, rg) owns columns 8cc..8cc+7 of rows rg, rg + RG, ...; it sums the valid
 // rows in fp64 and, for a K tile (PHI), sums phi(k) in fp32 and rewrites the tile in
-// place as phi(k) (zero past the sequence end). Partial sums go to part_d / part_f[rg].
+// place as phi(k) (zero past the sequence end). The row groups of a warp are summed with
+// shuffles; the warp's partial sums go to part_d / part_f[wq] (wq = warp within the group).
 template <int D, int ROWS, bool PHI>
-__device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int valid, double (*part_d)[D],
+__device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int wq, int valid, double (*part_d)[D],
                                             float (*part_f)[D]) {
   constexpr int RG = 128 / (D / 8);
   uint8_t* tile = tile0 + (cc / 8) * (ROWS * 128);
@@ -119,19 +120,29 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
     }
     if (PHI) *p = make_uint4(w[0], w[1], w[2], w[3]);
   }
+  // lanes that differ only in their row group hold the same columns
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    part_d[rg][cc * 8 + e] = ks[e];
-    part_f[rg][cc * 8 + e] = zs[e];
+  for (int o = D / 8; o < 32; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ks[e] += __shfl_xor_sync(0xffffffffu, ks[e], o);
+      zs[e] += __shfl_xor_sync(0xffffffffu, zs[e], o);
+    }
+  if ((threadIdx.x & 31) < D / 8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      part_d[wq][cc * 8 + e] = ks[e];
+      part_f[wq][cc * 8 + e] = zs[e];
+    }
   }
 }
 
-// Persistent, warp-specialised precompute; one CTA per SM, 448 threads.
+// Persistent, warp-specialised precompute; one CTA per SM, 576 threads.
 // A CTA walks the items g = blockIdx.x, blockIdx.x + gridDim.x, ... of the list
 // [KV blocks of every head | query blocks of every head (when qbar is set)].
 //   warp 0      TMA producer: K_j and V_j (or a query block) into a 4-slot ring
-//   warps 2..5 and 10..13
-//               two column-pass warpgroups taking alternate items: over 16-byte
+//   warps 2..5, 10..13 and 14..17
+//               three column-pass warpgroups taking items in turn: over 16-byte
 //               chunks, the sum of the valid rows in fp64 (block means), and for KV
 //               blocks the sum of phi(k) (z_j) while the K tile is rewritten in
 //               place as phi(k) (zero past the sequence end)
@@ -142,7 +153,7 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
 // For D = 64 the second half of phi(K)^T (rows 64..127 of the M=128 MMA) points
 // at a zero tile, so the result rows 64..127 are zero and ignored.
 template <int D>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(576, 1)
     prep_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_hout, PrepArgs a) {
   using L = PrepSmem<D>;
@@ -157,8 +168,8 @@ __global__ void __launch_bounds__(448, 1)
   __shared__ uint64_t full[NS], phi_done[NS], empty[NS], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ double part_d[2][RG][D];
-  __shared__ float part_f[2][RG][D];
+  __shared__ double part_d[3][4][D];  // [column warpgroup][warp][column]
+  __shared__ float part_f[3][4][D];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_kv = a.BH * a.Nk;
@@ -180,7 +191,7 @@ __global__ void __launch_bounds__(448, 1)
     fence_mbar_init();
   }
   if (D == 64) {
-    for (uint32_t o = tid * 16; o < L::ZERO; o += 448 * 16) *reinterpret_cast<uint4*>(zero + o) = make_uint4(0, 0, 0, 0);
+    for (uint32_t o = tid * 16; o < L::ZERO; o += 576 * 16) *reinterpret_cast<uint4*>(zero + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -258,12 +269,13 @@ __global__ void __launch_bounds__(448, 1)
     __syncwarp();
   } else if (warp < 6 || warp >= 10) {
     // ------------------------------------------------------------ column passes (2 x 128 threads)
-    const int cw = warp < 6 ? 0 : 1;         // this warpgroup takes the items with k % 2 == cw
-    const int wt = warp < 6 ? tid - 64 : tid - 320;
-    const int bar_id = cw == 0 ? 1 : 3;
+    const int cw = warp < 6 ? 0 : (warp < 14 ? 1 : 2);  // this warpgroup takes the items with k % 3 == cw
+    const int wt = tid - (cw == 0 ? 64 : (cw == 1 ? 320 : 448));
+    const int bar_id = cw == 0 ? 1 : (cw == 1 ? 3 : 4);
+    const int wq = wt >> 5;
     const int cc = wt % CPR, rg = wt / CPR;
     int k = cw;
-    for (int g = blockIdx.x + cw * gridDim.x; g < n_items; g += 2 * gridDim.x, k += 2) {
+    for (int g = blockIdx.x + cw * gridDim.x; g < n_items; g += 3 * gridDim.x, k += 3) {
       const int s = k % NS, r = k / NS;
       bool ok = mbar_wait(&full[s], r & 1, a.err, &abort_flag);
       if (!named_barrier_and(bar_id, 128, ok)) break;
@@ -283,11 +295,11 @@ __global__ void __launch_bounds__(448, 1)
       uint8_t* slotp = smem + s * L::SLOT;
       if (isq) {
         if (a.block_q == 128)
-          column_pass<D, 128, false>(slotp, cc, rg, valid, part_d[cw], part_f[cw]);
+          column_pass<D, 128, false>(slotp, cc, rg, wq, valid, part_d[cw], part_f[cw]);
         else
-          column_pass<D, 64, false>(slotp, cc, rg, valid, part_d[cw], part_f[cw]);
+          column_pass<D, 64, false>(slotp, cc, rg, wq, valid, part_d[cw], part_f[cw]);
       } else {
-        column_pass<D, 64, true>(slotp, cc, rg, valid, part_d[cw], part_f[cw]);
+        column_pass<D, 64, true>(slotp, cc, rg, wq, valid, part_d[cw], part_f[cw]);
       }
       if (!isq) fence_proxy_async_smem();
       named_barrier(bar_id, 128);
@@ -295,7 +307,7 @@ __global__ void __launch_bounds__(448, 1)
         double sum = 0.0;
         float zsum = 0.f;
 #pragma unroll
-        for (int q = 0; q < RG; ++q) {
+        for (int q = 0; q < 4; ++q) {
           sum += part_d[cw][q][wt];
           zsum += part_f[cw][q][wt];
         }

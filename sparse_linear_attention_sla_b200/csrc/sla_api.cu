@@ -265,7 +265,7 @@ sla_status launch_prep(const void* q, const void* k, const void* v, const Shape&
   SLA_TRY(allow_smem(sla::prep_kernel<D>, smem));
   const long long items = static_cast<long long>(s.BH) * s.Nk + (args.qbar ? static_cast<long long>(s.BH) * s.Nq : 0);
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
-  sla::prep_kernel<D><<<grid, 448, smem, st>>>(mq, mk, mv, mh, args);
+  sla::prep_kernel<D><<<grid, 576, smem, st>>>(mq, mk, mv, mh, args);
   return launched("prep_kernel");
 }
 
