@@ -338,7 +338,7 @@ def run_ours(args):
                      "bytes_alg": work["bytes"], "executed_tflops": round(work["flops"] / (ms_step * 1e-3) / 1e12, 2)}
 
     # End to end through the public call with host buffers (copies inside the timed region).
-    # One group per (batch, head); the host-to-device copy of group g+1, the forward of
+    # The heads are split into four groups; the host-to-device copy of group g+1, the forward of
     # group g and the device-to-host copy of group g-1 run on three streams and overlap
     # (PCIe is full duplex). Each group is one sla_forward call on a contiguous head range.
     e2e = None
@@ -349,7 +349,7 @@ def run_ours(args):
         dq, dk, dv, da = (torch.empty_like(t) for t in (q, k, v, alpha))
         h2d_stream, d2h_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         # groups of (batch, head range); every group is contiguous in the [B, H, N, D] layout
-        per = 1
+        per = max(1, w.H // 4)
         groups = [(b, h0, min(w.H, h0 + per)) for b in range(w.B) for h0 in range(0, w.H, per)]
 
         def e2e_step():

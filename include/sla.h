@@ -147,6 +147,21 @@ sla_status sla_check(void* ws, void* stream);
 sla_status sla_route_noalloc(const sla_problem* p, const void* q, const void* k, int8_t* mask_out,
                              int32_t* crit_idx_out, double* scores_out, void* stream);
 
+/* Self-test of the device-side failure path (no counterpart on the pages).
+ *
+ * Enqueues on `stream` one thread that waits on an mbarrier nothing ever arrives on,
+ * through the same bounded wait every kernel of the library uses, with a limit of
+ * limit_us microseconds instead of the kernels' 2 s. When the limit runs out the thread
+ * records the timeout in the workspace's error word and returns; no fault, trap or hang
+ * is involved and the context stays usable. A following sla_check on the same workspace
+ * returns SLA_ERR_TIMEOUT and clears the word.
+ *   ws, ws_bytes : a workspace (any problem's; only its 256-byte error word is used),
+ *                  256-byte aligned, at least 256 bytes.
+ *   limit_us     : 1 .. 1000000.
+ * Returns SLA_ERR_WORKSPACE or SLA_ERR_INVALID_ARG on bad arguments (nothing enqueued),
+ * SLA_ERR_CUDA if the launch fails, else SLA_OK. */
+sla_status sla_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned limit_us, void* stream);
+
 /* Message for the calling thread's most recent failed call ("" if none). */
 const char* sla_last_error(void);
 

@@ -27,7 +27,8 @@ _STATUS = {
 
 # Every symbol include/sla.h declares.
 EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sla_forward",
-           "sla_forward_timed", "sla_check", "sla_last_error", "sla_version", "sla_route_noalloc")
+           "sla_forward_timed", "sla_check", "sla_last_error", "sla_version", "sla_route_noalloc",
+           "sla_selftest_wait_timeout")
 
 
 class SlaError(RuntimeError):
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_forward_timed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(ctypes.c_float)]
         lib.sla_check.argtypes = [vp, vp]
+        lib.sla_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint, vp]
+        lib.sla_selftest_wait_timeout.restype = ctypes.c_int
         lib.sla_last_error.restype = ctypes.c_char_p
         lib.sla_version.restype = ctypes.c_char_p
         for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check"):
@@ -220,6 +223,15 @@ def check(ws: torch.Tensor):
     lib = load_library()
     with torch.cuda.device(ws.device):
         _raise(lib.sla_check(_ptr(ws), _stream_handle(ws.device)))
+
+
+def selftest_wait_timeout(ws: torch.Tensor, limit_us: int = 50000):
+    """Enqueue the device self-test of the bounded-wait path (see include/sla.h); a
+    following check(ws) raises SlaError with status SLA_ERR_TIMEOUT."""
+    lib = load_library()
+    with torch.cuda.device(ws.device):
+        _raise(lib.sla_selftest_wait_timeout(_ptr(ws), ctypes.c_size_t(ws.numel()), ctypes.c_uint(int(limit_us)),
+                                             _stream_handle(ws.device)))
 
 
 def version() -> str:

@@ -500,6 +500,20 @@ sla_status forward_checked(const sla_problem* p, const void* q, const void* k, c
 
 // ====================================================================== C ABI
 
+namespace {
+// One thread waits on an mbarrier that nothing arrives on, through the same bounded wait the
+// kernels use, with a caller-chosen limit: the timeout path records SLA_DEVERR_TIMEOUT in the
+// error word and the kernel returns normally, leaving the context usable.
+__global__ void wait_selftest_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  sla::mbar_init(&bar, 1);
+  abort_flag = 0;
+  sla::fence_mbar_init();
+  sla::mbar_wait_for(&bar, 0, err, &abort_flag, limit_ns);
+}
+}  // namespace
+
 extern "C" {
 
 sla_status sla_counts(const sla_problem* p, int* Nq, int* Nk, int* kc, int* kn) {
@@ -605,6 +619,15 @@ sla_status sla_check(void* ws, void* stream) {
   SLA_CUDA(cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice));
   if (word & sla::SLA_DEVERR_TIMEOUT) return fail(SLA_ERR_TIMEOUT, "a device-side wait timed out (error word %u)", word);
   return fail(SLA_ERR_BAD_MASK, "caller mask held a label outside {0,1,2} (error word %u)", word);
+}
+
+sla_status sla_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned limit_us, void* stream) {
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256) return fail(SLA_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (ws_bytes < 256) return fail(SLA_ERR_WORKSPACE, "workspace too small: %zu bytes given, 256 needed", ws_bytes);
+  if (limit_us < 1 || limit_us > 1000000) return fail(SLA_ERR_INVALID_ARG, "limit_us must be in [1, 1000000]");
+  wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(ws),
+                                                                       static_cast<uint64_t>(limit_us) * 1000u);
+  return launched("wait_selftest_kernel");
 }
 
 const char* sla_last_error(void) { return g_last_error.c_str(); }

@@ -70,22 +70,28 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Bounded wait for the phase with the given parity to complete. Returns false
-// (and records a timeout) if it does not complete within SLA_WAIT_LIMIT_NS, or
-// returns false early once *abort_flag becomes nonzero.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
-                                          volatile int* abort_flag) {
+// (and records a timeout) if it does not complete within limit_ns, or returns
+// false early once *abort_flag becomes nonzero.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                              volatile int* abort_flag, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u) {
       if (abort_flag && *abort_flag) return false;
-      if (global_timer_ns() - t0 > SLA_WAIT_LIMIT_NS) break;
+      if (global_timer_ns() - t0 > limit_ns) break;
     }
   }
   record_error(err, SLA_DEVERR_TIMEOUT);
   if (abort_flag) *abort_flag = 1;
   return false;
+}
+
+// The kernels' wait: bounded by SLA_WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          volatile int* abort_flag) {
+  return mbar_wait_for(bar, parity, err, abort_flag, SLA_WAIT_LIMIT_NS);
 }
 
 // Named barrier over `count` threads (a multiple of 32) that also ANDs a predicate:
