@@ -25,13 +25,13 @@ struct AggArgs {
   uint32_t* err;
 };
 
-constexpr int kAggStages = 3;
+constexpr int kAggStages = 4;
 constexpr uint32_t kAggStageBytes = 3 * 16384;  // A for two M-tiles + one B tile (64 x 128)
-constexpr uint32_t kAggStagingBytes = 65536;    // bf16 output tile: 2 M-tiles x 128 rows x 128 columns
+constexpr uint32_t kAggStagingBytes = 32768;    // bf16 output of one M-tile: 128 rows x 128 columns
 
-// Persistent, one CTA per SM, 224 threads: warp 0 TMA producer, warps 1 and 6 tcgen05
-// issuers (one per M-tile), warps 2..5 epilogue (TMEM -> bf16 -> shared-memory staging ->
-// TMA store). A tile is 128 state columns x up to two 128-row M-tiles of query
+// Persistent, one CTA per SM, 224 threads: warp 0 TMA producer (4-stage ring), warps 1
+// and 6 tcgen05 issuers (one per M-tile), warps 2..5 epilogue (TMEM -> bf16 -> one
+// shared-memory staging tile per M-tile in turn -> TMA store). A tile is 128 state columns x up to two 128-row M-tiles of query
 // blocks of one head (so each stacked-state tile is read once per head); tiles are walked
 // columns-fastest. Accumulators are double-buffered in TMEM (2 x 256 columns, M-tile t of
 // buffer b at column 256 b + 128 t) so the epilogue of a tile overlaps the next mainloop.
@@ -157,11 +157,14 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
       decode(t, n0, m0, bh, nm);
       const int ab = tc & 1;
       const bool ok = mbar_wait(&acc_full[ab], (tc >> 1) & 1, a.err, &abort_flag);
-      if (et == 0) tma_store_wait_read();  // the previous tile's store has left the staging tile
       if (!named_barrier_and(1, 128, ok)) break;
       tc_fence_after();
       const bool z_tile = n0 >= D * D;
       for (int tt = 0; tt < nm; ++tt) {
+        if (!z_tile) {  // the staging tile is free once the previous store has read it
+          if (et == 0) tma_store_wait_read();
+          named_barrier(1, 128);
+        }
         const int m = m0 + 128 * tt + rloc;
         uint32_t r[4][32];
 #pragma unroll
@@ -170,7 +173,7 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
         if (!z_tile) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint8_t* box = stg + tt * 32768 + (q >> 1) * 16384;
+            uint8_t* box = stg + (q >> 1) * 16384;
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               *reinterpret_cast<uint4*>(box + sw128_offset(rloc, ((q & 1) * 4 + v) * 16)) =
@@ -188,19 +191,17 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
               dst[8 * q + v] = make_float4(__uint_as_float(r[q][4 * v]), __uint_as_float(r[q][4 * v + 1]),
                                            __uint_as_float(r[q][4 * v + 2]), __uint_as_float(r[q][4 * v + 3]));
         }
+        if (!z_tile) {
+          fence_proxy_async_smem();
+          named_barrier(1, 128);
+          if (et == 0) {
+            for (int b = 0; b < 2; ++b) tma_store_3d(&map_out, stg + b * 16384, n0 + 64 * b, m0 + 128 * tt, bh);
+            tma_store_commit();
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);  // the accumulator has left TMEM
-      if (!z_tile) {
-        fence_proxy_async_smem();
-        named_barrier(1, 128);
-        if (et == 0) {
-          for (int tt = 0; tt < nm; ++tt)
-            for (int b = 0; b < 2; ++b)
-              tma_store_3d(&map_out, stg + tt * 32768 + b * 16384, n0 + 64 * b, m0 + 128 * tt, bh);
-          tma_store_commit();
-        }
-      }
     }
     if (et == 0) tma_store_wait_all();
   }
