@@ -247,3 +247,23 @@ def test_router_resolves_fp32_ties_in_fp64(cuda_device, N, D, bq, kh, kl):
     o_int = binding.forward(qd, kd, vd, alpha, bq, 64, kh, kl)
     o_ext = binding.forward(qd, kd, vd, alpha, bq, 64, kh, kl, mask=torch.from_numpy(rm)[None, None].to(cuda_device))
     assert torch.equal(o_int, o_ext)
+
+
+def test_long_rows_use_the_fp64_selection(cuda_device):
+    """Rows of more than 2048 KV blocks take the fp64 score and selection kernels."""
+    B, H, N, D, bq, kh, kl = 1, 1, 2049 * 64 + 17, 64, 128, 0.02, 0.05
+    q, k, v, alpha = random_inputs(B, H, N, D, seed=2049, device=cuda_device)
+    p = binding.problem(B, H, N, D, bq, 64, kh, kl)
+    Nq, Nk, kc, kn = binding.counts(p)
+    assert Nk > 2048
+    mask, _, _ = _route_parity(q, k, bq, kh, kl)
+    # the fused forward's own router gives the same labels (through the output), and a
+    # sample of query blocks matches the oracle
+    ws = binding.new_workspace(p, cuda_device)
+    out_int = binding.forward(q, k, v, alpha, bq, 64, kh, kl, ws=ws)
+    out_ext = binding.forward(q, k, v, alpha, bq, 64, kh, kl, mask=mask, ws=ws)
+    binding.check(ws)
+    assert torch.equal(out_int, out_ext)
+    qb = [0, 1, Nq // 2, Nq - 1]
+    ref = _oracle_rows(q, k, v, alpha, bq, mask, [(0, 0)], query_blocks=qb)
+    assert_outputs_close(out_ext.float().cpu().numpy(), ref, "long rows")
