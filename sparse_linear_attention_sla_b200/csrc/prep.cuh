@@ -1,10 +1,12 @@
 // Per-block precompute for the SLA forward:
-//   * pool_mean_kernel: mean of the valid query tokens of every query block (fp64)
-//   * kv_prep_kernel:   per KV block j, in one pass over K_j and V_j:
+//   * pool_mean_kernel: mean of the valid tokens of every query (or KV) block, fp64
+//     (the router entry point sla_route);
+//   * prep_kernel:      one persistent pass over the forward's items [KV blocks | query
+//     blocks]; per KV block j, from K_j and V_j:
 //       kbar_j = mean of the valid keys (fp64, router input),
 //       z_j    = colsum phi(K_j)            (linear-attention normaliser state),
 //       h_j    = phi(K_j)^T V_j (D x D)     (linear-attention state, tcgen05 MMA),
-//     with phi(x) = elu(x) + 1.
+//     with phi(x) = elu(x) + 1; per query block i, qbar_i = mean of the valid queries.
 //
 // Sources: "SLA2: Sparse-Linear Attention with Learnable Routing and QAT" §2.B
 // (pooling adjacent Q/K tokens for the router); "SLA: Beyond Sparsity in
