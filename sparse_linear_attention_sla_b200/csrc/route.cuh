@@ -442,16 +442,16 @@ struct CertArgs {
 template <int KPL>
 __device__ __forceinline__ void kth_values(const float (&x)[KPL], int nvalid_lane, const int (&k)[2], float* cand,
                                            float (&T)[2], bool (&ok)[2]) {
+  // Slots past the row end hold NaN: every comparison below is false for them and
+  // fminf/fmaxf ignore them, so no per-slot validity test is needed.
   const int lane = threadIdx.x & 31;
   float mn = INFINITY, mx = -INFINITY;
-  int nv = 0;
+  const int nv = nvalid_lane < 0 ? 0 : (nvalid_lane > KPL ? KPL : nvalid_lane);
 #pragma unroll
-  for (int t = 0; t < KPL; ++t)
-    if (t < nvalid_lane) {
-      mn = fminf(mn, x[t]);
-      mx = fmaxf(mx, x[t]);
-      ++nv;
-    }
+  for (int t = 0; t < KPL; ++t) {
+    mn = fminf(mn, x[t]);
+    mx = fmaxf(mx, x[t]);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -473,9 +473,8 @@ __device__ __forceinline__ void kth_values(const float (&x)[KPL], int nvalid_lan
     uint32_t c0 = 0, c1 = 0;
 #pragma unroll
     for (int t = 0; t < KPL; ++t) {
-      const bool v = t < nvalid_lane;
-      c0 += (v && x[t] > mid[0]) ? 1u : 0u;
-      c1 += (v && -x[t] > mid[1]) ? 1u : 0u;
+      c0 += x[t] > mid[0] ? 1u : 0u;
+      c1 += -x[t] > mid[1] ? 1u : 0u;
     }
     const int cnt[2] = {static_cast<int>(__reduce_add_sync(0xffffffffu, c0)),
                         static_cast<int>(__reduce_add_sync(0xffffffffu, c1))};
@@ -499,7 +498,7 @@ __device__ __forceinline__ void kth_values(const float (&x)[KPL], int nvalid_lan
 #pragma unroll
     for (int s = 0; s < 2; ++s) {
       const float y = s ? -x[t] : x[t];
-      const bool in = m[s] <= 32 && t < nvalid_lane && y >= L[s] && y <= H[s];
+      const bool in = m[s] <= 32 && y >= L[s] && y <= H[s];
       const uint32_t b = __ballot_sync(0xffffffffu, in);
       if (in) cand[32 * s + base[s] + __popc(b & lt_mask)] = y;
       base[s] += __popc(b);
@@ -542,8 +541,7 @@ __device__ __forceinline__ void certify_side(const float (&x)[KPL], int nvalid_l
   sure = 0;
 #pragma unroll
   for (int t = 0; t < KPL; ++t) {
-    if (t >= nvalid_lane) continue;
-    const float y = NEG ? -x[t] : x[t];
+    const float y = NEG ? -x[t] : x[t];  // NaN past the row end: neither certain nor in the band
     if (y > hi) {
       sure |= 1ull << t;
       ++nsure;
@@ -590,7 +588,7 @@ __global__ void __launch_bounds__(256, KPL <= 16 ? 3 : 1) select_cert_kernel(Cer
 #pragma unroll
   for (int t = 0; t < KPL; ++t) {
     const bool v = t < nvalid_lane;
-    x[t] = v ? srow[lane + 32 * t] : 0.f;
+    x[t] = v ? srow[lane + 32 * t] : __uint_as_float(0x7FC00000u);  // NaN marks a slot past the row end
     if (v) nkmax = fmaxf(nkmax, nkrow[lane + 32 * t]);
   }
   double qv[D / 32];
