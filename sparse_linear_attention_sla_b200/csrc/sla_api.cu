@@ -622,7 +622,8 @@ sla_status sla_check(void* ws, void* stream) {
 }
 
 sla_status sla_selftest_wait_timeout(void* ws, size_t ws_bytes, unsigned limit_us, void* stream) {
-  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256) return fail(SLA_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256)
+    return fail(SLA_ERR_WORKSPACE, "workspace must be non-NULL and 256-byte aligned");
   if (ws_bytes < 256) return fail(SLA_ERR_WORKSPACE, "workspace too small: %zu bytes given, 256 needed", ws_bytes);
   if (limit_us < 1 || limit_us > 1000000) return fail(SLA_ERR_INVALID_ARG, "limit_us must be in [1, 1000000]");
   wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t*>(ws),
