@@ -1,0 +1,120 @@
+"""fp64 reference of the low-bit (FP8 e4m3) sparse branch (test infrastructure only).
+
+Source: "SLA2: Sparse-Linear Attention with Learnable Routing and QAT", §2.C: the sparse
+attention branch runs with low-bit (INT8/FP8) operands in the forward pass, the backward
+pass stays in 16-bit. The page names no format details, so this module takes the plainest
+reading that keeps every quantised value exactly reproducible:
+
+* format: e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448,
+  smallest normal 2^-6, subnormals in steps of 2^-9; no infinities), rounding to nearest
+  with ties to even, saturating at +-448;
+* both matmuls of the sparse branch take e4m3 operands: Q K^T and P V;
+* Q is scaled per query block, K and V per KV block, by a power of two
+  s = 2^(ceil(log2(amax)) - 8), so amax / s lies in (128, 256] and the scaling is exact;
+* P = exp(s - m) in (0, 1] is quantised as e4m3(2^8 P) / 2^8;
+* the softmax normaliser l sums the unquantised P (the low-bit operands feed the matmuls,
+  the normalisation stays in full precision); everything else (router, linear branch,
+  blend) is the full-precision path of ``sla_oracle``.
+
+Parity status: the e4m3 rounding is pinned by the format (every finite code is a fixed
+point, halfway cases go to the even code, saturation, subnormal steps); the branch is pinned
+by the exact case (operands already on the scaled e4m3 grid and P exactly representable)
+reducing to the full-precision branch. Other values are the definition above.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Sequence, Tuple
+
+import numpy as np
+
+from .sla_oracle import (CRITICAL, MARGINAL, as_f64, block_counts, compressed_scores, kv_states, linear_branch,
+                         marginal_sums, route_from_scores)
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round to the nearest e4m3 value (ties to the even code), saturating at +-448."""
+    x = np.asarray(x, dtype=np.float64)
+    ax = np.abs(x)
+    _, ex = np.frexp(ax)  # ax = f * 2^ex with f in [0.5, 1): the binade is [2^(ex-1), 2^ex)
+    e = ex.astype(np.float64) - 1.0
+    # quantum: 2^(e-3) for normal values (exponent e >= -6), 2^-9 in the subnormal range
+    quantum = np.exp2(np.maximum(e, -6.0) - 3.0)
+    r = np.round(ax / quantum) * quantum  # np.round rounds halfway cases to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.where(x < 0, -r, r)
+
+
+def pow2_scale(amax: float) -> float:
+    """2^(ceil(log2(amax)) - 8): amax / scale lies in (128, 256]; 1 for amax = 0."""
+    if amax <= 0:
+        return 1.0
+    return math.ldexp(1.0, math.ceil(math.log2(amax)) - 8)
+
+
+def quantize_blocks(x: np.ndarray, block: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-block power-of-two scales and the e4m3 codes (as float64 values) of x [N, D]."""
+    N = x.shape[0]
+    q = np.empty_like(x)
+    scales = []
+    for s in range(0, N, block):
+        e = min(N, s + block)
+        sc = pow2_scale(float(np.abs(x[s:e]).max()))
+        scales.append(sc)
+        q[s:e] = e4m3_round(x[s:e] / sc)
+    return q, np.asarray(scales)
+
+
+def sparse_branch_fp8(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, crit_blocks: Sequence[int],
+                      block_kv: int) -> Tuple[np.ndarray, np.ndarray]:
+    """The sparse branch with e4m3 operands for Q K^T and P V (module docstring).
+
+    Returns (O_s [bq, D], l [bq]); with no critical block both are 0.
+    """
+    N, D = k.shape
+    if len(crit_blocks) == 0:
+        return np.zeros((q_blk.shape[0], D)), np.zeros(q_blk.shape[0])
+    sq = pow2_scale(float(np.abs(q_blk).max()))
+    qh = e4m3_round(q_blk / sq)
+    s_parts, v_parts = [], []
+    for j in crit_blocks:
+        a, e = j * block_kv, min(N, (j + 1) * block_kv)
+        sk = pow2_scale(float(np.abs(k[a:e]).max()))
+        sv = pow2_scale(float(np.abs(v[a:e]).max()))
+        s_parts.append((qh @ e4m3_round(k[a:e] / sk).T) * (sq * sk) / math.sqrt(D))
+        v_parts.append(e4m3_round(v[a:e] / sv) * sv)
+    s = np.concatenate(s_parts, axis=1)
+    vq = np.concatenate(v_parts, axis=0)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1)
+    pq = e4m3_round(p * 256.0) / 256.0
+    return (pq @ vq) / l[:, None], l
+
+
+def forward_fp8(q, k, v, alpha, block_q: int, block_kv: int, kh: float = 0.0, kl: float = 0.0, mask=None):
+    """SLA forward with the low-bit sparse branch; router and linear branch as in ``forward``."""
+    q, k, v, alpha = as_f64(q), as_f64(k), as_f64(v), as_f64(alpha)
+    B, H, N, D = q.shape
+    Nq, Nk, kc, kn = block_counts(N, block_q, block_kv, kh, kl)
+    if mask is None:
+        mask = np.zeros((B, H, Nq, Nk), dtype=np.int8)
+        for b in range(B):
+            for h in range(H):
+                mask[b, h] = route_from_scores(compressed_scores(q[b, h], k[b, h], block_q, block_kv), kc, kn)
+    mask = np.asarray(mask, dtype=np.int8)
+    O = np.empty((B, H, N, D))
+    for b in range(B):
+        for h in range(H):
+            hst, zst = kv_states(k[b, h], v[b, h], block_kv)
+            Hs, Zs = marginal_sums(mask[b, h], hst, zst)
+            for i in range(Nq):
+                s, e = i * block_q, min(N, (i + 1) * block_q)
+                row = mask[b, h, i]
+                os_, _ = sparse_branch_fp8(q[b, h, s:e], k[b, h], v[b, h], np.nonzero(row == CRITICAL)[0], block_kv)
+                ol_, _ = linear_branch(q[b, h, s:e], Hs[i], Zs[i], int(np.count_nonzero(row == MARGINAL)))
+                O[b, h, s:e] = alpha[h] * os_ + (1.0 - alpha[h]) * ol_
+    return O

@@ -1,0 +1,125 @@
+"""Pins of the low-bit sparse-branch reading in oracle/sla_oracle_fp8.py.
+
+The e4m3 rounding is checked against the format itself (every finite code is a fixed
+point, halfway cases go to the even code, saturation, subnormal steps) and against
+torch's own float8_e4m3fn conversion; the branch is checked on inputs where quantisation
+is exact, where it must equal the full-precision branch.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import sla_oracle as so
+from oracle import sla_oracle_fp8 as f8
+
+
+def _e4m3_codes():
+    """Every finite non-negative e4m3 value, from the format definition."""
+    vals = []
+    for E in range(16):
+        for M in range(8):
+            if E == 15 and M == 7:
+                continue  # the NaN code
+            vals.append(M * 2.0 ** -9 if E == 0 else (1 + M / 8) * 2.0 ** (E - 7))
+    return np.array(sorted(set(vals)))
+
+
+def test_codes_are_fixed_points_and_span_the_format():
+    c = _e4m3_codes()
+    assert c[0] == 0.0 and c[1] == 2.0 ** -9 and c[-1] == 448.0 and len(c) == 127
+    np.testing.assert_array_equal(f8.e4m3_round(c), c)
+    np.testing.assert_array_equal(f8.e4m3_round(-c), -c)
+
+
+def test_halfway_cases_round_to_the_even_code():
+    c = _e4m3_codes()
+    mids = (c[:-1] + c[1:]) / 2
+    r = f8.e4m3_round(mids)
+    # the even code of each pair has an even mantissa (or is the power of two above it)
+    lo, hi = c[:-1], c[1:]
+    def even(v):
+        if v == 0:
+            return True
+        if v < 2.0 ** -6:
+            return round(v / 2.0 ** -9) % 2 == 0
+        e = math.floor(math.log2(v))
+        return round(v / 2.0 ** (e - 3)) % 2 == 0
+    expect = np.array([a if even(a) else b for a, b in zip(lo, hi)])
+    np.testing.assert_array_equal(r, expect)
+
+
+def test_saturation_and_monotonicity():
+    np.testing.assert_array_equal(f8.e4m3_round([449.0, 1e9, -500.0]), [448.0, 448.0, -448.0])
+    x = np.linspace(-500, 500, 200001)
+    assert np.all(np.diff(f8.e4m3_round(x)) >= 0)
+
+
+def test_matches_torch_float8_e4m3fn_in_range():
+    g = np.random.default_rng(0)
+    x = np.concatenate([g.normal(0, 30, 20000), g.normal(0, 0.01, 20000), g.uniform(-448, 448, 20000)])
+    ref = torch.from_numpy(x).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    # torch rounds the fp32 value; x is exactly representable in fp32 only after rounding, so
+    # compare on fp32-rounded inputs
+    x32 = x.astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(f8.e4m3_round(x32), ref)
+
+
+def test_nearest_code():
+    g = np.random.default_rng(1)
+    c = _e4m3_codes()
+    allc = np.concatenate([-c[::-1], c])
+    x = g.uniform(-448, 448, 5000)
+    r = f8.e4m3_round(x)
+    d = np.abs(allc[None, :] - x[:, None]).min(axis=1)
+    np.testing.assert_allclose(np.abs(r - x), d, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("amax", [1e-3, 0.37, 1.0, 1.5, 127.9, 128.0, 200.0, 3e4])
+def test_pow2_scale(amax):
+    s = f8.pow2_scale(amax)
+    assert math.frexp(s)[0] == 0.5  # a power of two
+    assert 128.0 < amax / s <= 256.0
+
+
+def test_fp8_branch_equals_exact_branch_when_quantisation_is_exact():
+    g = np.random.default_rng(2)
+    D, bk = 16, 8
+    # values on the e4m3 grid after a power-of-two scale, and Q = 0 so every P is exactly 1
+    k = f8.e4m3_round(g.normal(0, 20, (40, D))) / 64.0
+    v = f8.e4m3_round(g.normal(0, 20, (40, D))) / 64.0
+    q = np.zeros((8, D))
+    crit = [0, 2, 4]
+    o8, l8 = f8.sparse_branch_fp8(q, k, v, crit, bk)
+    o, l = so.sparse_branch(q, k, v, crit, bk)
+    np.testing.assert_allclose(o8, o, rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(l8, l)
+
+
+def test_fp8_forward_close_to_full_precision():
+    g = np.random.default_rng(3)
+    B, H, N, D = 1, 1, 96, 16
+    q, k, v = (g.normal(0, 1, (B, H, N, D)) for _ in range(3))
+    alpha = g.uniform(0, 1, (H, D))
+    o = so.forward(q, k, v, alpha, 16, 8, 0.3, 0.2)
+    o8 = f8.forward_fp8(q, k, v, alpha, 16, 8, 0.3, 0.2)
+    err = np.abs(o8 - o)
+    assert err.max() < 0.1 and err.mean() < 0.02
+    assert not np.array_equal(o8, o)
+
+
+def test_quantize_blocks_scales_and_codes():
+    g = np.random.default_rng(4)
+    x = g.normal(0, 3, (70, 8))
+    codes, scales = f8.quantize_blocks(x, 32)
+    assert len(scales) == 3
+    for bi, s in enumerate(scales):
+        blk = slice(32 * bi, min(70, 32 * (bi + 1)))
+        assert math.frexp(s)[0] == 0.5
+        np.testing.assert_array_equal(f8.e4m3_round(codes[blk]), codes[blk])  # codes are e4m3 values
+        assert np.abs(codes[blk]).max() <= 256.0
+        # relative error of a normal e4m3 code is at most 2^-4
+        big = np.abs(x[blk] / s) >= 2.0 ** -6
+        assert np.all(np.abs(codes[blk][big] * s - x[blk][big]) <= 2.0 ** -4 * np.abs(x[blk][big]))
