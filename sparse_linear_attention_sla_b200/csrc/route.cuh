@@ -369,50 +369,35 @@ __device__ __forceinline__ double exact_score(const double (&qv)[D / 32], const 
 
 // Among the slots flagged in `band` (bit t of each lane = block lane + 32 t), pick `need`
 // in the order (fp64 score descending, index ascending) when best_high, or (fp64 score
-// ascending, index descending) otherwise; returns this lane's picks as a bit mask.
+// ascending, index descending) otherwise; returns this lane's picks as a bit mask. Each
+// pick walks the remaining band and recomputes its fp64 scores with the whole warp, so no
+// per-slot score array is held (the band is a handful of blocks except on degenerate rows).
 template <int KPL, int D>
 __device__ __forceinline__ uint64_t pick_band(uint64_t band, int need, bool best_high, const double (&qv)[D / 32],
                                               const double* kbar_row0) {
   const int lane = threadIdx.x & 31;
-  // fp64 scores of the band, computed by the whole warp one block at a time
-  double sc[KPL];
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) sc[t] = 0.0;
-#pragma unroll
-  for (int t = 0; t < KPL; ++t) {
-    uint32_t who = __ballot_sync(0xffffffffu, (band >> t) & 1ull);
-    while (who) {
-      const int l = __ffs(who) - 1;
-      who &= who - 1;
-      const double v = exact_score<D>(qv, kbar_row0 + static_cast<size_t>(l + 32 * t) * D);
-      if (lane == l) sc[t] = v;
-    }
-  }
   uint64_t picked = 0;
+#pragma unroll 1
   for (int it = 0; it < need; ++it) {
-    double bk = 0.0;
+    double best = 0.0;  // warp-uniform: every lane sees the same reduced scores
     int bj = -1;
-#pragma unroll
+#pragma unroll 1
     for (int t = 0; t < KPL; ++t) {
-      if (!(((band & ~picked) >> t) & 1ull)) continue;
-      const int j = lane + 32 * t;
-      const double v = best_high ? sc[t] : -sc[t];
-      if (bj < 0 || v > bk || (v == bk && (best_high ? j < bj : j > bj))) {
-        bk = v;
-        bj = j;
+      uint32_t who = __ballot_sync(0xffffffffu, ((band & ~picked) >> t) & 1ull);
+      while (who) {
+        const int l = __ffs(who) - 1;
+        who &= who - 1;
+        const int j = l + 32 * t;
+        const double v = exact_score<D>(qv, kbar_row0 + static_cast<size_t>(j) * D);
+        const double w = best_high ? v : -v;
+        if (bj < 0 || w > best || (w == best && (best_high ? j < bj : j > bj))) {
+          best = w;
+          bj = j;
+        }
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ov = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-      const bool take = oj >= 0 && (bj < 0 || ov > bk || (ov == bk && (best_high ? oj < bj : oj > bj)));
-      if (take) {
-        bk = ov;
-        bj = oj;
-      }
-    }
-    if (bj >= 0 && (bj & 31) == lane) picked |= 1ull << (bj >> 5);
+    if (bj < 0) break;
+    if ((bj & 31) == lane) picked |= 1ull << (bj >> 5);
   }
   return picked;
 }
@@ -572,7 +557,7 @@ __device__ __forceinline__ float threshold_from_keys(const float (&x)[KPL], int 
 }
 
 template <int KPL, int D>
-__global__ void __launch_bounds__(256, KPL <= 16 ? 3 : 1) select_cert_kernel(CertArgs a) {
+__global__ void __launch_bounds__(256, KPL <= 16 ? 3 : (KPL <= 40 ? 2 : 1)) select_cert_kernel(CertArgs a) {
   __shared__ float cand_all[8][64];
   grid_dep_launch();
   grid_dep_wait();  // scores come from the previous kernel

@@ -323,6 +323,7 @@ sla_status launch_router(const Shape& s, const Workspace& w, double* scores64, i
     if (s.Nk <= 32 * 8) return launch_cert<8, D>(a, st);
     if (s.Nk <= 32 * 16) return launch_cert<16, D>(a, st);
     if (s.Nk <= 32 * 32) return launch_cert<32, D>(a, st);
+    if (s.Nk <= 32 * 40) return launch_cert<40, D>(a, st);
     return launch_cert<64, D>(a, st);
   }
   double* S = scores64 ? scores64 : w.S;
