@@ -11,15 +11,28 @@ reading that keeps every quantised value exactly reproducible:
 * both matmuls of the sparse branch take e4m3 operands: Q K^T and P V;
 * Q is scaled per query block, K and V per KV block, by a power of two
   s = 2^(ceil(log2(amax)) - 8), so amax / s lies in (128, 256] and the scaling is exact;
-* P = exp(s - m) in (0, 1] is quantised as e4m3(2^8 P) / 2^8;
-* the softmax normaliser l sums the unquantised P (the low-bit operands feed the matmuls,
-  the normalisation stays in full precision); everything else (router, linear branch,
-  blend) is the full-precision path of ``sla_oracle``.
+* P is quantised as a single-pass (online-softmax) kernel produces it. Per query row the
+  critical KV blocks are visited in ascending index order, in log2 units x = s * log2(e).
+  A reference r starts at the first block's row maximum. It moves to a later block's row
+  maximum only when that exceeds r by more than P8_SLACK = 2.5, so every P = 2^(x - r)
+  stays below 2^2.5;
+* the P of a key in block j is quantised in the units of the largest V scale among the
+  row's critical blocks, s_max, at 2^P8_REF_EXP = 2^6 times its value: e4m3(2^6 * P *
+  sv_j / s_max) / 2^6 (sv_j / s_max is a power of two <= 1, applied before rounding; the
+  largest argument, 2^8.5 < 448, never saturates). It multiplies V_j's codes, is carried to
+  the final reference R by 2^(r - R), and the sum is scaled by s_max;
+* the softmax normaliser l = sum over the row's critical keys of 2^(x - R) uses the
+  unquantised P (the low-bit operands feed the matmuls, the normalisation stays in full
+  precision); everything else (router, linear branch, blend) is the full-precision path of
+  ``sla_oracle``.
 
-Parity status: the e4m3 rounding is pinned by the format (every finite code is a fixed
-point, halfway cases go to the even code, saturation, subnormal steps); the branch is pinned
-by the exact case (operands already on the scaled e4m3 grid and P exactly representable)
-reducing to the full-precision branch. Other values are the definition above.
+Parity status: the e4m3 rounding and decoding are pinned by the format (every finite code is
+a fixed point, halfway cases go to the even code, saturation, subnormal steps, torch's own
+float8_e4m3fn); the branch is pinned by the exact case (operands already on the scaled e4m3
+grid and P exactly representable, with V blocks at different scales) reducing to the
+full-precision branch, by the underflow case (a V block 2^18 below the row's largest drops
+out of the numerator but not out of l), and by hand-worked two-block rows on either side of
+the reference's slack. Other values are the definition above.
 """
 
 from __future__ import annotations
@@ -33,6 +46,8 @@ from .sla_oracle import (CRITICAL, MARGINAL, as_f64, block_counts, compressed_sc
                          marginal_sums, route_from_scores)
 
 E4M3_MAX = 448.0
+P8_REF_EXP = 6    # P is quantised at 2^6 times its value
+P8_SLACK = 2.5    # log2 units a block maximum may exceed the reference before it moves
 
 
 def e4m3_round(x) -> np.ndarray:
@@ -46,6 +61,19 @@ def e4m3_round(x) -> np.ndarray:
     r = np.round(ax / quantum) * quantum  # np.round rounds halfway cases to even
     r = np.minimum(r, E4M3_MAX)
     return np.where(x < 0, -r, r)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 byte (uint8 array): sign bit 7, exponent bits 3..6 (bias 7),
+    mantissa bits 0..2; exponent 0 is the subnormal range M * 2^-9. The code with all
+    exponent and mantissa bits set is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    E = (c >> 3) & 0xF
+    M = c & 0x7
+    mag = np.where(E == 0, M * 2.0 ** -9, (1.0 + M / 8.0) * np.exp2(E - 7.0))
+    mag = np.where((E == 15) & (M == 7), np.nan, mag)
+    return sign * mag
 
 
 def pow2_scale(amax: float) -> float:
@@ -68,31 +96,54 @@ def quantize_blocks(x: np.ndarray, block: int) -> Tuple[np.ndarray, np.ndarray]:
     return q, np.asarray(scales)
 
 
+def online_references(x_blocks: Sequence[np.ndarray]) -> list:
+    """Per-row reference (log2 units) in effect while each block is processed.
+
+    x_blocks[b] is [rows, keys of block b] in the order the blocks are visited."""
+    r = x_blocks[0].max(axis=1)
+    refs = [r]
+    for xb in x_blocks[1:]:
+        mb = xb.max(axis=1)
+        r = np.where(mb > r + P8_SLACK, mb, r)
+        refs.append(r)
+    return refs
+
+
 def sparse_branch_fp8(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, crit_blocks: Sequence[int],
                       block_kv: int) -> Tuple[np.ndarray, np.ndarray]:
     """The sparse branch with e4m3 operands for Q K^T and P V (module docstring).
 
-    Returns (O_s [bq, D], l [bq]); with no critical block both are 0.
+    Returns (O_s [bq, D], l [bq]) with l relative to the final reference; with no critical
+    block both are 0.
     """
     N, D = k.shape
     if len(crit_blocks) == 0:
         return np.zeros((q_blk.shape[0], D)), np.zeros(q_blk.shape[0])
+    blocks = sorted(int(j) for j in crit_blocks)
     sq = pow2_scale(float(np.abs(q_blk).max()))
     qh = e4m3_round(q_blk / sq)
-    s_parts, v_parts = [], []
-    for j in crit_blocks:
+    x_blocks, vh_blocks, sv = [], [], []
+    for j in blocks:
         a, e = j * block_kv, min(N, (j + 1) * block_kv)
         sk = pow2_scale(float(np.abs(k[a:e]).max()))
-        sv = pow2_scale(float(np.abs(v[a:e]).max()))
-        s_parts.append((qh @ e4m3_round(k[a:e] / sk).T) * (sq * sk) / math.sqrt(D))
-        v_parts.append(e4m3_round(v[a:e] / sv) * sv)
-    s = np.concatenate(s_parts, axis=1)
-    vq = np.concatenate(v_parts, axis=0)
-    m = s.max(axis=1, keepdims=True)
-    p = np.exp(s - m)
-    l = p.sum(axis=1)
-    pq = e4m3_round(p * 256.0) / 256.0
-    return (pq @ vq) / l[:, None], l
+        s_j = (qh @ e4m3_round(k[a:e] / sk).T) * (sq * sk) / math.sqrt(D)
+        x_blocks.append(s_j * math.log2(math.e))
+        sv_j = pow2_scale(float(np.abs(v[a:e]).max()))
+        vh_blocks.append(e4m3_round(v[a:e] / sv_j))
+        sv.append(sv_j)
+    s_max = max(sv)
+    refs = online_references(x_blocks)
+    R = refs[-1]
+    num = np.zeros((q_blk.shape[0], D))
+    l = np.zeros(q_blk.shape[0])
+    for xb, vh, sv_j, r in zip(x_blocks, vh_blocks, sv, refs):
+        p = np.exp2(xb - r[:, None])
+        ref = 2.0 ** P8_REF_EXP
+        pq = e4m3_round(ref * p * (sv_j / s_max)) / ref
+        carry = np.exp2(r - R)[:, None]
+        num += (pq @ vh) * carry
+        l += (p * carry).sum(axis=1)
+    return num * s_max / l[:, None], l
 
 
 def forward_fp8(q, k, v, alpha, block_q: int, block_kv: int, kh: float = 0.0, kl: float = 0.0, mask=None):

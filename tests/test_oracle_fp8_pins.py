@@ -2,8 +2,9 @@
 
 The e4m3 rounding is checked against the format itself (every finite code is a fixed
 point, halfway cases go to the even code, saturation, subnormal steps) and against
-torch's own float8_e4m3fn conversion; the branch is checked on inputs where quantisation
-is exact, where it must equal the full-precision branch.
+torch's own float8_e4m3fn conversion, and the decoder against every byte; the branch is
+checked on inputs where quantisation is exact, where it must equal the full-precision
+branch, and where one V block's P underflows in the units of the row's largest V scale.
 """
 
 import math
@@ -87,15 +88,86 @@ def test_pow2_scale(amax):
 def test_fp8_branch_equals_exact_branch_when_quantisation_is_exact():
     g = np.random.default_rng(2)
     D, bk = 16, 8
-    # values on the e4m3 grid after a power-of-two scale, and Q = 0 so every P is exactly 1
+    # values on the e4m3 grid after a power-of-two scale, and Q = 0 so every P is exactly 1;
+    # the V blocks sit at different scales (2^0, 2^2, 2^-3), so P is rounded in units of the
+    # largest and must stay exact
     k = f8.e4m3_round(g.normal(0, 20, (40, D))) / 64.0
     v = f8.e4m3_round(g.normal(0, 20, (40, D))) / 64.0
+    v[16:24] *= 4.0
+    v[32:40] /= 8.0
     q = np.zeros((8, D))
     crit = [0, 2, 4]
     o8, l8 = f8.sparse_branch_fp8(q, k, v, crit, bk)
     o, l = so.sparse_branch(q, k, v, crit, bk)
     np.testing.assert_allclose(o8, o, rtol=0, atol=1e-15)
     np.testing.assert_array_equal(l8, l)
+
+
+def test_fp8_branch_rounds_p_after_the_v_scale_ratio():
+    # Q = 0: every P is 1. Block 1's V scale is 2^-18 of block 0's, so its P in block 0's
+    # units, at 2^6, is 2^6 * 2^-18 = 2^-12, below half the smallest e4m3 step: it rounds to 0.
+    # Block 1 then adds nothing to the numerator but its 8 keys still count in l.
+    g = np.random.default_rng(5)
+    D, bk = 16, 8
+    k = g.normal(0, 1, (16, D))
+    v = np.zeros((16, D))
+    v[:8] = f8.e4m3_round(g.normal(0, 20, (8, D))) / 64.0
+    v[8:] = v[:8] * 2.0 ** -18  # the same codes, 18 binades lower
+    assert f8.pow2_scale(np.abs(v[8:]).max()) == f8.pow2_scale(np.abs(v[:8]).max()) * 2.0 ** -18
+    q = np.zeros((4, D))
+    o8, l8 = f8.sparse_branch_fp8(q, k, v, [0, 1], bk)
+    np.testing.assert_array_equal(l8, np.full(4, 16.0))
+    expect = np.broadcast_to(v[:8].sum(axis=0) / 16.0, (4, D))
+    np.testing.assert_allclose(o8, expect, rtol=0, atol=1e-15)
+
+
+def _two_block_row(t):
+    # one query row q = e_0; block 0 keys are 0 (x = 0), block 1 keys are t e_0, so block 1's
+    # x = t / sqrt(16) * log2(e). V: block 0 rows all v0, block 1 rows all v1, same amax.
+    D, bk = 16, 8
+    q = np.zeros((1, D))
+    q[0, 0] = 1.0
+    k = np.zeros((16, D))
+    k[8:, 0] = t
+    v0 = np.array([1.5, 0.5, -1.0, 0.25] * 4)
+    v1 = np.array([-1.5, 1.0, 0.75, -0.125] * 4)
+    v = np.concatenate([np.tile(v0, (8, 1)), np.tile(v1, (8, 1))])
+    o8, _ = f8.sparse_branch_fp8(q, k, v, [0, 1], bk)
+    return o8[0], v0, v1, t / 4.0 * math.log2(math.e)
+
+
+def test_reference_stays_within_the_slack():
+    # t = 6.5: x1 = 2.344 < 2.5, the reference stays at 0, block 1's P = 2^2.344 = 5.077 is
+    # quantised at 2^6: 324.9 lies in [256, 512) where e4m3 steps by 32, so it becomes 320,
+    # i.e. P = 5 exactly; l keeps the unquantised 8 (1 + 2^x1)
+    o, v0, v1, x1 = _two_block_row(6.5)
+    assert x1 < f8.P8_SLACK
+    expect = (v0 + 5.0 * v1) / (1.0 + 2.0 ** x1)
+    np.testing.assert_allclose(o, expect, rtol=0, atol=1e-12)
+
+
+def test_reference_moves_past_the_slack():
+    # t = 7.5: x1 = 2.705 > 2.5, the reference moves to x1, both blocks' P are exactly 1 at
+    # their own reference, and the result is the exact softmax
+    o, v0, v1, x1 = _two_block_row(7.5)
+    assert x1 > f8.P8_SLACK
+    w0 = 2.0 ** -x1
+    np.testing.assert_allclose(o, (w0 * v0 + v1) / (w0 + 1.0), rtol=0, atol=1e-12)
+
+
+def test_decode_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = f8.e4m3_decode(codes)
+    nan = np.isnan(vals)
+    assert list(np.nonzero(nan)[0]) == [0x7F, 0xFF]
+    fin = vals[~nan]
+    # the finite codes are the format's values, each a fixed point of the rounding
+    np.testing.assert_array_equal(np.unique(np.abs(fin)), _e4m3_codes())
+    np.testing.assert_array_equal(f8.e4m3_round(fin), fin)
+    # an independent decoder: torch's float8_e4m3fn reinterpretation of the same bytes
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(vals[~nan], ref[~nan])
+    assert f8.e4m3_decode([0x7E])[0] == 448.0 and f8.e4m3_decode([0x01])[0] == 2.0 ** -9
 
 
 def test_fp8_forward_close_to_full_precision():
