@@ -38,7 +38,7 @@ the reference's slack. Other values are the definition above.
 from __future__ import annotations
 
 import math
-from typing import Sequence, Tuple
+from typing import Iterable, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -48,6 +48,11 @@ from .sla_oracle import (CRITICAL, MARGINAL, as_f64, block_counts, compressed_sc
 E4M3_MAX = 448.0
 P8_REF_EXP = 6    # P is quantised at 2^6 times its value
 P8_SLACK = 2.5    # log2 units a block maximum may exceed the reference before it moves
+# Decisions a float32 kernel may take the other way (see ``sparse_branch_fp8``): a rounding
+# of 2^6 P within this relative distance of the midpoint between two codes, and a reference
+# move within this many log2 units of the slack.
+NEAR_MIDPOINT_REL = 3e-5
+NEAR_SLACK_ABS = 1e-4
 
 
 def e4m3_round(x) -> np.ndarray:
@@ -96,29 +101,48 @@ def quantize_blocks(x: np.ndarray, block: int) -> Tuple[np.ndarray, np.ndarray]:
     return q, np.asarray(scales)
 
 
-def online_references(x_blocks: Sequence[np.ndarray]) -> list:
-    """Per-row reference (log2 units) in effect while each block is processed.
+def online_references(x_blocks: Sequence[np.ndarray]) -> Tuple[list, np.ndarray]:
+    """Per-row reference (log2 units) in effect while each block is processed, and the rows
+    where some block's maximum lies within NEAR_SLACK_ABS of the slack (a move a float32
+    kernel may decide the other way).
 
     x_blocks[b] is [rows, keys of block b] in the order the blocks are visited."""
     r = x_blocks[0].max(axis=1)
     refs = [r]
+    near = np.zeros(r.shape, dtype=bool)
     for xb in x_blocks[1:]:
         mb = xb.max(axis=1)
+        near |= np.abs(mb - (r + P8_SLACK)) <= NEAR_SLACK_ABS
         r = np.where(mb > r + P8_SLACK, mb, r)
         refs.append(r)
-    return refs
+    return refs, near
+
+
+def e4m3_quantum(y) -> np.ndarray:
+    """Spacing of the e4m3 codes around |y| (the binade's step, 2^-9 below 2^-6)."""
+    _, ex = np.frexp(np.abs(np.asarray(y, dtype=np.float64)))
+    return np.exp2(np.maximum(ex.astype(np.float64) - 1.0, -6.0) - 3.0)
 
 
 def sparse_branch_fp8(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, crit_blocks: Sequence[int],
-                      block_kv: int) -> Tuple[np.ndarray, np.ndarray]:
+                      block_kv: int, with_slack: bool = False, x_rel_perturb: float = 0.0):
     """The sparse branch with e4m3 operands for Q K^T and P V (module docstring).
 
     Returns (O_s [bq, D], l [bq]) with l relative to the final reference; with no critical
     block both are 0.
+
+    with_slack=True also returns (slack [bq, D], near_rows [bq]). A kernel computes P in
+    float32, so where 2^6 P (times the V-scale ratio) lies within NEAR_MIDPOINT_REL of the
+    midpoint between two e4m3 codes it may round to the other code; slack bounds, per
+    element, how far O_s moves if every such key takes its other code. near_rows marks the
+    rows whose reference moves are themselves that close (NEAR_SLACK_ABS).
+    x_rel_perturb: the rounding (and only the rounding) sees 2^((x - r)(1 + x_rel_perturb))
+    in place of P, a test hook standing for float32 error in P.
     """
     N, D = k.shape
     if len(crit_blocks) == 0:
-        return np.zeros((q_blk.shape[0], D)), np.zeros(q_blk.shape[0])
+        z = np.zeros((q_blk.shape[0], D)), np.zeros(q_blk.shape[0])
+        return z + (np.zeros((q_blk.shape[0], D)), np.zeros(q_blk.shape[0], dtype=bool)) if with_slack else z
     blocks = sorted(int(j) for j in crit_blocks)
     sq = pow2_scale(float(np.abs(q_blk).max()))
     qh = e4m3_round(q_blk / sq)
@@ -132,40 +156,66 @@ def sparse_branch_fp8(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, crit_bloc
         vh_blocks.append(e4m3_round(v[a:e] / sv_j))
         sv.append(sv_j)
     s_max = max(sv)
-    refs = online_references(x_blocks)
+    refs, near_rows = online_references(x_blocks)
     R = refs[-1]
+    ref = 2.0 ** P8_REF_EXP
     num = np.zeros((q_blk.shape[0], D))
+    slack = np.zeros((q_blk.shape[0], D))
     l = np.zeros(q_blk.shape[0])
     for xb, vh, sv_j, r in zip(x_blocks, vh_blocks, sv, refs):
         p = np.exp2(xb - r[:, None])
-        ref = 2.0 ** P8_REF_EXP
-        pq = e4m3_round(ref * p * (sv_j / s_max)) / ref
+        y = ref * p * (sv_j / s_max)
+        y_seen = y * np.exp2((xb - r[:, None]) * x_rel_perturb) if x_rel_perturb else y
+        pq = e4m3_round(y_seen) / ref
         carry = np.exp2(r - R)[:, None]
         num += (pq @ vh) * carry
         l += (p * carry).sum(axis=1)
-    return num * s_max / l[:, None], l
+        if with_slack:
+            qn = e4m3_quantum(y)
+            t = y / qn
+            near = np.abs(t - np.floor(t) - 0.5) * qn <= NEAR_MIDPOINT_REL * y
+            slack += ((near * qn / ref * carry) @ np.abs(vh))
+    out = num * s_max / l[:, None], l
+    if with_slack:
+        return out + (slack * s_max / l[:, None], near_rows)
+    return out
 
 
-def forward_fp8(q, k, v, alpha, block_q: int, block_kv: int, kh: float = 0.0, kl: float = 0.0, mask=None):
-    """SLA forward with the low-bit sparse branch; router and linear branch as in ``forward``."""
+def forward_fp8(q, k, v, alpha, block_q: int, block_kv: int, kh: float = 0.0, kl: float = 0.0, mask=None,
+                heads: Optional[Iterable[Tuple[int, int]]] = None, query_blocks: Optional[Iterable[int]] = None,
+                with_slack: bool = False):
+    """SLA forward with the low-bit sparse branch; router and linear branch as in ``forward``.
+
+    ``heads`` (list of (b, h)) and ``query_blocks`` (list of i) restrict the work to a
+    sample; rows outside it are NaN in the returned float64 [B,H,N,D] array. With
+    ``with_slack`` the result is (O, slack, near_rows): alpha times the sparse branch's
+    slack [B,H,N,D] and its near rows [B,H,N] (``sparse_branch_fp8``)."""
     q, k, v, alpha = as_f64(q), as_f64(k), as_f64(v), as_f64(alpha)
     B, H, N, D = q.shape
     Nq, Nk, kc, kn = block_counts(N, block_q, block_kv, kh, kl)
+    heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else list(heads)
+    qbs = list(range(Nq)) if query_blocks is None else list(query_blocks)
     if mask is None:
         mask = np.zeros((B, H, Nq, Nk), dtype=np.int8)
-        for b in range(B):
-            for h in range(H):
-                mask[b, h] = route_from_scores(compressed_scores(q[b, h], k[b, h], block_q, block_kv), kc, kn)
+        for b, h in heads:
+            mask[b, h] = route_from_scores(compressed_scores(q[b, h], k[b, h], block_q, block_kv), kc, kn)
     mask = np.asarray(mask, dtype=np.int8)
-    O = np.empty((B, H, N, D))
-    for b in range(B):
-        for h in range(H):
-            hst, zst = kv_states(k[b, h], v[b, h], block_kv)
-            Hs, Zs = marginal_sums(mask[b, h], hst, zst)
-            for i in range(Nq):
-                s, e = i * block_q, min(N, (i + 1) * block_q)
-                row = mask[b, h, i]
-                os_, _ = sparse_branch_fp8(q[b, h, s:e], k[b, h], v[b, h], np.nonzero(row == CRITICAL)[0], block_kv)
-                ol_, _ = linear_branch(q[b, h, s:e], Hs[i], Zs[i], int(np.count_nonzero(row == MARGINAL)))
-                O[b, h, s:e] = alpha[h] * os_ + (1.0 - alpha[h]) * ol_
+    O = np.full((B, H, N, D), np.nan)
+    slack = np.zeros((B, H, N, D))
+    near_rows = np.zeros((B, H, N), dtype=bool)
+    for b, h in heads:
+        hst, zst = kv_states(k[b, h], v[b, h], block_kv)
+        Hs, Zs = marginal_sums(mask[b, h, qbs], hst, zst)
+        for r, i in enumerate(qbs):
+            s, e = i * block_q, min(N, (i + 1) * block_q)
+            row = mask[b, h, i]
+            res = sparse_branch_fp8(q[b, h, s:e], k[b, h], v[b, h], np.nonzero(row == CRITICAL)[0], block_kv,
+                                    with_slack=with_slack)
+            ol_, _ = linear_branch(q[b, h, s:e], Hs[r], Zs[r], int(np.count_nonzero(row == MARGINAL)))
+            O[b, h, s:e] = alpha[h] * res[0] + (1.0 - alpha[h]) * ol_
+            if with_slack:
+                slack[b, h, s:e] = alpha[h] * res[2]
+                near_rows[b, h, s:e] = res[3]
+    if with_slack:
+        return O, slack, near_rows
     return O

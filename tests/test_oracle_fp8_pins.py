@@ -195,3 +195,38 @@ def test_quantize_blocks_scales_and_codes():
         # relative error of a normal e4m3 code is at most 2^-4
         big = np.abs(x[blk] / s) >= 2.0 ** -6
         assert np.all(np.abs(codes[blk][big] * s - x[blk][big]) <= 2.0 ** -4 * np.abs(x[blk][big]))
+
+
+def test_slack_covers_float32_sized_score_errors():
+    # Let the rounding see P with its log2 argument off by a relative 2e-6 (about what float32
+    # scores give): every code that changes must be one the slack counts, so the output moves
+    # by at most the slack.
+    g = np.random.default_rng(6)
+    D, bk = 32, 16
+    q = g.normal(0, 1.0, (256, D))
+    k = g.normal(0, 1.0, (256, D)) * np.repeat(2.0 ** g.integers(-1, 2, 16), 16)[:, None]
+    v0 = g.normal(0, 1.0, (256, D)) * np.repeat(2.0 ** g.integers(-3, 2, 16), 16)[:, None]
+    crit = list(range(0, 16, 2))
+    for vscale in (1.0, 1000.0):  # V scales below and above 1
+        v = v0 * vscale
+        o, _, slack, near = f8.sparse_branch_fp8(q, k, v, crit, bk, with_slack=True)
+        assert slack.max() > 0 and not near.any()
+        moved = 0
+        for d in (2e-6, -2e-6, 1e-6, -1e-6):
+            od, _ = f8.sparse_branch_fp8(q, k, v, crit, bk, x_rel_perturb=d)
+            diff = np.abs(od - o)
+            assert np.all(diff <= slack * (1 + 1e-9) + 1e-13 * vscale)
+            moved += int(np.count_nonzero(diff > 1e-13 * vscale))
+        assert moved > 0  # some code did flip, so the check above was not vacuous
+        # a perturbation a hundred times the window's size flips codes the slack does not count
+        od, _ = f8.sparse_branch_fp8(q, k, v, crit, bk, x_rel_perturb=2e-4)
+        assert np.any(np.abs(od - o) > slack * (1 + 1e-9) + 1e-13 * vscale)
+
+
+def test_slack_is_zero_where_no_code_is_near_a_midpoint():
+    # Q = 0: every 2^6 P is exactly 2^6 times a power of two, a code, far from any midpoint
+    g = np.random.default_rng(7)
+    k = g.normal(0, 1, (32, 16))
+    v = g.normal(0, 1, (32, 16))
+    _, _, slack, near = f8.sparse_branch_fp8(np.zeros((4, 16)), k, v, [0, 1, 3], 8, with_slack=True)
+    assert not slack.any() and not near.any()
