@@ -51,6 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the low-bit (e4m3) sparse-branch measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline sample")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
@@ -423,6 +424,46 @@ def run_ours(args):
                  "speedup_of_sparse_over_dense": round(ms_d / ms_step, 3)}
         del wsd
 
+    # the low-bit sparse branch (SLA2 §2.C) on the same inputs: sla_forward_fp8, L2 flushed,
+    # events on the launching stream; the attention kernel against the e4m3 tensor peak
+    # (twice the measured bf16 peak, the nominal dense fp8 : bf16 ratio)
+    low = None
+    if not args.no_fp8 and w.D == 128:
+        wsf = binding.new_workspace(p, dev, fp8=True)
+        times, stages_f = [], []
+        n_f = min(args.steps, 20)
+        for it in range(3 + n_f):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binding.forward_fp8(q, k, v, alpha, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=wsf)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        for it in range(n_f):
+            flush.zero_()
+            _, st_f = binding.forward_fp8_timed(q, k, v, alpha, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=wsf)
+            stages_f.append(st_f)
+        binding.check(wsf)
+        ms_f = rank_max(sum(times) / len(times))
+        st_f = [sum(x[i] for x in stages_f) / len(stages_f) for i in range(5)]
+        attn_f = rank_max(st_f[4])
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        ach_f = work["f_attn_kernel"] / (attn_f * 1e-3) / 1e12
+        low = {"call": "sla_forward_fp8", "ms_per_call": round(ms_f, 4),
+               "effective_tflops": round(eff_flops / (ms_f * 1e-3) / 1e12, 2),
+               "speedup_over_bf16": round(ms_step / ms_f, 3),
+               "stage_ms": {"precompute": round(st_f[0], 4), "route": round(st_f[1], 4),
+                            "aggregate": round(st_f[2], 4), "quantise_kv": round(st_f[3], 4),
+                            "attention": round(st_f[4], 4)},
+               "roofline": {"bound": "tensor", "kernel": "attn_fp8_kernel", "achieved": round(ach_f, 2),
+                            "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(ach_f / fp8_peak, 4),
+                            "peak_source": "2 x measured bf16 burst (nominal e4m3 : bf16 dense ratio)",
+                            "kernel_ms": round(attn_f, 4)},
+               "timed_calls": n_f}
+        del wsf
+
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         tf, spent, heads, threads = cpu_oracle_sample(w, args.cpu_seconds)
@@ -447,7 +488,7 @@ def run_ours(args):
                      "sum": round(sum(stage_ms), 4), "how": "sla_forward_timed, same steps, after the timed loop"},
         "roofline": roofline, "path_roofline": path_roofline,
         "clocks": clock_info, "e2e": e2e, "gpu_launches": LAUNCHES_PER_FORWARD * args.steps,
-        "dense_reference": dense, "cpu_baseline": cpu,
+        "dense_reference": dense, "low_bit": low, "cpu_baseline": cpu,
         "wall_s_timed": round(wall, 3),
     }
     print(json.dumps(line), flush=True)

@@ -118,6 +118,51 @@ sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k,
                              const float* alpha, const int8_t* mask, void* out, void* ws,
                              size_t ws_bytes, void* stream, float* stage_ms);
 
+/* ---------------------------------------------------------------- low-bit sparse branch
+ *
+ * SLA2 §2.C ("SLA2: Sparse-Linear Attention with Learnable Routing and QAT"): the
+ * sparse branch runs with low-bit operands in the forward pass. The page fixes no
+ * format; the library's reading:
+ *   - e4m3 codes (round to nearest even, saturating at +-448) with one power-of-two
+ *     scale 2^e per block, amax / 2^e in (128, 256] (e = 0 for an all-zero block):
+ *     Q per query block, K and V per KV block; both matmuls of the sparse branch,
+ *     Q K^T and P V, take e4m3 operands with fp32 accumulation;
+ *   - per query row the critical blocks are visited in ascending order against a
+ *     reference maximum r (log2 units) that starts at the first block's row maximum
+ *     and moves to a later block's only when that exceeds r by more than 2.5; the P
+ *     of a key of block j is rounded as e4m3(2^6 * 2^(x - r) * 2^(ev_j - ev_max)),
+ *     ev_max the largest V exponent among the row's critical blocks; the softmax
+ *     normaliser sums the unquantised P;
+ *   - the router, the linear branch and the blend are those of sla_forward.
+ * Supported: D = 128 (else SLA_ERR_UNSUPPORTED), the block sizes of sla_forward. */
+
+/* Workspace bytes for sla_forward_fp8: sla_workspace_size plus the e4m3 codes of K
+ * and V (2 * B*H*N*D bytes) and their block exponents. 0 for an invalid problem. */
+size_t sla_workspace_size_fp8(const sla_problem* p);
+
+/* Fused forward with the low-bit sparse branch. Arguments as for sla_forward; ws
+ * must hold sla_workspace_size_fp8(p) bytes. */
+sla_status sla_forward_fp8(const sla_problem* p, const void* q, const void* k, const void* v,
+                           const float* alpha, const int8_t* mask, void* out, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* sla_forward_fp8 plus per-stage device times, stage_ms[5] (host): [0] precompute,
+ * [1] routing, [2] aggregation, [3] K/V quantiser, [4] fused attention. Synchronises
+ * the stream; meant for measurement. */
+sla_status sla_forward_fp8_timed(const sla_problem* p, const void* q, const void* k, const void* v,
+                                 const float* alpha, const int8_t* mask, void* out, void* ws,
+                                 size_t ws_bytes, void* stream, float* stage_ms);
+
+/* The K/V block quantiser of the low-bit branch on its own.
+ *   k, v                [B,H,N,D] bf16 device, 16-byte aligned
+ *   k8_out, v8_out      [B,H,N,D] uint8 device e4m3 codes (8-byte aligned): sign bit 7,
+ *                       exponent bits 3..6 (bias 7), mantissa bits 0..2; code * 2^exp
+ *                       approximates the input
+ *   kexp_out, vexp_out  [B,H,Nk] int32 device: the exponent of each KV block's scale
+ * D = 64 or 128. Asynchronous on the stream; writes nothing on an argument error. */
+sla_status sla_quantize_kv(const sla_problem* p, const void* k, const void* v, uint8_t* k8_out,
+                           uint8_t* v8_out, int32_t* kexp_out, int32_t* vexp_out, void* stream);
+
 /* Synchronise the stream, read and clear the workspace's device error word.
  * Returns SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_BAD_MASK (or SLA_ERR_CUDA). */
 sla_status sla_check(void* ws, void* stream);

@@ -28,7 +28,8 @@ _STATUS = {
 # Every symbol include/sla.h declares.
 EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sla_forward",
            "sla_forward_timed", "sla_check", "sla_last_error", "sla_version", "sla_route_noalloc",
-           "sla_selftest_wait_timeout")
+           "sla_selftest_wait_timeout", "sla_workspace_size_fp8", "sla_forward_fp8", "sla_forward_fp8_timed",
+           "sla_quantize_kv")
 
 
 class SlaError(RuntimeError):
@@ -69,11 +70,17 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_forward_timed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(ctypes.c_float)]
         lib.sla_check.argtypes = [vp, vp]
+        lib.sla_workspace_size_fp8.argtypes = [P]
+        lib.sla_workspace_size_fp8.restype = sz
+        lib.sla_forward_fp8.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_forward_fp8_timed.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp, ctypes.POINTER(ctypes.c_float)]
+        lib.sla_quantize_kv.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         lib.sla_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint, vp]
         lib.sla_selftest_wait_timeout.restype = ctypes.c_int
         lib.sla_last_error.restype = ctypes.c_char_p
         lib.sla_version.restype = ctypes.c_char_p
-        for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check"):
+        for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check",
+                     "sla_forward_fp8", "sla_forward_fp8_timed", "sla_quantize_kv"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -100,9 +107,14 @@ def workspace_size(p: Problem) -> int:
     return int(load_library().sla_workspace_size(ctypes.byref(p)))
 
 
-def new_workspace(p: Problem, device) -> torch.Tensor:
-    """A zero-headed workspace for problem p on device (bytes, 256-byte aligned by the allocator)."""
-    n = workspace_size(p)
+def workspace_size_fp8(p: Problem) -> int:
+    return int(load_library().sla_workspace_size_fp8(ctypes.byref(p)))
+
+
+def new_workspace(p: Problem, device, fp8: bool = False) -> torch.Tensor:
+    """A zero-headed workspace for problem p on device (bytes, 256-byte aligned by the allocator);
+    fp8=True sizes it for forward_fp8."""
+    n = workspace_size_fp8(p) if fp8 else workspace_size(p)
     if n == 0:
         counts(p)  # raises with the library's message
     ws = torch.empty(n, dtype=torch.uint8, device=device)
@@ -171,7 +183,7 @@ def kv_states(k, v, block_kv=64, ws=None):
     return h, z
 
 
-def _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws):
+def _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws, fp8=False):
     B, H, N, D = q.shape
     dev = q.device
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -189,7 +201,7 @@ def _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws):
     else:
         _check_act("out", out, B, H, N, D, dev)
     if ws is None:
-        ws = new_workspace(p, dev)
+        ws = new_workspace(p, dev, fp8)
     return p, out, ws
 
 
@@ -216,6 +228,51 @@ def forward_timed(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, ma
                                    _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(q.device), ms)
     _raise(st)
     return out, [float(x) for x in ms]
+
+
+def forward_fp8(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, out=None, ws=None):
+    """forward() with the low-bit (e4m3) sparse branch (include/sla.h states the reading); D = 128."""
+    p, out, ws = _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws, fp8=True)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        st = lib.sla_forward_fp8(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(mask), _ptr(out),
+                                 _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(q.device))
+    _raise(st)
+    return out
+
+
+def forward_fp8_timed(q, k, v, alpha, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, out=None, ws=None):
+    """forward_fp8() plus per-stage device milliseconds (precompute, route, aggregate, quantise,
+    attention). Synchronises the current stream."""
+    p, out, ws = _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws, fp8=True)
+    ms = (ctypes.c_float * 5)()
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        st = lib.sla_forward_fp8_timed(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(mask),
+                                       _ptr(out), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(q.device), ms)
+    _raise(st)
+    return out, [float(x) for x in ms]
+
+
+def quantize_kv(k, v, block_kv=64):
+    """e4m3 codes of K and V ([B,H,N,D] uint8) and their per-KV-block scale exponents
+    ([B,H,Nk] int32): code * 2^exp approximates the input."""
+    B, H, N, D = k.shape
+    _check_act("k", k, B, H, N, D, k.device)
+    _check_act("v", v, B, H, N, D, k.device)
+    p = problem(B, H, N, D, 128 if D == 128 else 64, block_kv)
+    _, Nk, _, _ = counts(p)
+    dev = k.device
+    k8 = torch.empty(B, H, N, D, dtype=torch.uint8, device=dev)
+    v8 = torch.empty(B, H, N, D, dtype=torch.uint8, device=dev)
+    kexp = torch.empty(B, H, Nk, dtype=torch.int32, device=dev)
+    vexp = torch.empty(B, H, Nk, dtype=torch.int32, device=dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_quantize_kv(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(k8), _ptr(v8), _ptr(kexp), _ptr(vexp),
+                                 _stream_handle(dev))
+    _raise(st)
+    return k8, v8, kexp, vexp
 
 
 def check(ws: torch.Tensor):

@@ -13,6 +13,8 @@
 #include "../../include/sla.h"
 #include "aggregate.cuh"
 #include "attention.cuh"
+#include "attention_fp8.cuh"
+#include "fp8.cuh"
 #include "prep.cuh"
 #include "route.cuh"
 
@@ -20,6 +22,7 @@ namespace {
 
 using sla::AggArgs;
 using sla::AttnArgs;
+using sla::AttnFp8Args;
 using sla::MaskListArgs;
 using sla::CertArgs;
 using sla::SelectArgs;
@@ -102,12 +105,17 @@ struct Workspace {
   __nv_bfloat16* hst;
   __nv_bfloat16* Hagg;
   float* Zagg;
+  // low-bit sparse branch only
+  uint8_t* k8;     // e4m3 codes of K [BH, N, D]
+  uint8_t* v8;     // e4m3 codes of V [BH, N, D]
+  int32_t* kexp;   // K block scale exponents [BH, Nk]
+  int32_t* vexp;   // V block scale exponents [BH, Nk]
   size_t bytes;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-Workspace layout(const Shape& s, uint8_t* base) {
+Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false) {
   Workspace w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -130,14 +138,20 @@ Workspace layout(const Shape& s, uint8_t* base) {
   w.hst = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(s.LD) * 2));
   w.Hagg = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nq * static_cast<size_t>(s.D) * s.D * 2));
   w.Zagg = reinterpret_cast<float*>(take(BH * s.Nq * s.D * sizeof(float)));
+  if (fp8) {
+    w.k8 = take(BH * s.N * static_cast<size_t>(s.D));
+    w.v8 = take(BH * s.N * static_cast<size_t>(s.D));
+    w.kexp = reinterpret_cast<int32_t*>(take(BH * s.Nk * sizeof(int32_t)));
+    w.vexp = reinterpret_cast<int32_t*>(take(BH * s.Nk * sizeof(int32_t)));
+  }
   w.bytes = off;
   return w;
 }
 
-sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w) {
+sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w, bool fp8 = false) {
   if (!ws) return fail(SLA_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(SLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  *w = layout(s, static_cast<uint8_t*>(ws));
+  *w = layout(s, static_cast<uint8_t*>(ws), fp8);
   if (ws_bytes < w->bytes)
     return fail(SLA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, w->bytes);
   return SLA_OK;
@@ -160,9 +174,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle. dims/strides in elements (innermost first).
+// Tensor map with 128-byte swizzle (bf16, or uint8 for e4m3 codes). dims/strides in
+// elements (innermost first).
 sla_status make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims, const uint64_t* strides_el,
-                    const uint32_t* box) {
+                    const uint32_t* box, bool u8 = false) {
   auto fn = encode_fn();
   if (!fn) return fail(SLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t d[5], st[4];
@@ -172,8 +187,8 @@ sla_status make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* d
     b[r] = box[r];
     es[r] = 1;
   }
-  for (int r = 0; r + 1 < rank; ++r) st[r] = strides_el[r] * 2;
-  CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), d, st, b, es,
+  for (int r = 0; r + 1 < rank; ++r) st[r] = strides_el[r] * (u8 ? 1 : 2);
+  CUresult res = fn(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), d, st, b, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (res != CUDA_SUCCESS) return fail(SLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(res));
@@ -186,6 +201,14 @@ sla_status act_map(CUtensorMap* m, const void* ptr, const Shape& s, uint32_t row
   const uint64_t strides[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.N) * s.D};
   const uint32_t box[3] = {64, rows, 1};
   return make_map(m, ptr, 3, dims, strides, box);
+}
+
+// [BH, N, 128] e4m3-code map with a box of `rows` tokens x 128 channels (128 bytes).
+sla_status code_map(CUtensorMap* m, const void* ptr, const Shape& s, uint32_t rows) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.N), static_cast<uint64_t>(s.BH)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.N) * s.D};
+  const uint32_t box[3] = {128, rows, 1};
+  return make_map(m, ptr, 3, dims, strides, box, true);
 }
 
 // ------------------------------------------------------------------ launch helpers
@@ -414,6 +437,55 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, a);
 }
 
+template <int D>
+sla_status launch_quant(const Shape& s, const void* k, const void* v, uint8_t* k8, uint8_t* v8, int32_t* kexp,
+                        int32_t* vexp, cudaStream_t st, bool dependent) {
+  const dim3 grid(s.Nk, s.BH);
+  auto kb = static_cast<const __nv_bfloat16*>(k);
+  auto vb = static_cast<const __nv_bfloat16*>(v);
+  if (dependent)
+    return launch_dependent(sla::quant_kv_kernel<D>, grid, dim3(256), 0, st, "quant_kv_kernel", kb, vb, k8, v8, kexp,
+                            vexp, s.N, s.Nk);
+  sla::quant_kv_kernel<D><<<grid, 256, 0, st>>>(kb, vb, k8, v8, kexp, vexp, s.N, s.Nk);
+  return launched("quant_kv_kernel");
+}
+
+sla_status launch_attn_fp8(const Shape& s, const void* q, const float* alpha, void* out, const Workspace& w,
+                           int crit_ld, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mh;
+  SLA_TRY(act_map(&mq, q, s, 128));
+  SLA_TRY(code_map(&mk, w.k8, s, 64));
+  SLA_TRY(code_map(&mv, w.v8, s, 64));
+  {
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.BH) * s.Nq * s.D};
+    const uint64_t strides[1] = {static_cast<uint64_t>(s.D)};
+    const uint32_t box[2] = {64, 64};
+    SLA_TRY(make_map(&mh, w.Hagg, 2, dims, strides, box));
+  }
+  constexpr int smem = sla::AttnFp8Smem::total();
+  SLA_TRY(allow_smem(sla::attn_fp8_kernel, smem));
+  AttnFp8Args a;
+  a.H = s.H;
+  a.N = s.N;
+  a.Nq = s.Nq;
+  a.Nk = s.Nk;
+  a.block_q = s.bq;
+  a.n_tiles = s.BH * s.Nq;
+  a.crit = w.crit;
+  a.crit_ld = crit_ld;
+  a.crit_cnt = w.crit_cnt;
+  a.kexp = w.kexp;
+  a.vexp = w.vexp;
+  a.Zagg = w.Zagg;
+  a.alpha = alpha;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(s.D)));
+  a.err = w.err;
+  const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
+  return launch_dependent(sla::attn_fp8_kernel, dim3(grid), dim3(192), smem, st, "attn_fp8_kernel", mq, mk, mv, mh,
+                          a);
+}
+
 // ------------------------------------------------------------------ entry points (templated on D)
 
 template <int D>
@@ -427,8 +499,9 @@ sla_status route_impl(const Shape& s, const void* q, const void* k, int8_t* mask
 
 // Stage boundaries for sla_forward_timed: ev[0] before the per-block precompute,
 // ev[1] after it, ev[2] after routing, ev[3] after aggregation, ev[4] after attention.
+// sla_forward_fp8_timed: ev[4] after the K/V quantiser, ev[5] after attention.
 struct StageEvents {
-  cudaEvent_t ev[5];
+  cudaEvent_t ev[6];
   bool on;
   sla_status mark(int i, cudaStream_t st) {
     if (!on) return SLA_OK;
@@ -440,7 +513,8 @@ struct StageEvents {
 
 template <int D>
 sla_status forward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
-                        const int8_t* mask, void* out, const Workspace& w, cudaStream_t st, StageEvents& ev) {
+                        const int8_t* mask, void* out, const Workspace& w, cudaStream_t st, StageEvents& ev,
+                        bool fp8 = false) {
   sla::PrepArgs pa{};
   pa.BH = s.BH;
   pa.N = s.N;
@@ -467,13 +541,22 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
   SLA_TRY(ev.mark(2, st));
   SLA_TRY(launch_agg<D>(s, w, st));
   SLA_TRY(ev.mark(3, st));
+  if (fp8) {
+    if constexpr (D == 128) {
+      SLA_TRY(launch_quant<D>(s, k, v, w.k8, w.v8, w.kexp, w.vexp, st, true));
+      SLA_TRY(ev.mark(4, st));
+      SLA_TRY(launch_attn_fp8(s, q, alpha, out, w, s.Nk, st));
+      return ev.mark(5, st);
+    }
+    return fail(SLA_ERR_UNSUPPORTED, "the low-bit sparse branch needs D=128");
+  }
   SLA_TRY(launch_attn<D>(s, q, k, v, alpha, out, w, s.Nk, st));
   return ev.mark(4, st);
 }
 
 sla_status forward_checked(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
                            const int8_t* mask, void* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                           StageEvents& ev);
+                           StageEvents& ev, bool fp8 = false);
 
 bool overlaps(const void* a, const void* b, size_t bytes) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
@@ -482,9 +565,10 @@ bool overlaps(const void* a, const void* b, size_t bytes) {
 
 sla_status forward_checked(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
                            const int8_t* mask, void* out, void* ws, size_t ws_bytes, cudaStream_t st,
-                           StageEvents& ev) {
+                           StageEvents& ev, bool fp8) {
   Shape s;
   SLA_TRY(make_shape(p, &s));
+  if (fp8 && s.D != 128) return fail(SLA_ERR_UNSUPPORTED, "the low-bit sparse branch needs D=128 (got %d)", s.D);
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return fail(SLA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
   if (!alpha || reinterpret_cast<uintptr_t>(alpha) % 4) return fail(SLA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
@@ -492,9 +576,34 @@ sla_status forward_checked(const sla_problem* p, const void* q, const void* k, c
   if (overlaps(out, q, act) || overlaps(out, k, act) || overlaps(out, v, act))
     return fail(SLA_ERR_INVALID_ARG, "out must not alias q, k or v");
   Workspace w;
-  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
-  if (s.D == 64) return forward_impl<64>(s, q, k, v, alpha, mask, out, w, st, ev);
-  return forward_impl<128>(s, q, k, v, alpha, mask, out, w, st, ev);
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w, fp8));
+  if (s.D == 64) return forward_impl<64>(s, q, k, v, alpha, mask, out, w, st, ev, fp8);
+  return forward_impl<128>(s, q, k, v, alpha, mask, out, w, st, ev, fp8);
+}
+
+// Shared body of the two timed entry points: `n` stages between n + 1 events.
+sla_status forward_timed_common(const sla_problem* p, const void* q, const void* k, const void* v,
+                                const float* alpha, const int8_t* mask, void* out, void* ws, size_t ws_bytes,
+                                cudaStream_t st, float* stage_ms, bool fp8) {
+  if (!stage_ms) return fail(SLA_ERR_INVALID_ARG, "stage_ms is NULL");
+  const int n = fp8 ? 5 : 4;
+  StageEvents ev{};
+  ev.on = true;
+  for (int i = 0; i <= n; ++i) {
+    cudaError_t e = cudaEventCreate(&ev.ev[i]);
+    if (e != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev.ev[j]);
+      return fail(SLA_ERR_CUDA, "cudaEventCreate: %s", cudaGetErrorString(e));
+    }
+  }
+  sla_status rc = forward_checked(p, q, k, v, alpha, mask, out, ws, ws_bytes, st, ev, fp8);
+  if (rc == SLA_OK) {
+    cudaError_t e = cudaEventSynchronize(ev.ev[n]);
+    for (int i = 0; i < n && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&stage_ms[i], ev.ev[i], ev.ev[i + 1]);
+    if (e != cudaSuccess) rc = fail(SLA_ERR_CUDA, "timing events: %s", cudaGetErrorString(e));
+  }
+  for (int i = 0; i <= n; ++i) cudaEventDestroy(ev.ev[i]);
+  return rc;
 }
 
 }  // namespace
@@ -588,25 +697,43 @@ sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const
 sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
                              const int8_t* mask, void* out, void* ws, size_t ws_bytes, void* stream,
                              float* stage_ms) {
-  if (!stage_ms) return fail(SLA_ERR_INVALID_ARG, "stage_ms is NULL");
+  return forward_timed_common(p, q, k, v, alpha, mask, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                              stage_ms, false);
+}
+
+size_t sla_workspace_size_fp8(const sla_problem* p) {
+  Shape s;
+  if (make_shape(p, &s) != SLA_OK) return 0;
+  return layout(s, nullptr, true).bytes;
+}
+
+sla_status sla_forward_fp8(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                           const int8_t* mask, void* out, void* ws, size_t ws_bytes, void* stream) {
   StageEvents ev{};
-  ev.on = true;
-  for (int i = 0; i < 5; ++i) {
-    cudaError_t e = cudaEventCreate(&ev.ev[i]);
-    if (e != cudaSuccess) {
-      for (int j = 0; j < i; ++j) cudaEventDestroy(ev.ev[j]);
-      return fail(SLA_ERR_CUDA, "cudaEventCreate: %s", cudaGetErrorString(e));
-    }
-  }
+  ev.on = false;
+  return forward_checked(p, q, k, v, alpha, mask, out, ws, ws_bytes, static_cast<cudaStream_t>(stream), ev, true);
+}
+
+sla_status sla_forward_fp8_timed(const sla_problem* p, const void* q, const void* k, const void* v,
+                                 const float* alpha, const int8_t* mask, void* out, void* ws, size_t ws_bytes,
+                                 void* stream, float* stage_ms) {
+  return forward_timed_common(p, q, k, v, alpha, mask, out, ws, ws_bytes, static_cast<cudaStream_t>(stream),
+                              stage_ms, true);
+}
+
+sla_status sla_quantize_kv(const sla_problem* p, const void* k, const void* v, uint8_t* k8_out, uint8_t* v8_out,
+                           int32_t* kexp_out, int32_t* vexp_out, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(k) || !aligned16(v)) return fail(SLA_ERR_INVALID_ARG, "k and v must be non-NULL and 16-byte aligned");
+  if (!k8_out || !v8_out || reinterpret_cast<uintptr_t>(k8_out) % 8 || reinterpret_cast<uintptr_t>(v8_out) % 8)
+    return fail(SLA_ERR_INVALID_ARG, "k8_out and v8_out must be non-NULL and 8-byte aligned");
+  if (!kexp_out || !vexp_out || reinterpret_cast<uintptr_t>(kexp_out) % 4 ||
+      reinterpret_cast<uintptr_t>(vexp_out) % 4)
+    return fail(SLA_ERR_INVALID_ARG, "kexp_out and vexp_out must be non-NULL and 4-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  sla_status rc = forward_checked(p, q, k, v, alpha, mask, out, ws, ws_bytes, st, ev);
-  if (rc == SLA_OK) {
-    cudaError_t e = cudaEventSynchronize(ev.ev[4]);
-    for (int i = 0; i < 4 && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&stage_ms[i], ev.ev[i], ev.ev[i + 1]);
-    if (e != cudaSuccess) rc = fail(SLA_ERR_CUDA, "timing events: %s", cudaGetErrorString(e));
-  }
-  for (int i = 0; i < 5; ++i) cudaEventDestroy(ev.ev[i]);
-  return rc;
+  if (s.D == 64) return launch_quant<64>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st, false);
+  return launch_quant<128>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st, false);
 }
 
 sla_status sla_check(void* ws, void* stream) {

@@ -1,0 +1,157 @@
+"""GPU parity of the low-bit (e4m3) sparse branch against the fp64 oracle of the same reading.
+
+The K/V quantiser must match the oracle bit for bit (every code and every block exponent).
+The fused forward must match the low-bit oracle within the output tolerances of the
+full-precision path, with the oracle's labels passed in, beyond the oracle's rounding slack:
+where 2^6 P lies within a relative 3e-5 of the midpoint between two e4m3 codes the float32
+kernel may take the other code, and the slack bounds what those keys can move (rows whose
+reference move is itself that close are left out and counted). The internal router must
+give the same output whenever its labels equal the oracle's. Inputs are seeded; K and V blocks
+are rescaled by powers of two so that the per-block exponents (and the largest V exponent
+a row's P is rounded against) vary.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import sla_oracle_fp8 as f8
+from sparse_linear_attention_sla_b200 import binding
+from sparse_linear_attention_sla_b200.workloads import WORKLOADS, make_inputs, random_inputs
+from tests.parity_utils import MAX_ABS, MEAN_ABS, output_errors
+
+pytestmark = pytest.mark.gpu
+
+
+def _rescale_blocks(x: torch.Tensor, seed: int, lo: int = -3, hi: int = 2) -> torch.Tensor:
+    """x [B,H,N,D] with every 64-token block multiplied by 2^u, u uniform in [lo, hi]."""
+    B, H, N, D = x.shape
+    Nk = -(-N // 64)
+    g = torch.Generator().manual_seed(seed)
+    u = torch.randint(lo, hi + 1, (B, H, Nk), generator=g).to(torch.float32)
+    f = torch.exp2(u).repeat_interleave(64, dim=-1)[..., :N, None]
+    return (x.float().cpu() * f).to(torch.bfloat16)
+
+
+def _assert_close_beyond_slack(got, ref, slack, near_rows, what):
+    """max / mean of the error beyond the slack over the oracle's rows, near rows left out."""
+    rows = ~np.isnan(ref[..., 0]) & ~near_rows
+    assert np.all(np.isfinite(got[rows])), f"{what}: non-finite GPU output"
+    d = np.abs(got[rows] - ref[rows])
+    excess = np.maximum(d - slack[rows], 0.0)
+    mx, mean = float(excess.max()), float(excess.mean())
+    n_slack = int(np.count_nonzero(slack[rows] > 0))
+    print(f"{what}: beyond-slack max-abs {mx:.3e} mean-abs {mean:.3e}; raw max-abs {d.max():.3e}; "
+          f"{n_slack} elements with slack, {int(near_rows.sum())} near rows left out")
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max-abs {mx:.3e}, mean-abs {mean:.3e} beyond the slack"
+    assert near_rows.sum() <= max(2, rows.size // 1000), f"{what}: {int(near_rows.sum())} near rows"
+    return mx, mean
+
+
+def _oracle_masks(q, k, bq, kh, kl):
+    B, H = q.shape[:2]
+    return np.stack([np.stack([oracle.route(q[b, h].cpu(), k[b, h].cpu(), bq, 64, kh, kl)[0] for h in range(H)])
+                     for b in range(B)])
+
+
+@pytest.mark.parametrize("N, D", [(1000, 128), (333, 64), (64, 128), (4096 + 17, 128)])
+def test_quantize_kv_bit_exact(cuda_device, N, D):
+    B, H = 1, 2
+    g = torch.Generator().manual_seed(N + D)
+    k = torch.randn(B, H, N, D, generator=g)
+    v = 3.0 * torch.randn(B, H, N, D, generator=g)
+    k = _rescale_blocks(k, N, -6, 6)
+    v = _rescale_blocks(v, N + 1, -6, 6)
+    if N >= 128:
+        v[0, 0, 64:128] = 0                       # an all-zero block: exponent 0, codes 0
+        k[0, 1, 64:128] = k[0, 1, 64:128] * 1e-37  # amax near 2^-120: the two-step power-of-two scaling
+    k8, v8, kexp, vexp = binding.quantize_kv(k.to(cuda_device), v.to(cuda_device))
+    for x, codes, exps in ((k, k8, kexp), (v, v8, vexp)):
+        codes, exps = codes.cpu().numpy(), exps.cpu().numpy()
+        for h in range(H):
+            vals, scales = f8.quantize_blocks(x[0, h].double().numpy(), 64)
+            np.testing.assert_array_equal(np.exp2(exps[0, h].astype(np.float64)), scales)
+            np.testing.assert_array_equal(f8.e4m3_decode(codes[0, h]), vals)
+
+
+FP8_CASES = [
+    # B, H, N, bq, kh, kl
+    (1, 2, 1000, 128, 0.25, 0.25),
+    (1, 2, 700, 64, 0.25, 0.25),
+    (2, 1, 333, 128, 0.5, 0.2),
+    (1, 3, 4113, 128, 0.1, 0.2),
+    (1, 2, 1000, 128, 1.0, 0.0),   # every block critical: dense low-bit attention
+    (1, 2, 1000, 128, 0.0, 0.5),   # empty sparse branch: the linear branch alone
+    (1, 2, 1000, 128, 0.5, 0.5),   # empty linear branch
+    (1, 1, 64, 128, 0.5, 0.0),     # a single KV block
+]
+
+
+@pytest.mark.parametrize("case", FP8_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_forward_fp8_matches_oracle(cuda_device, case):
+    B, H, N, bq, kh, kl = case
+    D = 128
+    q, k, v, alpha = random_inputs(B, H, N, D, seed=7 * N + H, device="cpu")
+    # K blocks up and down, V blocks down only: outputs stay O(1), where the tolerances hold
+    # (at |O| ~ 8 half a bf16 ulp of the output alone is 2^-5)
+    k = _rescale_blocks(k, N)
+    v = _rescale_blocks(v, N + 1, -3, 0)
+    q, k, v, alpha = (t.to(cuda_device) for t in (q, k, v, alpha))
+    omask = _oracle_masks(q, k, bq, kh, kl)
+    ws = binding.new_workspace(binding.problem(B, H, N, D, bq, 64, kh, kl), cuda_device, fp8=True)
+    out_m = binding.forward_fp8(q, k, v, alpha, bq, 64, kh, kl, mask=torch.from_numpy(omask).to(cuda_device), ws=ws)
+    out = binding.forward_fp8(q, k, v, alpha, bq, 64, kh, kl, ws=ws)
+    binding.check(ws)
+    qc, kc_, vc, ac = (t.cpu() for t in (q, k, v, alpha))
+    ref, slack, near = f8.forward_fp8(qc, kc_, vc, ac, bq, 64, mask=omask, with_slack=True)
+    got = out_m.float().cpu().numpy()
+    _assert_close_beyond_slack(got, ref, slack, near, f"low-bit, oracle labels {case}")
+    gmask = binding.route(q, k, bq, 64, kh, kl)[0].cpu().numpy()
+    if np.array_equal(gmask, omask):
+        assert torch.equal(out, out_m), "router path and caller-mask path disagree on the same labels"
+    # as accurate against full precision as the low-bit definition itself
+    full = oracle.forward(qc, kc_, vc, ac, bq, 64, mask=omask)
+    got = np.where(near[..., None], np.nan, got)
+    ref = np.where(near[..., None], np.nan, ref)
+    full = np.where(near[..., None], np.nan, full)
+    e_gpu = output_errors(got, full)[1]
+    e_def = output_errors(ref, full)[1]
+    assert e_gpu <= 1.25 * e_def + 1e-3, f"mean-abs vs full precision {e_gpu:.3e}, definition {e_def:.3e}"
+
+
+def _workload_fp8(w, device, heads, query_blocks=None):
+    q, k, v, alpha = make_inputs(w, device="cpu")
+    q, k, v, alpha = (t.to(device) for t in (q, k, v, alpha))
+    B, H = w.B, w.H
+    Nq = -(-w.N // w.block_q)
+    Nk = -(-w.N // 64)
+    om = np.zeros((B, H, Nq, Nk), dtype=np.int8)
+    for b, h in heads:
+        om[b, h] = oracle.route(q[b, h].cpu(), k[b, h].cpu(), w.block_q, 64, w.kh, w.kl)[0]
+    gmask = binding.route(q, k, w.block_q, 64, w.kh, w.kl)[0]
+    mask = gmask.cpu().numpy().copy()
+    for b, h in heads:
+        mask[b, h] = om[b, h]
+    ws = binding.new_workspace(binding.problem(B, H, w.N, w.D, w.block_q, 64, w.kh, w.kl), device, fp8=True)
+    out = binding.forward_fp8(q, k, v, alpha, w.block_q, 64, w.kh, w.kl, mask=torch.from_numpy(mask).to(device),
+                              ws=ws)
+    binding.check(ws)
+    ref, slack, near = f8.forward_fp8(q.cpu(), k.cpu(), v.cpu(), alpha.cpu(), w.block_q, 64, mask=mask, heads=heads,
+                                      query_blocks=query_blocks, with_slack=True)
+    _assert_close_beyond_slack(out.float().cpu().numpy(), ref, slack, near, w.name + " low-bit")
+
+
+def test_fp8_field1d_b1h12_n8192_d128(cuda_device):
+    _workload_fp8(WORKLOADS["field1d_b1h12_n8192_d128"], cuda_device, heads=[(0, 0), (0, 5), (0, 11)])
+
+
+def test_fp8_wan13b_b1h12_n32760_d128_sampled(cuda_device):
+    _workload_fp8(WORKLOADS["wan13b_b1h12_n32760_d128"], cuda_device, heads=[(0, 0), (0, 7)],
+                  query_blocks=[0, 1, 100, 200, 254, 255])
+
+
+def test_fp8_needs_d128(cuda_device):
+    q, k, v, alpha = random_inputs(1, 1, 256, 64, seed=1, device=cuda_device)
+    with pytest.raises(binding.SlaError, match="D=128"):
+        binding.forward_fp8(q, k, v, alpha, 64, 64, 0.25, 0.25)
