@@ -129,8 +129,8 @@ sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k,
  *     Q K^T and P V, take e4m3 operands with fp32 accumulation;
  *   - per query row the critical blocks are visited in ascending order against a
  *     reference maximum r (log2 units) that starts at the first block's row maximum
- *     and moves to a later block's only when that exceeds r by more than 2.5; the P
- *     of a key of block j is rounded as e4m3(2^6 * 2^(x - r) * 2^(ev_j - ev_max)),
+ *     and moves to a later block's only when that exceeds r by more than 8; the P
+ *     of a key of block j is rounded as e4m3(2^(x - r) * 2^(ev_j - ev_max)) (<= 256),
  *     ev_max the largest V exponent among the row's critical blocks; the softmax
  *     normaliser sums the unquantised P;
  *   - the router, the linear branch and the blend are those of sla_forward.

@@ -14,13 +14,14 @@ reading that keeps every quantised value exactly reproducible:
 * P is quantised as a single-pass (online-softmax) kernel produces it. Per query row the
   critical KV blocks are visited in ascending index order, in log2 units x = s * log2(e).
   A reference r starts at the first block's row maximum. It moves to a later block's row
-  maximum only when that exceeds r by more than P8_SLACK = 2.5, so every P = 2^(x - r)
-  stays below 2^2.5;
+  maximum only when that exceeds r by more than P8_SLACK = 8, so every P = 2^(x - r)
+  stays at or below 2^8;
 * the P of a key in block j is quantised in the units of the largest V scale among the
-  row's critical blocks, s_max, at 2^P8_REF_EXP = 2^6 times its value: e4m3(2^6 * P *
-  sv_j / s_max) / 2^6 (sv_j / s_max is a power of two <= 1, applied before rounding; the
-  largest argument, 2^8.5 < 448, never saturates). It multiplies V_j's codes, is carried to
-  the final reference R by 2^(r - R), and the sum is scaled by s_max;
+  row's critical blocks, s_max, at its own value (2^P8_REF_EXP = 2^0): e4m3(P * sv_j /
+  s_max) (sv_j / s_max is a power of two <= 1, applied before rounding; the largest
+  argument, 2^8 = 256 < 448, never saturates, and e4m3's range below it reaches P = 2^-10).
+  It multiplies V_j's codes, is carried to the final reference R by 2^(r - R), and the sum
+  is scaled by s_max;
 * the softmax normaliser l = sum over the row's critical keys of 2^(x - R) uses the
   unquantised P (the low-bit operands feed the matmuls, the normalisation stays in full
   precision); everything else (router, linear branch, blend) is the full-precision path of
@@ -46,10 +47,10 @@ from .sla_oracle import (CRITICAL, MARGINAL, as_f64, block_counts, compressed_sc
                          marginal_sums, route_from_scores)
 
 E4M3_MAX = 448.0
-P8_REF_EXP = 6    # P is quantised at 2^6 times its value
-P8_SLACK = 2.5    # log2 units a block maximum may exceed the reference before it moves
+P8_REF_EXP = 0    # P is quantised at 2^0 times its value
+P8_SLACK = 8.0    # log2 units a block maximum may exceed the reference before it moves
 # Decisions a float32 kernel may take the other way (see ``sparse_branch_fp8``): a rounding
-# of 2^6 P within this relative distance of the midpoint between two codes, and a reference
+# of P within this relative distance of the midpoint between two codes, and a reference
 # move within this many log2 units of the slack.
 NEAR_MIDPOINT_REL = 3e-5
 NEAR_SLACK_ABS = 1e-4
@@ -132,7 +133,7 @@ def sparse_branch_fp8(q_blk: np.ndarray, k: np.ndarray, v: np.ndarray, crit_bloc
     block both are 0.
 
     with_slack=True also returns (slack [bq, D], near_rows [bq]). A kernel computes P in
-    float32, so where 2^6 P (times the V-scale ratio) lies within NEAR_MIDPOINT_REL of the
+    float32, so where P (times the V-scale ratio) lies within NEAR_MIDPOINT_REL of the
     midpoint between two e4m3 codes it may round to the other code; slack bounds, per
     element, how far O_s moves if every such key takes its other code. near_rows marks the
     rows whose reference moves are themselves that close (NEAR_SLACK_ABS).

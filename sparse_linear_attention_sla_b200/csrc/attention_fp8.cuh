@@ -16,10 +16,11 @@
 //   K,V per KV block: codes and exponents come from quant_kv_kernel;
 //   P   per row, against a running reference r (log2 units) that starts at the first
 //       block's row maximum and moves to a later block's maximum only when that exceeds
-//       r by more than kP8Slack; a key of block j contributes e4m3(2^6 * 2^(x - r) *
-//       2^(ev_j - ev_max)) with ev_max the largest V exponent of the tile's critical
-//       blocks; the normaliser l sums the unquantised 2^(x - r).
-//   O_s = 2^(ev_max - 6) * acc / l.
+//       r by more than kP8Slack = 8 (the lazy-rescale threshold of attn_kernel); a key of
+//       block j contributes e4m3(2^(x - r) * 2^(ev_j - ev_max)) <= 256 < 448 with ev_max the
+//       largest V exponent of the tile's critical blocks; the normaliser l sums the
+//       unquantised 2^(x - r).
+//   O_s = 2^ev_max * acc / l.
 //
 // Persistent, two CTAs per SM (<= 100 KB shared memory, 256 TMEM columns each). Warp roles
 // (192 threads):
@@ -38,8 +39,8 @@
 
 namespace sla {
 
-constexpr int kP8RefExp = 6;       // P is quantised at 2^6 times its value
-constexpr float kP8Slack = 2.5f;   // log2 units a block maximum may pass the reference
+constexpr int kP8RefExp = 0;       // P is quantised at 2^0 times its value
+constexpr float kP8Slack = 8.f;    // log2 units a block maximum may pass the reference
 
 struct AttnFp8Args {
   int H, N, Nq, Nk, block_q, n_tiles;
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__(192, 2)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, k & 1, a.err, &abort_flag));
       if (!(ok = named_barrier_and(1, 128, ok))) break;
 
-      // Epilogue: O = alpha * O_s + (1 - alpha) * O_l / den, with O_s = 2^(vmax - 6) acc / l.
+      // Epilogue: O = alpha * O_s + (1 - alpha) * O_l / den, with O_s = 2^(vmax - kP8RefExp) acc / l.
       tc_fence_after();
       const float inv_l = l_run > 0.f ? mul_pow2(1.f / l_run, vmax - kP8RefExp) : 0.f;
       const float inv_d = den_tot > 0.f ? 1.f / den_tot : 0.f;

@@ -3,7 +3,7 @@
 The K/V quantiser must match the oracle bit for bit (every code and every block exponent).
 The fused forward must match the low-bit oracle within the output tolerances of the
 full-precision path, with the oracle's labels passed in, beyond the oracle's rounding slack:
-where 2^6 P lies within a relative 3e-5 of the midpoint between two e4m3 codes the float32
+where P lies within a relative 3e-5 of the midpoint between two e4m3 codes the float32
 kernel may take the other code, and the slack bounds what those keys can move (rows whose
 reference move is itself that close are left out and counted). The internal router must
 give the same output whenever its labels equal the oracle's. Inputs are seeded; K and V blocks

@@ -105,7 +105,7 @@ def test_fp8_branch_equals_exact_branch_when_quantisation_is_exact():
 
 def test_fp8_branch_rounds_p_after_the_v_scale_ratio():
     # Q = 0: every P is 1. Block 1's V scale is 2^-18 of block 0's, so its P in block 0's
-    # units, at 2^6, is 2^6 * 2^-18 = 2^-12, below half the smallest e4m3 step: it rounds to 0.
+    # units is 2^-18, below half the smallest e4m3 step (2^-9): it rounds to 0.
     # Block 1 then adds nothing to the numerator but its 8 keys still count in l.
     g = np.random.default_rng(5)
     D, bk = 16, 8
@@ -137,19 +137,28 @@ def _two_block_row(t):
 
 
 def test_reference_stays_within_the_slack():
-    # t = 6.5: x1 = 2.344 < 2.5, the reference stays at 0, block 1's P = 2^2.344 = 5.077 is
-    # quantised at 2^6: 324.9 lies in [256, 512) where e4m3 steps by 32, so it becomes 320,
-    # i.e. P = 5 exactly; l keeps the unquantised 8 (1 + 2^x1)
+    # t = 6.5: x1 = 2.344 < 8, the reference stays at 0, block 1's P = 2^2.344 = 5.077 lies
+    # in [4, 8) where e4m3 steps by 0.5, so it becomes 5 exactly; l keeps the unquantised
+    # 8 (1 + 2^x1)
     o, v0, v1, x1 = _two_block_row(6.5)
     assert x1 < f8.P8_SLACK
     expect = (v0 + 5.0 * v1) / (1.0 + 2.0 ** x1)
     np.testing.assert_allclose(o, expect, rtol=0, atol=1e-12)
 
 
+def test_reference_stays_for_a_growth_of_four_binades():
+    # t = 12: x1 = 4.328 is inside the slack of 8, so block 1's P = 2^4.328 = 20.09 is rounded
+    # at the old reference: in [16, 32) e4m3 steps by 2, so it becomes 20 (not saturated:
+    # it is rounded at its own value, not scaled up)
+    o, v0, v1, x1 = _two_block_row(12.0)
+    assert 4 < x1 < f8.P8_SLACK
+    np.testing.assert_allclose(o, (v0 + 20.0 * v1) / (1.0 + 2.0 ** x1), rtol=0, atol=1e-12)
+
+
 def test_reference_moves_past_the_slack():
-    # t = 7.5: x1 = 2.705 > 2.5, the reference moves to x1, both blocks' P are exactly 1 at
+    # t = 24: x1 = 8.656 > 8, the reference moves to x1, both blocks' P are exactly 1 at
     # their own reference, and the result is the exact softmax
-    o, v0, v1, x1 = _two_block_row(7.5)
+    o, v0, v1, x1 = _two_block_row(24.0)
     assert x1 > f8.P8_SLACK
     w0 = 2.0 ** -x1
     np.testing.assert_allclose(o, (w0 * v0 + v1) / (w0 + 1.0), rtol=0, atol=1e-12)
@@ -224,7 +233,7 @@ def test_slack_covers_float32_sized_score_errors():
 
 
 def test_slack_is_zero_where_no_code_is_near_a_midpoint():
-    # Q = 0: every 2^6 P is exactly 2^6 times a power of two, a code, far from any midpoint
+    # Q = 0: every P is a power of two, a code, far from any midpoint
     g = np.random.default_rng(7)
     k = g.normal(0, 1, (32, 16))
     v = g.normal(0, 1, (32, 16))
