@@ -123,23 +123,30 @@ def whole_job_tflops(world, flops_per_rank, ms_step):
     return world * flops_per_rank / (ms_step * 1e-3) / 1e12
 
 
-def kernel_source_sha():
+# sources each attention kernel is built from (its recorded traffic is void once one changes)
+KERNEL_SOURCES = {
+    "attn_kernel": ("attention.cuh", "sm100.cuh"),
+    "attn_fp8_kernel": ("attention_fp8.cuh", "fp8.cuh", "attention.cuh", "sm100.cuh"),
+}
+
+
+def kernel_source_sha(kernel="attn_kernel"):
     h = hashlib.sha256()
-    for name in ("attention.cuh", "sm100.cuh"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "sparse_linear_attention_sla_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload):
-    """DRAM bytes per attention-kernel launch from the committed ncu summary, if still current."""
-    path = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+def recorded_traffic(workload, kernel="attn_kernel"):
+    """DRAM bytes per launch of an attention kernel from the committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
-    if t.get("source_sha") != kernel_source_sha() or t.get("workload") != workload:
+    if t.get("source_sha") != kernel_source_sha(kernel) or t.get("workload") != workload:
         return None
     return float(t["dram_bytes_per_launch"])
 
@@ -460,7 +467,8 @@ def run_ours(args):
                "roofline": {"bound": "tensor", "kernel": "attn_fp8_kernel", "achieved": round(ach_f, 2),
                             "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(ach_f / fp8_peak, 4),
                             "peak_source": "2 x measured bf16 burst (nominal e4m3 : bf16 dense ratio)",
-                            "kernel_ms": round(attn_f, 4)},
+                            "kernel_ms": round(attn_f, 4),
+                            "traffic": recorded_traffic(w.name, "attn_fp8_kernel")},
                "timed_calls": n_f}
         del wsf
 
