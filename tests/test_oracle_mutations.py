@@ -124,3 +124,50 @@ def test_mutation_softmax_over_all_keys(monkeypatch):
 
     _patch(monkeypatch, "sparse_branch", all_keys)
     assert _golden_any_fails()
+
+
+# ---------------------------------------------------------------- the low-bit oracle
+
+from oracle import sla_oracle_fp8 as f8  # noqa: E402
+from tests import test_oracle_fp8_pins as pins8  # noqa: E402
+
+
+def test_mutation_fp8_old_slack(monkeypatch):
+    monkeypatch.setattr(f8, "P8_SLACK", 2.5)
+    assert _fails(pins8.test_reference_stays_for_a_growth_of_four_binades)
+
+
+def test_mutation_fp8_p_scaled_up_before_rounding(monkeypatch):
+    monkeypatch.setattr(f8, "P8_REF_EXP", 6)  # 2^6 P saturates at 448 within the slack
+    assert _fails(pins8.test_reference_stays_for_a_growth_of_four_binades)
+
+
+def test_mutation_fp8_reference_moves_on_any_growth(monkeypatch):
+    def eager(x_blocks):
+        r = x_blocks[0].max(axis=1)
+        refs = [r]
+        for xb in x_blocks[1:]:
+            r = np.maximum(r, xb.max(axis=1))
+            refs.append(r)
+        return refs, np.zeros(r.shape, dtype=bool)
+
+    monkeypatch.setattr(f8, "online_references", eager)
+    assert _fails(pins8.test_reference_stays_within_the_slack)
+
+
+def test_mutation_fp8_ties_away_from_zero(monkeypatch):
+    def away(x):
+        x = np.asarray(x, dtype=np.float64)
+        ax = np.abs(x)
+        _, ex = np.frexp(ax)
+        q = np.exp2(np.maximum(ex - 1.0, -6.0) - 3.0)
+        r = np.minimum(np.floor(ax / q + 0.5) * q, f8.E4M3_MAX)
+        return np.where(x < 0, -r, r)
+
+    monkeypatch.setattr(f8, "e4m3_round", away)
+    assert _fails(pins8.test_halfway_cases_round_to_the_even_code)
+
+
+def test_mutation_fp8_slack_window_too_narrow(monkeypatch):
+    monkeypatch.setattr(f8, "NEAR_MIDPOINT_REL", 3e-7)
+    assert _fails(pins8.test_slack_covers_float32_sized_score_errors)
