@@ -93,3 +93,33 @@ def test_entry_points_reject_bad_pointers_before_any_launch(lib):
     assert lib.sla_forward(ctypes.byref(p), fake, fake, fake, fake, null, ctypes.c_void_p(2 << 20),
                            ctypes.c_void_p(8 << 20), small, null) == 3
     assert lib.sla_check(null, null) == 3
+
+
+def test_low_bit_entry_points_host_checks(lib):
+    B, H, N, D = 1, 2, 1000, 128
+    p = binding.problem(B, H, N, D, 128, 64, 0.25, 0.25)
+    _, Nk, _, _ = binding.counts(p)
+    base, full = binding.workspace_size(p), binding.workspace_size_fp8(p)
+    # the low-bit workspace adds the e4m3 codes of K and V and their block exponents
+    extra = full - base
+    assert 2 * B * H * N * D + 2 * B * H * Nk * 4 <= extra <= 2 * B * H * N * D + 2 * B * H * Nk * 4 + 4 * 256
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)
+    out = ctypes.c_void_p(8 << 20)
+    ws = ctypes.c_void_p(16 << 20)
+    # a workspace sized for sla_forward is too small for sla_forward_fp8
+    assert lib.sla_forward_fp8(ctypes.byref(p), fake, fake, fake, fake, null, out, ws, base, null) == 3
+    assert lib.sla_forward_fp8(ctypes.byref(p), null, fake, fake, fake, null, out, ws, full, null) == 1
+    assert lib.sla_forward_fp8_timed(ctypes.byref(p), fake, fake, fake, fake, null, out, ws, full, null, None) == 1
+    # the low-bit branch needs D = 128
+    p64 = binding.problem(1, 1, 256, 64, 64, 64, 0.25, 0.25)
+    assert lib.sla_forward_fp8(ctypes.byref(p64), fake, fake, fake, fake, null, out, ws,
+                               binding.workspace_size_fp8(p64), null) == 2
+    assert "D=128" in lib.sla_last_error().decode()
+    # the quantiser: NULL and misaligned outputs
+    assert lib.sla_quantize_kv(ctypes.byref(p), null, fake, fake, fake, fake, fake, null) == 1
+    assert lib.sla_quantize_kv(ctypes.byref(p), fake, fake, ctypes.c_void_p((1 << 20) + 4), fake, fake, fake,
+                               null) == 1
+    assert lib.sla_quantize_kv(ctypes.byref(p), fake, fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), fake,
+                               null) == 1
+    assert binding.workspace_size_fp8(binding.problem(1, 1, 64, 96, 64, 64, 0.1, 0.1)) == 0
