@@ -171,3 +171,25 @@ def test_mutation_fp8_ties_away_from_zero(monkeypatch):
 def test_mutation_fp8_slack_window_too_narrow(monkeypatch):
     monkeypatch.setattr(f8, "NEAR_MIDPOINT_REL", 3e-7)
     assert _fails(pins8.test_slack_covers_float32_sized_score_errors)
+
+
+# ---------------------------------------------------------------- the backward oracle
+
+from oracle import sla_oracle_bwd as bw  # noqa: E402
+from tests import test_oracle_bwd_pins as pinsb  # noqa: E402
+
+
+def test_mutation_bwd_feature_map_derivative_dropped(monkeypatch):
+    monkeypatch.setattr(bw, "dphi", lambda x: np.ones_like(np.asarray(x, dtype=np.float64)))
+    assert _fails(pinsb.test_matches_central_differences, 0, 8)
+
+
+def test_mutation_bwd_transposed_states(monkeypatch):
+    orig = bw.kv_states
+
+    def transposed(k, v, bk):
+        h, z = orig(k, v, bk)
+        return np.swapaxes(h, -1, -2), z
+
+    monkeypatch.setattr(bw, "kv_states", transposed)
+    assert _fails(pinsb.test_matches_central_differences, 0, 8)
