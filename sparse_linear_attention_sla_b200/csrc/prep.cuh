@@ -162,7 +162,6 @@ __global__ void __launch_bounds__(576, 1)
   constexpr int NS = L::NSLOT;
   constexpr int KBOX = D / 64;  // 64-column boxes per row
   constexpr int CPR = D / 8;    // 16-byte chunks per row
-  constexpr int RG = 128 / CPR; // row groups of the column pass
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage0 = smem + NS * L::SLOT;
@@ -192,7 +191,7 @@ __global__ void __launch_bounds__(576, 1)
     abort_flag = 0;
     fence_mbar_init();
   }
-  if (D == 64) {
+  if constexpr (D == 64) {
     for (uint32_t o = tid * 16; o < L::ZERO; o += 576 * 16) *reinterpret_cast<uint4*>(zero + o) = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
