@@ -193,3 +193,38 @@ def test_mutation_bwd_transposed_states(monkeypatch):
 
     monkeypatch.setattr(bw, "kv_states", transposed)
     assert _fails(pinsb.test_matches_central_differences, 0, 8)
+
+
+# ---------------------------------------------------------------- the PISA oracle
+
+import types  # noqa: E402
+
+from tests import test_oracle_pisa_pins as pinsp  # noqa: E402
+
+
+def _mutated_pisa(old, new):
+    """A copy of oracle.sla_oracle_pisa with one source fragment replaced."""
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "sla_oracle_pisa.py")
+    src = open(path).read()
+    assert src.count(old) == 1, old
+    mod = types.ModuleType("oracle.sla_oracle_pisa_mutant")
+    mod.__package__ = "oracle"
+    exec(compile(src.replace(old, new), path, "exec"), mod.__dict__)
+    return mod
+
+
+FIRST_ORDER = "+ (qb * scale) @ Hbar * A.sum(axis=1, keepdims=True)"
+
+
+@pytest.mark.parametrize("new", ["", "- (qb * scale) @ Hbar * A.sum(axis=1, keepdims=True)",
+                                 "+ qb @ Hbar * A.sum(axis=1, keepdims=True)"],
+                         ids=["dropped", "sign", "unscaled"])
+def test_mutation_pisa_first_order_term(monkeypatch, new):
+    monkeypatch.setattr(pinsp, "pisa", _mutated_pisa(FIRST_ORDER, new))
+    assert _fails(pinsp.test_error_falls_as_the_square_of_the_key_spread)
+
+
+def test_mutation_pisa_denominator_without_block_counts(monkeypatch):
+    monkeypatch.setattr(pinsp, "pisa", _mutated_pisa("den = Pe.sum(axis=1) + A @ n[~crit]",
+                                                     "den = Pe.sum(axis=1) + A.sum(axis=1)"))
+    assert _fails(pinsp.test_blocks_of_equal_keys_make_the_expansion_exact, 1)
