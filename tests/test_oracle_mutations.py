@@ -228,3 +228,24 @@ def test_mutation_pisa_denominator_without_block_counts(monkeypatch):
     monkeypatch.setattr(pinsp, "pisa", _mutated_pisa("den = Pe.sum(axis=1) + A @ n[~crit]",
                                                      "den = Pe.sum(axis=1) + A.sum(axis=1)"))
     assert _fails(pinsp.test_blocks_of_equal_keys_make_the_expansion_exact, 1)
+
+
+# ---------------------------------------------------------------- the second-order block score
+
+from oracle import sla_oracle_route2 as r2  # noqa: E402
+from tests import test_oracle_route2_pins as pinsr  # noqa: E402
+
+
+def test_mutation_route2_quadratic_term_without_the_half(monkeypatch):
+    orig = r2.block_variance
+    monkeypatch.setattr(r2, "block_variance", lambda k, bk: 2.0 * orig(k, bk))
+    assert _fails(pinsr.test_score_matches_the_exact_block_mean_to_fourth_order)
+
+
+def test_mutation_route2_sample_variance(monkeypatch):
+    def sample_var(k, bk):
+        N = k.shape[-2]
+        return np.stack([np.var(k[..., s:min(N, s + bk), :], axis=-2, ddof=1) for s in range(0, N, bk)], axis=-2)
+
+    monkeypatch.setattr(r2, "block_variance", sample_var)
+    assert _fails(pinsr.test_score_matches_the_exact_block_mean_to_fourth_order)
