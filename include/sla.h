@@ -184,11 +184,17 @@ sla_status sla_check(void* ws, void* stream);
  *     than 32 MiB is rejected with SLA_ERR_WORKSPACE before anything is enqueued
  *     (the Wan2.1-1.3B shape B=1, H=12, N=32760, D=128 fits with both outputs NULL).
  *   - The library allocates nothing (no cudaMalloc, cudaFree or allocating library
- *     routine). The first call on each device looks up the array's device address
- *     with that device current; make that first call before any stream capture.
+ *     routine). Every call looks up the array's device address in the calling
+ *     thread's current context (cudaGetSymbolAddress), so the call follows the
+ *     context: after a cudaDeviceReset the next call uses the array of the new
+ *     context. The first call on a device loads the module there; make it before
+ *     any stream capture.
  *   - Every call shares the one array, which keeps the last call's contents. Calls
  *     whose work overlaps on the GPU (other streams, other host threads) race on it
- *     and must be ordered by the caller. */
+ *     and must be ordered by the caller.
+ *   - There is no error word: the router's kernels have no bounded waits and read no
+ *     caller labels, so they raise no device-side error for sla_check to report.
+ *     Launch failures are returned as SLA_ERR_CUDA. */
 sla_status sla_route_noalloc(const sla_problem* p, const void* q, const void* k, int8_t* mask_out,
                              int32_t* crit_idx_out, double* scores_out, void* stream);
 

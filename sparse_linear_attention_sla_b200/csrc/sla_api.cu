@@ -778,26 +778,17 @@ namespace {
 constexpr size_t kRouteScratchBytes = size_t(32) << 20;  // 32 MiB
 __device__ __align__(256) unsigned char g_route_scratch[kRouteScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_route_scratch_mu;
-void* g_route_scratch_addr[kMaxDevices] = {};
-
-// Device address of g_route_scratch on the current device. Looked up once per
-// device (with that device current) on its first use; host code must never
-// pass the array's name itself to a kernel, only this address.
+// Device address of g_route_scratch in the calling thread's current CUDA context.
+// Looked up on every call: the lookup is a host-side table read, and an address
+// cached per device number would go stale when the context it came from is
+// destroyed (cudaDeviceReset) or when the caller runs under another context of the
+// same device. Host code must never pass the array's name itself to a kernel (it
+// is a host-side stand-in there), only this address.
 sla_status route_scratch_address(void** out) {
-  int dev = 0;
-  SLA_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(SLA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  std::lock_guard<std::mutex> lock(g_route_scratch_mu);
-  if (!g_route_scratch_addr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(SLA_ERR_CUDA, "cudaGetSymbolAddress(route scratch): %s", cudaGetErrorString(e));
-    g_route_scratch_addr[dev] = p;
-  }
-  *out = g_route_scratch_addr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+  if (e != cudaSuccess || !p) return fail(SLA_ERR_CUDA, "cudaGetSymbolAddress(route scratch): %s", cudaGetErrorString(e));
+  *out = p;
   return SLA_OK;
 }
 

@@ -123,3 +123,40 @@ def test_low_bit_entry_points_host_checks(lib):
     assert lib.sla_quantize_kv(ctypes.byref(p), fake, fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), fake,
                                null) == 1
     assert binding.workspace_size_fp8(binding.problem(1, 1, 64, 96, 64, 64, 0.1, 0.1)) == 0
+
+
+def _noalloc(lib):
+    fn = lib.sla_route_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(binding.Problem), vp, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    return fn
+
+
+def test_route_noalloc_host_checks(lib):
+    """sla_route_noalloc's argument errors and its size refusal return before any CUDA call."""
+    fn = _noalloc(lib)
+    p = binding.problem(1, 2, 1000, 128, 128, 64, 0.1, 0.2)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced on the host
+    assert fn(ctypes.byref(p), null, fake, fake, null, null, null) == 1           # q NULL
+    assert fn(ctypes.byref(p), fake, ctypes.c_void_p((1 << 20) + 8), fake, null, null, null) == 1  # k misaligned
+    assert fn(ctypes.byref(p), fake, fake, null, null, null, null) == 1           # mask_out NULL
+    assert "mask_out" in lib.sla_last_error().decode()
+    assert fn(ctypes.byref(p), fake, fake, fake, ctypes.c_void_p((1 << 20) + 2), null, null) == 1  # crit misaligned
+    assert fn(ctypes.byref(p), fake, fake, fake, null, ctypes.c_void_p((1 << 20) + 4), null) == 1  # scores misaligned
+    for bad, status in [((1, 1, 64, 96, 64, 64, 0.1, 0.1), 2), ((1, 1, 0, 64, 64, 64, 0.1, 0.1), 1),
+                        ((1, 1, 64, 64, 64, 64, 0.7, 0.4), 1)]:
+        assert fn(ctypes.byref(binding.problem(*bad)), fake, fake, fake, null, null, null) == status
+
+
+def test_route_noalloc_refuses_oversize_problem(lib):
+    fn = _noalloc(lib)
+    # 16 heads of N = 131072 need ~200 MB of scratch without caller outputs: refused on the host.
+    p = binding.problem(1, 16, 131072, 128, 128, 64, 0.05, 0.1)
+    fake = ctypes.c_void_p(1 << 20)
+    null = ctypes.c_void_p(0)
+    assert fn(ctypes.byref(p), fake, fake, fake, null, null, null) == 3
+    assert "maximum" in lib.sla_last_error().decode()
+    # the same problem with both outputs given by the caller still needs more than the array holds
+    assert fn(ctypes.byref(p), fake, fake, fake, fake, ctypes.c_void_p(2 << 20), null) == 3

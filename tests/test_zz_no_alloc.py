@@ -5,7 +5,9 @@ inside a runtime that owns all device memory, a loop with a fixed memory
 budget). sla_route_noalloc keeps its scratch in an array compiled into the
 library instead. These tests call it through the C ABI and check that it gives
 exactly what sla_route (with a caller workspace) gives, on consecutive calls
-that reuse the shared scratch, and that an oversize problem is refused up front.
+that reuse the shared scratch, including rows long enough that the fp64 scores
+are kept in that scratch. The host-side refusals (bad arguments, a problem too
+large for the scratch) are checked without a GPU in test_abi_host.py.
 
 This file is named to be collected last: it passes on its own in a fresh
 process and after the rest of the GPU suite.
@@ -53,7 +55,7 @@ def _call_noalloc(q, k, bq, kh, kl, want_crit, want_scores):
 PROBLEMS = [(1, 3, 4113, 128, 128, 0.1, 0.2), (2, 2, 1000, 64, 64, 0.25, 0.25)]
 
 
-@pytest.mark.parametrize("want_crit, want_scores", [(True, True), (False, False), (True, False)])
+@pytest.mark.parametrize("want_crit, want_scores", [(True, True), (False, False), (True, False), (False, True)])
 def test_noalloc_router_matches_workspace_router(cuda_device, want_crit, want_scores):
     for rep in range(2):  # two calls in a row per problem, alternating problems
         for case in PROBLEMS:
@@ -69,11 +71,17 @@ def test_noalloc_router_matches_workspace_router(cuda_device, want_crit, want_sc
                 np.testing.assert_allclose(scores.cpu().numpy(), ref_scores.cpu().numpy(), rtol=1e-12, atol=0)
 
 
-def test_noalloc_router_refuses_oversize_problem(cuda_device):
-    lib, fn = _noalloc_fn()
-    # 16 heads of N = 131072 need ~200 MB of scratch without caller outputs: refused on the host.
-    p = binding.problem(1, 16, 131072, 128, 128, 64, 0.05, 0.1)
-    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the size check comes first
-    st = fn(ctypes.byref(p), fake, fake, fake, ctypes.c_void_p(0), ctypes.c_void_p(0), ctypes.c_void_p(0))
-    assert st == 3
-    assert "maximum" in lib.sla_last_error().decode()
+@pytest.mark.parametrize("want_crit, want_scores", [(False, False), (True, True)])
+def test_noalloc_router_long_rows(cuda_device, want_crit, want_scores):
+    """Rows of more than 2048 KV blocks: with scores_out NULL the fp64 scores live in the
+    static scratch (about 27 MiB here with the critical lists), else in the caller's buffer."""
+    B, H, N, D, bq, kh, kl = 1, 1, 2050 * 64, 64, 128, 0.03, 0.05
+    q, k, _, _ = random_inputs(B, H, N, D, seed=2050, device=cuda_device)
+    ref_mask, ref_crit, ref_scores = binding.route(q, k, bq, 64, kh, kl, want_scores=True, want_crit=True)
+    for _ in range(2):
+        mask, crit, scores = _call_noalloc(q, k, bq, kh, kl, want_crit, want_scores)
+        assert torch.equal(mask, ref_mask)
+        if want_crit:
+            assert torch.equal(crit, ref_crit)
+        if want_scores:
+            np.testing.assert_allclose(scores.cpu().numpy(), ref_scores.cpu().numpy(), rtol=1e-12, atol=0)
