@@ -52,6 +52,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the low-bit (e4m3) sparse-branch measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration table (the other workloads, the kh sweep and its tail)")
+    ap.add_argument("--config-steps", type=int, default=10, help="timed calls per configuration of that table")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline sample")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
@@ -246,6 +249,69 @@ def cpu_oracle_sample(w, target_s, max_heads=None):
             break
     del torch
     return per_head * done / spent / 1e12, spent, done, threads
+
+
+# ---------------------------------------------------------------- the other configurations
+
+
+def config_table_workloads():
+    """The workloads measured beside the headline one: the 1D-field and Wan2.1-14B 720p
+    shapes, every point of the kh sweep on the Wan2.1-1.3B grid (kh = 100% is the dense
+    reference) and the sweep's ragged N = 32700 case."""
+    from sparse_linear_attention_sla_b200.workloads import SWEEP_KH, WORKLOADS, sweep_workload
+
+    ws = [WORKLOADS["field1d_b1h12_n8192_d128"], WORKLOADS["wan14b720p_b2h40_n75600_d128"]]
+    ws += [sweep_workload(kh) for kh in SWEEP_KH]
+    ws.append(sweep_workload(0.05, N=32700))
+    return ws
+
+
+def measure_config(w, dev, flush, stream, steps, warmup, peaks):
+    """ms per sla_forward call (L2 flushed before each, CUDA events on the launching stream),
+    per-stage times, the whole-path roofline fraction and the attention kernel's fraction."""
+    import torch
+
+    from sparse_linear_attention_sla_b200 import binding
+    from sparse_linear_attention_sla_b200.workloads import make_inputs
+
+    q, k, v, alpha = make_inputs(w, device=dev)
+    p = binding.problem(w.B, w.H, w.N, w.D, w.block_q, w.block_kv, w.kh, w.kl)
+    ws = binding.new_workspace(p, dev)
+    out = torch.empty_like(q)
+    times, stages = [], []
+    for it in range(warmup + steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        binding.forward(q, k, v, alpha, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=ws)
+        e1.record(stream)
+        e1.synchronize()
+        if it >= warmup:
+            times.append(e0.elapsed_time(e1))
+    for _ in range(steps):
+        flush.zero_()
+        _, st = binding.forward_timed(q, k, v, alpha, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=ws)
+        stages.append(st)
+    binding.check(ws)
+    mask, _, _ = binding.route(q, k, w.block_q, w.block_kv, w.kh, w.kl)
+    work = algorithmic_work(w, mask)
+    del mask, q, k, v, out, ws
+    ms = statistics.median(times)
+    st = [statistics.median(x[i] for x in stages) for i in range(4)]
+    t_roof = max(work["flops"] / (peaks["bf16_tflops"] * 1e12), work["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    attn_tf = work["f_attn_kernel"] / (st[3] * 1e-3) / 1e12
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "kh": w.kh, "kl": w.kl,
+            "ms_per_call": round(ms, 4), "ms_p10_p90": [round(float(x), 4) for x in
+                                                       (sorted(times)[len(times) // 10], sorted(times)[-1 - len(times) // 10])],
+            "effective_tflops": round(dense_equivalent_flops(w) / (ms * 1e-3) / 1e12, 2),
+            "executed_tflops": round(work["flops"] / (ms * 1e-3) / 1e12, 2),
+            "stage_ms": {"precompute": round(st[0], 4), "route": round(st[1], 4), "aggregate": round(st[2], 4),
+                         "attention": round(st[3], 4)},
+            "path_roofline": {"t_roof_us": round(t_roof * 1e6, 2), "frac": round(t_roof / (ms * 1e-3), 4),
+                              "bound": "tensor" if work["flops"] / (peaks["bf16_tflops"] * 1e12) >=
+                              work["bytes"] / (peaks["hbm_gbs"] * 1e9) else "hbm"},
+            "attn_kernel": {"achieved_tflops": round(attn_tf, 2), "frac": round(attn_tf / peaks["bf16_tflops"], 4)},
+            "timed_calls": steps}
 
 
 # ---------------------------------------------------------------- our arm
@@ -472,10 +538,19 @@ def run_ours(args):
                "timed_calls": n_f}
         del wsf
 
+    # the other configurations: one table, same timing rules (c3 stays the headline value)
+    configs = None
+    if not args.no_configs:
+        configs = [measure_config(wc, dev, flush, stream, args.config_steps, 3, peaks)
+                   for wc in config_table_workloads()]
+        torch.cuda.empty_cache()
+
     cpu = None
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         tf, spent, heads, threads = cpu_oracle_sample(w, args.cpu_seconds)
         cpu = {"value": round(tf, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "cores_meaning": "threads of numpy's BLAS pool, which runs the oracle's matrix products; "
+                                "its Python loops over blocks run on one of them",
                "sample": f"fp64 oracle on {heads} of {w.B * w.H} heads of {w.name} (all {math.ceil(w.N / w.block_q)} "
                          f"query blocks each: router, states, both branches), {spent:.1f} s"}
 
@@ -496,7 +571,7 @@ def run_ours(args):
                      "sum": round(sum(stage_ms), 4), "how": "sla_forward_timed, same steps, after the timed loop"},
         "roofline": roofline, "path_roofline": path_roofline,
         "clocks": clock_info, "e2e": e2e, "gpu_launches": LAUNCHES_PER_FORWARD * args.steps,
-        "dense_reference": dense, "low_bit": low, "cpu_baseline": cpu,
+        "dense_reference": dense, "low_bit": low, "configs": configs, "cpu_baseline": cpu,
         "wall_s_timed": round(wall, 3),
     }
     print(json.dumps(line), flush=True)
@@ -547,6 +622,8 @@ def run_reference(args):
                    "block_kv": w.block_kv, "kh": w.kh, "kl": w.kl, "inputs": w.kind,
                    "step": "one head, all query blocks"},
         "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "cores_meaning": "threads of numpy's BLAS pool, which runs the oracle's matrix products; "
+                                          "its Python loops over blocks run on one of them",
                          "sample": f"one of {w.B * w.H} heads of {w.name} per step (router, states, both branches)"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

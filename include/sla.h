@@ -127,12 +127,13 @@ sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k,
  *     scale 2^e per block, amax / 2^e in (128, 256] (e = 0 for an all-zero block):
  *     Q per query block, K and V per KV block; both matmuls of the sparse branch,
  *     Q K^T and P V, take e4m3 operands with fp32 accumulation;
- *   - per query row the critical blocks are visited in ascending order against a
- *     reference maximum r (log2 units) that starts at the first block's row maximum
- *     and moves to a later block's only when that exceeds r by more than 8; the P
- *     of a key of block j is rounded as e4m3(2^(x - r) * 2^(ev_j - ev_max)) (<= 256),
- *     ev_max the largest V exponent among the row's critical blocks; the softmax
- *     normaliser sums the unquantised P;
+ *   - P enters P V as e4m3 codes: with x the row's logits in log2 units and m their
+ *     maximum, the P of a key of block j is coded as e4m3(2^(x - r) * 2^(ev_j - u)) for a
+ *     reference r <= m and a unit exponent ev_j <= u <= ev_max (the largest V exponent
+ *     among the row's critical blocks) that saturate no code. The reading leaves r and u
+ *     to the kernel, and every such choice is a valid result: this kernel keeps r at a
+ *     block's row maximum, moved to a later block's only when that exceeds r by more than
+ *     8, and u = ev_max. The softmax normaliser sums the unrounded P;
  *   - the router, the linear branch and the blend are those of sla_forward.
  * Supported: D = 128 (else SLA_ERR_UNSUPPORTED), the block sizes of sla_forward. */
 

@@ -14,11 +14,13 @@
 //       2^eq with amax / 2^eq in (128, 256] and writes the e4m3 tile next to the bf16 one
 //       (which stays for phi(Q) in the linear branch);
 //   K,V per KV block: codes and exponents come from quant_kv_kernel;
-//   P   per row, against a running reference r (log2 units) that starts at the first
-//       block's row maximum and moves to a later block's maximum only when that exceeds
-//       r by more than kP8Slack = 8 (the lazy-rescale threshold of attn_kernel); a key of
-//       block j contributes e4m3(2^(x - r) * 2^(ev_j - ev_max)) <= 256 < 448 with ev_max the
-//       largest V exponent of the tile's critical blocks; the normaliser l sums the
+//   P   coded as e4m3 against a per-row reference r (log2 units). Any r at or below the
+//       row maximum that saturates no code gives a valid result; this kernel starts r at
+//       the first block's row maximum and moves it to a later block's maximum only when
+//       that exceeds r by more than kP8Slack = 8 (so O is rescaled rarely, as in
+//       attn_kernel). r is always some block's maximum, so r <= the row maximum, and a key
+//       of block j contributes e4m3(2^(x - r) * 2^(ev_j - ev_max)) <= 256 < 448 with ev_max
+//       the largest V exponent of the tile's critical blocks; the normaliser l sums the
 //       unquantised 2^(x - r).
 //   O_s = 2^ev_max * acc / l.
 //

@@ -1,14 +1,14 @@
 """GPU parity of the low-bit (e4m3) sparse branch against the fp64 oracle of the same reading.
 
 The K/V quantiser must match the oracle bit for bit (every code and every block exponent).
-The fused forward must match the low-bit oracle within the output tolerances of the
-full-precision path, with the oracle's labels passed in, beyond the oracle's rounding slack:
-where P lies within a relative 3e-5 of the midpoint between two e4m3 codes the float32
-kernel may take the other code, and the slack bounds what those keys can move (rows whose
-reference move is itself that close are left out and counted). The internal router must
-give the same output whenever its labels equal the oracle's. Inputs are seeded; K and V blocks
-are rescaled by powers of two so that the per-block exponents (and the largest V exponent
-a row's P is rounded against) vary.
+The fused forward is checked against the oracle's centre (P unrounded) with the oracle's
+labels passed in: the reading leaves the rounding reference of P to the kernel, and the
+oracle bounds, per output element, how far any admissible rounding can move the result.
+The error beyond that bound must stay within max-abs 2e-2 and mean-abs 2e-3 times the
+output's per-channel magnitude, max(1, max |O*|). The internal router must give the same
+output whenever its labels equal the oracle's. Inputs are seeded; K and V blocks are
+rescaled by powers of two, up and down, so that the per-block exponents (and the largest V
+exponent a row's P is coded against) vary.
 """
 
 import numpy as np
@@ -34,18 +34,23 @@ def _rescale_blocks(x: torch.Tensor, seed: int, lo: int = -3, hi: int = 2) -> to
     return (x.float().cpu() * f).to(torch.bfloat16)
 
 
-def _assert_close_beyond_slack(got, ref, slack, near_rows, what):
-    """max / mean of the error beyond the slack over the oracle's rows, near rows left out."""
-    rows = ~np.isnan(ref[..., 0]) & ~near_rows
-    assert np.all(np.isfinite(got[rows])), f"{what}: non-finite GPU output"
-    d = np.abs(got[rows] - ref[rows])
-    excess = np.maximum(d - slack[rows], 0.0)
+def _assert_within_bound(got, ref, bound, what):
+    """Error beyond the oracle's rounding bound, against the tolerances scaled by the output's
+    per-channel magnitude, over the rows the oracle computed."""
+    rows = ~np.isnan(ref[..., 0])
+    g, r, bd = got[rows], ref[rows], bound[rows]
+    assert np.all(np.isfinite(g)), f"{what}: non-finite GPU output"
+    # per (b, h, channel) magnitude of the output, broadcast back to the rows
+    mag = np.maximum(1.0, np.nanmax(np.abs(ref), axis=-2, keepdims=True))
+    scale = np.broadcast_to(mag, ref.shape)[rows]
+    d = np.abs(g - r)
+    excess = np.maximum(d - bd, 0.0) / scale
     mx, mean = float(excess.max()), float(excess.mean())
-    n_slack = int(np.count_nonzero(slack[rows] > 0))
-    print(f"{what}: beyond-slack max-abs {mx:.3e} mean-abs {mean:.3e}; raw max-abs {d.max():.3e}; "
-          f"{n_slack} elements with slack, {int(near_rows.sum())} near rows left out")
-    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max-abs {mx:.3e}, mean-abs {mean:.3e} beyond the slack"
-    assert near_rows.sum() <= max(2, rows.size // 1000), f"{what}: {int(near_rows.sum())} near rows"
+    used = float(d.mean() / max(bd.mean(), 1e-300))
+    print(f"{what}: beyond-bound max {mx:.3e} mean {mean:.3e} (scaled); raw max-abs {d.max():.3e} "
+          f"mean-abs {d.mean():.3e}; mean bound {bd.mean():.3e} ({used:.3f} of it used on average); "
+          f"largest |O*| {float(mag.max()):.2f}")
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max {mx:.3e}, mean {mean:.3e} beyond the bound"
     return mx, mean
 
 
@@ -93,10 +98,10 @@ def test_forward_fp8_matches_oracle(cuda_device, case):
     B, H, N, bq, kh, kl = case
     D = 128
     q, k, v, alpha = random_inputs(B, H, N, D, seed=7 * N + H, device="cpu")
-    # K blocks up and down, V blocks down only: outputs stay O(1), where the tolerances hold
-    # (at |O| ~ 8 half a bf16 ulp of the output alone is 2^-5)
+    # K and V blocks rescaled up and down (V by 2^-3 .. 2^2): outputs reach |O| ~ 4 - 8, where the
+    # tolerances scale with the output's magnitude
     k = _rescale_blocks(k, N)
-    v = _rescale_blocks(v, N + 1, -3, 0)
+    v = _rescale_blocks(v, N + 1, -3, 2)
     q, k, v, alpha = (t.to(cuda_device) for t in (q, k, v, alpha))
     omask = _oracle_masks(q, k, bq, kh, kl)
     ws = binding.new_workspace(binding.problem(B, H, N, D, bq, 64, kh, kl), cuda_device, fp8=True)
@@ -104,20 +109,19 @@ def test_forward_fp8_matches_oracle(cuda_device, case):
     out = binding.forward_fp8(q, k, v, alpha, bq, 64, kh, kl, ws=ws)
     binding.check(ws)
     qc, kc_, vc, ac = (t.cpu() for t in (q, k, v, alpha))
-    ref, slack, near = f8.forward_fp8(qc, kc_, vc, ac, bq, 64, mask=omask, with_slack=True)
+    ref, bound = f8.forward_fp8(qc, kc_, vc, ac, bq, 64, mask=omask, with_bound=True)
     got = out_m.float().cpu().numpy()
-    _assert_close_beyond_slack(got, ref, slack, near, f"low-bit, oracle labels {case}")
+    _assert_within_bound(got, ref, bound, f"low-bit, oracle labels {case}")
     gmask = binding.route(q, k, bq, 64, kh, kl)[0].cpu().numpy()
     if np.array_equal(gmask, omask):
         assert torch.equal(out, out_m), "router path and caller-mask path disagree on the same labels"
-    # as accurate against full precision as the low-bit definition itself
+    # accuracy against full precision: no worse than the low-bit definition's own (its centre)
+    # by more than the rounding of P the bound allows on average
     full = oracle.forward(qc, kc_, vc, ac, bq, 64, mask=omask)
-    got = np.where(near[..., None], np.nan, got)
-    ref = np.where(near[..., None], np.nan, ref)
-    full = np.where(near[..., None], np.nan, full)
     e_gpu = output_errors(got, full)[1]
     e_def = output_errors(ref, full)[1]
-    assert e_gpu <= 1.25 * e_def + 1e-3, f"mean-abs vs full precision {e_gpu:.3e}, definition {e_def:.3e}"
+    assert e_gpu <= e_def + float(np.nanmean(bound)) + 1e-3, \
+        f"mean-abs vs full precision {e_gpu:.3e}, definition {e_def:.3e}"
 
 
 def _workload_fp8(w, device, heads, query_blocks=None):
@@ -137,9 +141,9 @@ def _workload_fp8(w, device, heads, query_blocks=None):
     out = binding.forward_fp8(q, k, v, alpha, w.block_q, 64, w.kh, w.kl, mask=torch.from_numpy(mask).to(device),
                               ws=ws)
     binding.check(ws)
-    ref, slack, near = f8.forward_fp8(q.cpu(), k.cpu(), v.cpu(), alpha.cpu(), w.block_q, 64, mask=mask, heads=heads,
-                                      query_blocks=query_blocks, with_slack=True)
-    _assert_close_beyond_slack(out.float().cpu().numpy(), ref, slack, near, w.name + " low-bit")
+    ref, bound = f8.forward_fp8(q.cpu(), k.cpu(), v.cpu(), alpha.cpu(), w.block_q, 64, mask=mask, heads=heads,
+                                query_blocks=query_blocks, with_bound=True)
+    _assert_within_bound(out.float().cpu().numpy(), ref, bound, w.name + " low-bit")
 
 
 def test_fp8_field1d_b1h12_n8192_d128(cuda_device):

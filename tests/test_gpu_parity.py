@@ -151,15 +151,26 @@ def test_wan14b720p_sampled(cuda_device):
     _workload_parity(w, cuda_device, heads=heads, query_blocks=qbs, gen_device=cuda_device)
 
 
-@pytest.mark.parametrize("kh", SWEEP_KH)
-def test_sparsity_sweep_sampled(cuda_device, kh):
-    w = sweep_workload(kh)
-    _workload_parity(w, cuda_device, heads=[(0, 0), (0, 11)], query_blocks=[0, 1, 77, 128, 200, 255])
+@pytest.mark.parametrize("kh", [kh for kh in SWEEP_KH if kh < 1.0])
+def test_sparsity_sweep_full(cuda_device, kh):
+    """Every head and every query block of the sweep point, router parity on every head."""
+    _workload_parity(sweep_workload(kh), cuda_device)
+
+
+def test_sparsity_sweep_dense_sampled(cuda_device):
+    """kh = 100% (every block critical: alpha times dense softmax attention): router on every head, outputs
+    on a seeded sample of heads and query blocks (the full fp64 run is ~6.6 TFLOP)."""
+    w = sweep_workload(1.0)
+    rng = np.random.default_rng(100)
+    heads = [(0, 0), (0, 11)] + [(0, int(h)) for h in rng.choice(np.arange(1, 11), size=2, replace=False)]
+    Nq = -(-w.N // w.block_q)
+    qbs = sorted({0, 1, Nq - 1, *[int(x) for x in rng.integers(2, Nq - 1, size=5)]})
+    _workload_parity(w, cuda_device, heads=heads, query_blocks=qbs)
 
 
 def test_sparsity_sweep_tail_n32700(cuda_device):
-    w = sweep_workload(0.05, N=32700)
-    _workload_parity(w, cuda_device, heads=[(0, 3)], query_blocks=[0, 100, 254, 255])
+    """The sweep's ragged case (N = 32700: 60-token last query and KV blocks), in full."""
+    _workload_parity(sweep_workload(0.05, N=32700), cuda_device)
 
 
 def test_output_invariants(cuda_device):

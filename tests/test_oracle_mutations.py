@@ -132,27 +132,68 @@ from oracle import sla_oracle_fp8 as f8  # noqa: E402
 from tests import test_oracle_fp8_pins as pins8  # noqa: E402
 
 
-def test_mutation_fp8_old_slack(monkeypatch):
-    monkeypatch.setattr(f8, "P8_SLACK", 2.5)
-    assert _fails(pins8.test_reference_stays_for_a_growth_of_four_binades)
+def test_mutation_fp8_half_step_too_small(monkeypatch):
+    monkeypatch.setattr(f8, "HALF_STEP_REL", 2.0 ** -5)  # a quarter step: rounding can exceed it
+    assert _fails(pins8.test_a_key_half_a_step_from_a_code_reaches_the_bound)
+    assert _fails(pins8.test_bound_by_hand_normal_terms_dominate)
 
 
-def test_mutation_fp8_p_scaled_up_before_rounding(monkeypatch):
-    monkeypatch.setattr(f8, "P8_REF_EXP", 6)  # 2^6 P saturates at 448 within the slack
-    assert _fails(pins8.test_reference_stays_for_a_growth_of_four_binades)
+def test_mutation_fp8_half_step_too_large(monkeypatch):
+    monkeypatch.setattr(f8, "HALF_STEP_REL", 2.0 ** -3)  # a whole step: no rounding comes near it
+    assert _fails(pins8.test_a_key_half_a_step_from_a_code_reaches_the_bound)
 
 
-def test_mutation_fp8_reference_moves_on_any_growth(monkeypatch):
-    def eager(x_blocks):
-        r = x_blocks[0].max(axis=1)
-        refs = [r]
-        for xb in x_blocks[1:]:
-            r = np.maximum(r, xb.max(axis=1))
-            refs.append(r)
-        return refs, np.zeros(r.shape, dtype=bool)
+def test_mutation_fp8_subnormal_floor_dropped(monkeypatch):
+    monkeypatch.setattr(f8, "HALF_STEP_ABS", 0.0)
+    assert _fails(pins8.test_every_schedule_stays_inside_the_bound, 1.0)
+    assert _fails(pins8.test_subnormal_floor_is_reached_by_a_low_reference)
 
-    monkeypatch.setattr(f8, "online_references", eager)
-    assert _fails(pins8.test_reference_stays_within_the_slack)
+
+def _branch_variant(drop_v_ratio=False, raw_q=False):
+    """A copy of the low-bit branch with one planted mistake."""
+    import math as _m
+
+    def branch(q_blk, k, v, crit_blocks, block_kv):
+        N, D = k.shape
+        bq = q_blk.shape[0]
+        if len(crit_blocks) == 0:
+            return np.zeros((bq, D)), np.zeros(bq), np.zeros((bq, D))
+        sq = f8.pow2_scale(float(np.abs(q_blk).max()))
+        qh = q_blk if raw_q else f8.e4m3_round(q_blk / sq) * sq
+        xs, vs, svs = [], [], []
+        for j in sorted(int(j) for j in crit_blocks):
+            a, e = j * block_kv, min(N, (j + 1) * block_kv)
+            sk = f8.pow2_scale(float(np.abs(k[a:e]).max()))
+            xs.append((qh @ (f8.e4m3_round(k[a:e] / sk) * sk).T) / _m.sqrt(D) * _m.log2(_m.e))
+            sv = f8.pow2_scale(float(np.abs(v[a:e]).max()))
+            vs.append(f8.e4m3_round(v[a:e] / sv) * sv)
+            svs.append(np.full(e - a, sv))
+        x, vh, sv = np.concatenate(xs, axis=1), np.concatenate(vs), np.concatenate(svs)
+        p = np.exp2(x - x.max(axis=1, keepdims=True))
+        l = p.sum(axis=1)
+        ratio = np.ones_like(sv) if drop_v_ratio else sv.max() / sv
+        w = np.maximum(f8.HALF_STEP_REL * p, f8.HALF_STEP_ABS * ratio[None, :])
+        return (p @ vh) / l[:, None], l, (w @ np.abs(vh)) / l[:, None]
+
+    return branch
+
+
+def test_mutation_fp8_variant_harness_is_faithful(monkeypatch):
+    # the unmutated copy passes the pins the mutations below are caught by
+    monkeypatch.setattr(f8, "sparse_branch_fp8", _branch_variant())
+    pins8.test_every_schedule_stays_inside_the_bound(1.0)
+    pins8.test_subnormal_floor_is_reached_by_a_low_reference()
+    pins8.test_centre_is_the_exact_branch_of_the_quantised_operands()
+
+
+def test_mutation_fp8_v_scale_ratio_dropped_from_the_floor(monkeypatch):
+    monkeypatch.setattr(f8, "sparse_branch_fp8", _branch_variant(drop_v_ratio=True))
+    assert _fails(pins8.test_subnormal_floor_is_reached_by_a_low_reference)
+
+
+def test_mutation_fp8_q_left_unquantised(monkeypatch):
+    monkeypatch.setattr(f8, "sparse_branch_fp8", _branch_variant(raw_q=True))
+    assert _fails(pins8.test_centre_is_the_exact_branch_of_the_quantised_operands)
 
 
 def test_mutation_fp8_ties_away_from_zero(monkeypatch):
@@ -166,11 +207,6 @@ def test_mutation_fp8_ties_away_from_zero(monkeypatch):
 
     monkeypatch.setattr(f8, "e4m3_round", away)
     assert _fails(pins8.test_halfway_cases_round_to_the_even_code)
-
-
-def test_mutation_fp8_slack_window_too_narrow(monkeypatch):
-    monkeypatch.setattr(f8, "NEAR_MIDPOINT_REL", 3e-7)
-    assert _fails(pins8.test_slack_covers_float32_sized_score_errors)
 
 
 # ---------------------------------------------------------------- the backward oracle
