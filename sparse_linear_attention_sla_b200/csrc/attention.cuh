@@ -21,11 +21,13 @@
 //   warp 0      TMA producer: per tile Q, then K_j / V_j of every critical block
 //               through a 2-slot ring, then H_i into the next slot (a pseudo-block
 //               of the ring: its two halves complete the slot's K and V barriers).
-//   warp 1      TMEM owner and single-thread tcgen05 issuer:
+//   warp 1      TMEM owner and tcgen05 issuer (the warp runs the loop, one elected lane
+//               issues):
 //               S = Q K_j^T (M=128, N=64), O_s += P V_j (M=128, N=D, P read from
 //               TMEM), O_l = phi(Q) H_i (M=128, N=D).
 //   warps 2..5  softmax / epilogue warpgroup: a thread owns one query row (= TMEM lane)
-//               and all 64 columns of each S block; S_{n+1} is loaded while P_n is stored.
+//               and all 64 columns of each S block; P_n is published before S_{n+1} is
+//               waited for.
 //
 // TMEM columns: S ping-pong [0,64) [64,128) (P, bf16, is written back over the
 // first 32 columns of its S), O_s [128,128+D); after a tile's sparse loop O_l
@@ -180,78 +182,88 @@ __global__ void __launch_bounds__(192, 2)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);
-      const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing);
-      uint32_t nb = 0, ns = 0;  // ring uses, S/P blocks
-      bool ok = true;
-      // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites O_s.
-      auto issue_pv = [&](uint32_t nbm, uint32_t nsm, bool first) -> bool {
-        const int s = nbm & 1, b = nsm & 1;
-        if (!mbar_wait(&p_full[b], (nsm >> 1) & 1, a.err, &abort_flag)) return false;
-        if (!mbar_wait(&v_full[s], (nbm >> 1) & 1, a.err, &abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vb = ring0 + s * L::SLOT + L::KV;
+    // The whole warp runs the loop (waits and descriptors are warp-uniform); one elected
+    // lane issues each tcgen05 operation.
+    const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);
+    const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t q0 = smem_u32(sQ), ring0 = smem_u32(sRing);
+    uint32_t nb = 0, ns = 0;  // ring uses, S/P blocks
+    bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, a.err, &abort_flag));
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) umma_commit(bar);
+      __syncwarp();
+    };
+    // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites O_s.
+    auto issue_pv = [&](uint32_t nbm, uint32_t nsm, bool first) -> bool {
+      const int s = nbm & 1, b = nsm & 1;
+      if (!wait_all(&p_full[b], (nsm >> 1) & 1)) return false;
+      if (!wait_all(&v_full[s], (nbm >> 1) & 1)) return false;
+      tc_fence_after();
+      const uint32_t vb = ring0 + s * L::SLOT + L::KV;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = smem_desc_sw128(vb + kk * 2048, 8192, 1024);
-          umma_bf16_ts(tmem + OS, tmem + b * 64 + kk * 8, bd, id_o, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&pv_done[b]);
-        umma_commit(&v_empty[s]);
-        return true;
-      };
-      int k = 0;
-      for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
-        const int kc = a.crit_cnt[t];
-        if (!(ok = mbar_wait(&q_full, k & 1, a.err, &abort_flag))) break;
-        // the epilogue of the previous tile has read O_s and O_l out of TMEM
-        if (k > 0 && !(ok = mbar_wait(&tmem_free, (k - 1) & 1, a.err, &abort_flag))) break;
-        for (int n = 0; n < kc; ++n, ++nb, ++ns) {
-          const int s = nb & 1, b = ns & 1;
-          if (!(ok = mbar_wait(&k_full[s], (nb >> 1) & 1, a.err, &abort_flag))) break;
-          tc_fence_after();
-          const uint32_t kb = ring0 + s * L::SLOT;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-            umma_bf16_ss(tmem + b * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[b]);
-          umma_commit(&k_empty[s]);
-          if (n >= 1 && !(ok = issue_pv(nb - 1, ns - 1, n == 1))) break;
-        }
-        if (!ok) break;
-        if (kc > 0 && !(ok = issue_pv(nb - 1, ns - 1, kc == 1))) break;
-        // linear branch: O_l = phi(Q) H_i once H_i has landed and the warpgroups rewrote Q as phi(Q)
-        const int s = nb & 1;
-        if (!(ok = mbar_wait(&k_full[s], (nb >> 1) & 1, a.err, &abort_flag))) break;
-        if (!(ok = mbar_wait(&v_full[s], (nb >> 1) & 1, a.err, &abort_flag))) break;
-        if (!(ok = mbar_wait(&phiq_full, k & 1, a.err, &abort_flag))) break;
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = smem_desc_sw128(vb + kk * 2048, 8192, 1024);
+        if (elect_one()) umma_bf16_ts(tmem + OS, tmem + b * 64 + kk * 8, bd, id_o, (first && kk == 0) ? 0u : 1u);
+        __syncwarp();
+      }
+      commit(&pv_done[b]);
+      commit(&v_empty[s]);
+      return true;
+    };
+    int k = 0;
+    for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
+      const int kc = a.crit_cnt[t];
+      if (!(ok = wait_all(&q_full, k & 1))) break;
+      // the epilogue of the previous tile has read O_s and O_l out of TMEM
+      if (k > 0 && !(ok = wait_all(&tmem_free, (k - 1) & 1))) break;
+      for (int n = 0; n < kc; ++n, ++nb, ++ns) {
+        const int s = nb & 1, b = ns & 1;
+        if (!(ok = wait_all(&k_full[s], (nb >> 1) & 1))) break;
         tc_fence_after();
-        const uint32_t hb = ring0 + s * L::SLOT;
+        const uint32_t kb = ring0 + s * L::SLOT;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(hb + (kk >> 2) * DB * 8192 + (kk & 3) * 2048, 8192, 1024);
-          umma_bf16_ss(tmem + OL, ad, bd, id_o, kk > 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+          if (elect_one()) umma_bf16_ss(tmem + b * 64, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          __syncwarp();
         }
-        umma_commit(&ol_done);
-        umma_commit(&q_free);
-        umma_commit(&k_empty[s]);
-        umma_commit(&v_empty[s]);
-        ++nb;
+        commit(&s_full[b]);
+        commit(&k_empty[s]);
+        if (n >= 1 && !(ok = issue_pv(nb - 1, ns - 1, n == 1))) break;
       }
-      umma_commit(&drain);  // every MMA issued above has finished once this arrives
-      mbar_wait(&drain, 0, nullptr, nullptr);
+      if (!ok) break;
+      if (kc > 0 && !(ok = issue_pv(nb - 1, ns - 1, kc == 1))) break;
+      // linear branch: O_l = phi(Q) H_i once H_i has landed and the warpgroup rewrote Q as phi(Q)
+      const int s = nb & 1;
+      if (!(ok = wait_all(&k_full[s], (nb >> 1) & 1))) break;
+      if (!(ok = wait_all(&v_full[s], (nb >> 1) & 1))) break;
+      if (!(ok = wait_all(&phiq_full, k & 1))) break;
+      tc_fence_after();
+      const uint32_t hb = ring0 + s * L::SLOT;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = smem_desc_sw128(hb + (kk >> 2) * DB * 8192 + (kk & 3) * 2048, 8192, 1024);
+        if (elect_one()) umma_bf16_ss(tmem + OL, ad, bd, id_o, kk > 0 ? 1u : 0u);
+        __syncwarp();
+      }
+      commit(&ol_done);
+      commit(&q_free);
+      commit(&k_empty[s]);
+      commit(&v_empty[s]);
+      ++nb;
     }
-    __syncwarp();
+    commit(&drain);  // every MMA issued above has finished once this arrives
+    mbar_wait(&drain, 0, nullptr, nullptr);
   } else {
     // ------------------------------------------------------------ softmax / epilogue warpgroup
-    // Thread = query row r = TMEM lane; it owns all 64 columns of every S block. The load of
-    // S_{n+1} is issued before P_n is published, so its latency overlaps the store of P_n.
+    // Thread = query row r = TMEM lane; it owns all 64 columns of every S block. P_n is
+    // published as soon as it is stored, so the MMA warp can issue P_n V_n and S_{n+2}
+    // while this warpgroup waits for S_{n+1}.
     const int quarter = warp & 3;               // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;          // query row within the tile
     const int wt = tid - 64;                    // 0..127
@@ -357,19 +369,20 @@ __global__ void __launch_bounds__(192, 2)
         const uint64_t pst = f2_add(ps2, ps2b);
         l_run += f2_lo(pst) + f2_hi(pst);
         tmem_st32(lane_addr + b * 64, pk);  // P over the first 32 columns of its S
-        // the next block's S: its load overlaps the store of P
+        // Publish P_n before waiting for S_{n+1}: P*V of this block, and the S two blocks on
+        // (which reuses these columns), can then be issued while S_{n+1} is still in flight.
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
         if (n + 1 < kc) {
           ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b ^ 1], ((ns + 1) >> 1) & 1, a.err, &abort_flag));
           if (ok) {
             tc_fence_after();
             tmem_ld32(lane_addr + (b ^ 1) * 64, sa);
             tmem_ld32(lane_addr + (b ^ 1) * 64 + 32, sb);
+            tmem_wait_ld();
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[b]);
-        if (n + 1 < kc) tmem_wait_ld();
         j_cur = j_next;
       }
       // Every MMA that reads Q (or the S/P columns) has finished once the last PV has.

@@ -436,18 +436,19 @@ __global__ void __launch_bounds__(192, 2)
         const uint64_t pst = f2_add(ps2, ps2b);
         l_run += mul_pow2(f2_lo(pst) + f2_hi(pst), -pe);
         tmem_st16(lane_addr + b * 64, pk);  // P8 over the first 16 columns of its S
+        // P_n is published before S_{n+1} is waited for (see attn_kernel)
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
         if (n + 1 < kc) {
           ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b ^ 1], ((ns + 1) >> 1) & 1, a.err, &abort_flag));
           if (ok) {
             tc_fence_after();
             tmem_ld32(lane_addr + (b ^ 1) * 64, sa);
             tmem_ld32(lane_addr + (b ^ 1) * 64 + 32, sb);
+            tmem_wait_ld();
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[b]);
-        if (n + 1 < kc) tmem_wait_ld();
         j_cur = j_nxt;
         j_nxt = j_nn;
         ek_cur = ek_next;

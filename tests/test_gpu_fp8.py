@@ -40,16 +40,16 @@ def _assert_within_bound(got, ref, bound, what):
     rows = ~np.isnan(ref[..., 0])
     g, r, bd = got[rows], ref[rows], bound[rows]
     assert np.all(np.isfinite(g)), f"{what}: non-finite GPU output"
-    # per (b, h, channel) magnitude of the output, broadcast back to the rows
-    mag = np.maximum(1.0, np.nanmax(np.abs(ref), axis=-2, keepdims=True))
+    # per (b, h, channel) magnitude of the output over the computed rows, broadcast back
+    absref = np.where(rows[..., None], np.abs(np.nan_to_num(ref)), 0.0)
+    mag = np.maximum(1.0, absref.max(axis=-2, keepdims=True))
     scale = np.broadcast_to(mag, ref.shape)[rows]
     d = np.abs(g - r)
     excess = np.maximum(d - bd, 0.0) / scale
     mx, mean = float(excess.max()), float(excess.mean())
-    used = float(d.mean() / max(bd.mean(), 1e-300))
+    used = f"{d.mean() / bd.mean():.3f} of it used on average" if bd.mean() > 0 else "no sparse branch"
     print(f"{what}: beyond-bound max {mx:.3e} mean {mean:.3e} (scaled); raw max-abs {d.max():.3e} "
-          f"mean-abs {d.mean():.3e}; mean bound {bd.mean():.3e} ({used:.3f} of it used on average); "
-          f"largest |O*| {float(mag.max()):.2f}")
+          f"mean-abs {d.mean():.3e}; mean bound {bd.mean():.3e} ({used}); largest |O*| {float(mag.max()):.2f}")
     assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max {mx:.3e}, mean {mean:.3e} beyond the bound"
     return mx, mean
 
