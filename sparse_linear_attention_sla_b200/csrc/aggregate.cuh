@@ -23,7 +23,13 @@ struct AggArgs {
   __nv_bfloat16* Hagg;   // [BH, Nq, D*D]
   float* Zagg;           // [BH, Nq, D]
   uint32_t* err;
+  // Nullable. When set, column e of H_i (head h) is written times
+  // gamma = (1 - alpha[h, e]) / max(alpha[h, e], kAlphaFloor): the fused attention then adds
+  // the linear branch into the sparse branch's accumulator (see attn_kernel). Z_i is unscaled.
+  const float* alpha;    // [H, D]
+  int H;
 };
+
 
 constexpr int kAggStages = 4;
 constexpr uint32_t kAggStageBytes = 3 * 16384;  // A for two M-tiles + one B tile (64 x 128)
@@ -151,6 +157,7 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
     const int rloc = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint8_t* stg = smem + kAggStages * kAggStageBytes;
+    __shared__ float sGamma[128];  // per-column factor of the current tile (1 when alpha is not given)
     int tc = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
       int n0, m0, bh, nm;
@@ -160,6 +167,13 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
       if (!named_barrier_and(1, 128, ok)) break;
       tc_fence_after();
       const bool z_tile = n0 >= D * D;
+      if (a.alpha && !z_tile) {  // column c of the tile is channel (n0 + c) % D of h_j's rows
+        const float al = a.alpha[(bh % a.H) * D + (n0 + et) % D];
+        sGamma[et] = (1.f - al) / fmaxf(al, kAlphaFloor);
+      } else {
+        sGamma[et] = 1.f;
+      }
+      named_barrier(1, 128);
       for (int tt = 0; tt < nm; ++tt) {
         if (!z_tile) {  // the staging tile is free once the previous store has read it
           if (et == 0) tma_store_wait_read();
@@ -175,12 +189,14 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
           for (int q = 0; q < 4; ++q) {
             uint8_t* box = stg + (q >> 1) * 16384;
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              *reinterpret_cast<uint4*>(box + sw128_offset(rloc, ((q & 1) * 4 + v) * 16)) =
-                  make_uint4(pack_bf16x2(__uint_as_float(r[q][8 * v + 0]), __uint_as_float(r[q][8 * v + 1])),
-                             pack_bf16x2(__uint_as_float(r[q][8 * v + 2]), __uint_as_float(r[q][8 * v + 3])),
-                             pack_bf16x2(__uint_as_float(r[q][8 * v + 4]), __uint_as_float(r[q][8 * v + 5])),
-                             pack_bf16x2(__uint_as_float(r[q][8 * v + 6]), __uint_as_float(r[q][8 * v + 7])));
+            for (int v = 0; v < 4; ++v) {
+              const float* g = &sGamma[32 * q + 8 * v];
+              *reinterpret_cast<uint4*>(box + sw128_offset(rloc, ((q & 1) * 4 + v) * 16)) = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[q][8 * v + 0]) * g[0], __uint_as_float(r[q][8 * v + 1]) * g[1]),
+                  pack_bf16x2(__uint_as_float(r[q][8 * v + 2]) * g[2], __uint_as_float(r[q][8 * v + 3]) * g[3]),
+                  pack_bf16x2(__uint_as_float(r[q][8 * v + 4]) * g[4], __uint_as_float(r[q][8 * v + 5]) * g[5]),
+                  pack_bf16x2(__uint_as_float(r[q][8 * v + 6]) * g[6], __uint_as_float(r[q][8 * v + 7]) * g[7]));
+            }
           }
         } else if (m < a.Nq) {
           float4* dst = reinterpret_cast<float4*>(a.Zagg + (static_cast<size_t>(bh) * a.Nq + m) * D);

@@ -4,7 +4,7 @@
 //   sparse branch  O_s = softmax over the keys of the critical KV blocks only
 //                        (online softmax, renormalised over that set)
 //   linear branch  O_l = phi(Q_i) H_i / (phi(Q_i) Z_i), H_i, Z_i = sums of the
-//                        marginal blocks' states (precomputed per row)
+//                        marginal blocks' states (aggregated per query block)
 //   blend          O   = alpha_h * O_s + (1 - alpha_h) * O_l        (per channel)
 //
 // Sources: "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
@@ -19,21 +19,33 @@
 // in head-major order, so a head's K/V stay in L2 and the next tile's loads overlap the
 // current tile's epilogue. Warp roles (192 threads):
 //   warp 0      TMA producer: per tile Q, then K_j / V_j of every critical block
-//               through a 2-slot ring, then H_i into the next slot (a pseudo-block
-//               of the ring: its two halves complete the slot's K and V barriers).
+//               through a 2-slot ring, then H~_i into the next slot (a pseudo-block
+//               of the ring: its two halves complete the slot's K and V barriers). The
+//               next tile's Q is loaded once the tile's last S MMA is done and every row
+//               of the warpgroup has read its Q for phi(q).
 //   warp 1      TMEM owner and tcgen05 issuer (the warp runs the loop, one elected lane
 //               issues):
-//               S = Q K_j^T (M=128, N=64), O_s += P V_j (M=128, N=D, P read from
-//               TMEM), O_l = phi(Q) H_i (M=128, N=D).
+//               S = Q K_j^T (M=128, N=64), acc += P V_j (M=128, N=D, P read from
+//               TMEM), and after the last block acc += P_lin H~_i (P_lin from TMEM).
 //   warps 2..5  softmax / epilogue warpgroup: a thread owns one query row (= TMEM lane)
 //               and all 64 columns of each S block; P_n is published before S_{n+1} is
 //               waited for.
 //
+// The linear branch shares the sparse branch's accumulator. With l the softmax
+// normaliser, den = phi(q) . Z_i and H~_i = H_i diag((1 - alpha) / alpha) (the aggregation
+// writes H_i scaled so), the blend is
+//     O = alpha acc / l + (1 - alpha) phi(q) H_i / den = alpha (acc + (l / den) phi(q) H~_i) / l,
+// so the warpgroup writes P_lin = (l / den) phi(q) into TMEM and the epilogue reads one
+// accumulator (alpha is floored at 2^-24 on both sides).
+//
 // TMEM columns: S ping-pong [0,64) [64,128) (P, bf16, is written back over the
-// first 32 columns of its S), O_s [128,128+D); after a tile's sparse loop O_l
-// reuses [0,D) until the epilogue has read it. tcgen05 MMAs issued by one thread
-// run in order, so S_{n+2} never overwrites P_n before PV_n has read it.
-// An empty critical set gives O_s = 0; an empty marginal set gives Z_i = 0 and O_l = 0.
+// first 32 columns of its S), acc [128,128+D); after a tile's sparse loop P_lin takes the
+// S columns the next block would have used. tcgen05 MMAs issued by one thread run in
+// order, so S_{n+2} never overwrites P_n before PV_n has read it, and the next tile's S
+// never overwrites P_lin before the linear MMA has read it. The next tile's first write
+// of acc waits for this tile's epilogue.
+// An empty critical set gives O_s = 0 (l taken as 1); an empty marginal set gives Z_i = 0
+// and no linear term.
 #pragma once
 
 #include "sm100.cuh"
@@ -71,7 +83,8 @@ struct AttnSmem {
 template <int D>
 __global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h, AttnArgs a) {
+                const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
+                const __grid_constant__ CUtensorMap map_o, AttnArgs a) {
   using L = AttnSmem<D>;
   constexpr int DB = D / 64;  // 64-column boxes per row
   constexpr uint32_t TMEM_COLS = 256;
@@ -81,21 +94,21 @@ __global__ void __launch_bounds__(192, 2)
   uint8_t* sQ = base;
   uint8_t* sRing = sQ + L::Q;  // slot s at sRing + s * SLOT: K at +0, V at +KV
 
-  __shared__ uint64_t q_full, q_free, phiq_full, ol_done, tmem_free, drain;
+  __shared__ uint64_t q_full, q_free, plin_full, lin_done, tmem_free, drain;
   __shared__ uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
-  __shared__ __align__(16) float sZ[D];
-  __shared__ __align__(16) float sAlpha[D];
+  __shared__ __align__(16) float sZ[D];      // Z_i of the current tile
+  __shared__ __align__(16) float sAlpha[D];  // max(alpha, 2^-24) of the current tile's head
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
-    mbar_init(&q_free, 1);
-    mbar_init(&phiq_full, 128);
-    mbar_init(&ol_done, 1);
+    mbar_init(&q_free, 1 + 128);  // the tile's last S MMA, and every row read for phi(q)
+    mbar_init(&plin_full, 128);
+    mbar_init(&lin_done, 1);
     mbar_init(&tmem_free, 128);
     mbar_init(&drain, 1);
     for (int s = 0; s < 2; ++s) {
@@ -196,9 +209,12 @@ __global__ void __launch_bounds__(192, 2)
       if (elect_one()) umma_commit(bar);
       __syncwarp();
     };
-    // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites O_s.
+    // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites O_s, which the
+    // previous tile's epilogue must have read (tile k > 0).
+    int k = 0;
     auto issue_pv = [&](uint32_t nbm, uint32_t nsm, bool first) -> bool {
       const int s = nbm & 1, b = nsm & 1;
+      if (first && k > 0 && !wait_all(&tmem_free, (k - 1) & 1)) return false;
       if (!wait_all(&p_full[b], (nsm >> 1) & 1)) return false;
       if (!wait_all(&v_full[s], (nbm >> 1) & 1)) return false;
       tc_fence_after();
@@ -213,12 +229,9 @@ __global__ void __launch_bounds__(192, 2)
       commit(&v_empty[s]);
       return true;
     };
-    int k = 0;
     for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
       const int kc = a.crit_cnt[t];
       if (!(ok = wait_all(&q_full, k & 1))) break;
-      // the epilogue of the previous tile has read O_s and O_l out of TMEM
-      if (k > 0 && !(ok = wait_all(&tmem_free, (k - 1) & 1))) break;
       for (int n = 0; n < kc; ++n, ++nb, ++ns) {
         const int s = nb & 1, b = ns & 1;
         if (!(ok = wait_all(&k_full[s], (nb >> 1) & 1))) break;
@@ -233,28 +246,31 @@ __global__ void __launch_bounds__(192, 2)
         }
         commit(&s_full[b]);
         commit(&k_empty[s]);
+        if (n + 1 == kc) commit(&q_free);  // no MMA of this tile reads Q after its last S
         if (n >= 1 && !(ok = issue_pv(nb - 1, ns - 1, n == 1))) break;
       }
       if (!ok) break;
+      if (kc == 0) commit(&q_free);
       if (kc > 0 && !(ok = issue_pv(nb - 1, ns - 1, kc == 1))) break;
-      // linear branch: O_l = phi(Q) H_i once H_i has landed and the warpgroup rewrote Q as phi(Q)
+      // Linear branch, added into the sparse accumulator: O_s += P_lin H~_i with
+      // P_lin = (l / den) phi(Q) written by the warpgroup into the S columns after the last
+      // block (ns & 1) and H~_i (H_i with its columns scaled by (1 - alpha) / alpha) in the
+      // next ring slot. With no critical block this is the first write of O_s.
       const int s = nb & 1;
+      if (kc == 0 && k > 0 && !(ok = wait_all(&tmem_free, (k - 1) & 1))) break;
       if (!(ok = wait_all(&k_full[s], (nb >> 1) & 1))) break;
       if (!(ok = wait_all(&v_full[s], (nb >> 1) & 1))) break;
-      if (!(ok = wait_all(&phiq_full, k & 1))) break;
+      if (!(ok = wait_all(&plin_full, k & 1))) break;
       tc_fence_after();
       const uint32_t hb = ring0 + s * L::SLOT;
+      const uint32_t pl = tmem + (ns & 1) * 64;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t ad = smem_desc_sw128(q0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
         const uint64_t bd = smem_desc_sw128(hb + (kk >> 2) * DB * 8192 + (kk & 3) * 2048, 8192, 1024);
-        if (elect_one()) umma_bf16_ss(tmem + OL, ad, bd, id_o, kk > 0 ? 1u : 0u);
+        if (elect_one()) umma_bf16_ts(tmem + OS, pl + kk * 8, bd, id_o, (kc > 0 || kk > 0) ? 1u : 0u);
         __syncwarp();
       }
-      commit(&ol_done);
-      commit(&q_free);
-      commit(&k_empty[s]);
-      commit(&v_empty[s]);
+      commit(&lin_done);  // the H~_i slot is released by the warpgroup once the output staged there is stored
       ++nb;
     }
     commit(&drain);  // every MMA issued above has finished once this arrives
@@ -269,21 +285,36 @@ __global__ void __launch_bounds__(192, 2)
     const int wt = tid - 64;                    // 0..127
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float sc = a.scale_log2;
-    uint32_t ns = 0;  // S/P blocks so far
+    uint32_t ns = 0;   // S/P blocks so far
+    uint32_t nbw = 0;  // ring uses so far (K/V blocks and H~_i pseudo-blocks)
     bool ok = true;
     int k = 0;
+    // This thread's entries of Z_i and alpha for the tile after the current one, loaded
+    // during the current tile so that their latency stays off the tile boundary.
+    float z_next = 0.f, a_next = 0.f;
+    if (wt < D && static_cast<int>(blockIdx.x) < a.n_tiles) {
+      z_next = a.Zagg[static_cast<size_t>(blockIdx.x) * D + wt];
+      a_next = a.alpha[(blockIdx.x / a.Nq % a.H) * D + wt];
+    }
     // Every barrier of the warpgroup ANDs the threads' status, so a failed wait makes all
     // 128 threads leave together.
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++k) {
-      const int bh = t / a.Nq, i = t % a.Nq, h = bh % a.H;
+      const int bh = t / a.Nq, i = t % a.Nq;
       const int kc = a.crit_cnt[t];
       const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
+      const uint32_t hs = (nbw + kc) & 1;  // ring slot of this tile's H~_i, reused to stage O
+      nbw += kc + 1;
       if (!named_barrier_and(1, 128, ok)) break;  // the previous tile's epilogue is done with sZ / sAlpha
-      for (int c = wt; c < D; c += 128) {
-        sZ[c] = a.Zagg[static_cast<size_t>(t) * D + c];
-        sAlpha[c] = a.alpha[h * D + c];
+      if (wt < D) {
+        sZ[wt] = z_next;
+        sAlpha[wt] = fmaxf(a_next, kAlphaFloor);
       }
       if (!named_barrier_and(1, 128, ok)) break;  // sZ / sAlpha of this tile are visible
+      if (wt < D && t + static_cast<int>(gridDim.x) < a.n_tiles) {
+        const int tn = t + gridDim.x;
+        z_next = a.Zagg[static_cast<size_t>(tn) * D + wt];
+        a_next = a.alpha[(tn / a.Nq % a.H) * D + wt];
+      }
       float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and row sum
       uint32_t sa[32], sb[32];               // S columns [0, 32) and [32, 64) of the current block
       int j_cur = kc > 0 ? clist[0] : 0;
@@ -385,31 +416,34 @@ __global__ void __launch_bounds__(192, 2)
         }
         j_cur = j_next;
       }
-      // Every MMA that reads Q (or the S/P columns) has finished once the last PV has.
-      if (ok && kc > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
+      // Linear branch. P_lin goes into the S columns the next block would have used
+      // (ns & 1); their last reader is the P*V two blocks back (with one block or none, an
+      // MMA of an earlier tile, finished before this tile's lin_done was seen).
+      if (ok && kc >= 2)
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 2) & 1], ((ns - 2) >> 1) & 1, a.err, &abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, k & 1, a.err, &abort_flag));
-
-      // phi(Q) in place (bf16) over the row, and the linear-branch denominator phi(q) . Z_i
-      // with the same rounded phi(q) the MMA sees. Column pairs in paired arithmetic:
-      // phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e); even and odd columns' products
-      // with Z_i are summed in the two lanes.
+      // Pass 1: phi(q) (bf16, as the tensor core takes it) into the P_lin columns, 32
+      // elements at a time, and den = phi(q) . Z_i from those rounded values; then the Q tile
+      // is released (the next tile's Q may land). Column pairs in paired arithmetic:
+      // phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e).
+      const uint32_t pl = lane_addr + (ns & 1) * 64;
       uint64_t den2 = 0ull;
       if (ok) {
         const uint64_t one2 = f2_make(1.f, 1.f), log2e2 = f2_make(1.4426950408889634f, 1.4426950408889634f);
-#pragma unroll 2
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          uint4* p = reinterpret_cast<uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
-          uint4 u = *p;
-          uint32_t w[4] = {u.x, u.y, u.z, u.w};
-          const uint4 z01 = *reinterpret_cast<const uint4*>(&sZ[c8 * 8]);
-          const uint4 z23 = *reinterpret_cast<const uint4*>(&sZ[c8 * 8 + 4]);
-          const uint64_t z2[4] = {static_cast<uint64_t>(z01.x) | (static_cast<uint64_t>(z01.y) << 32),
-                                  static_cast<uint64_t>(z01.z) | (static_cast<uint64_t>(z01.w) << 32),
-                                  static_cast<uint64_t>(z23.x) | (static_cast<uint64_t>(z23.y) << 32),
-                                  static_cast<uint64_t>(z23.z) | (static_cast<uint64_t>(z23.w) << 32)};
+#pragma unroll 1
+        for (int g = 0; g < D / 32; ++g) {
+          uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int c = 0; c < 4; ++c) {
+            const int c8 = 4 * g + c;
+            const uint4 u = *reinterpret_cast<const uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
+            w[4 * c] = u.x;
+            w[4 * c + 1] = u.y;
+            w[4 * c + 2] = u.z;
+            w[4 * c + 3] = u.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
             // bf16 -> fp32 is a shift into the high half-word
             const uint64_t x2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
             const uint64_t pos2 = f2_add(x2, one2);
@@ -418,54 +452,86 @@ __global__ void __launch_bounds__(192, 2)
             const float g1 = f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
             w[e] = pack_bf16x2(g0, g1);
             const uint64_t gr2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
-            den2 = f2_fma(gr2, z2[e], den2);
+            den2 = f2_fma(gr2, *reinterpret_cast<const uint64_t*>(&sZ[32 * g + 2 * e]), den2);
           }
-          *p = make_uint4(w[0], w[1], w[2], w[3]);
+          tmem_st16(pl + 16 * g, w);
         }
-        fence_proxy_async_smem();
       }
+      mbar_arrive(&q_free);
+      // The blend O = alpha O_s / l + (1 - alpha) O_l / den, with the accumulator holding
+      // l O_s and H~_i = H_i (1 - alpha) / alpha, is alpha (acc + (l / den) phi(q) H~_i) / l.
+      // With no critical block l is taken as 1 (acc starts at 0); with no marginal block
+      // (den = 0) the linear term is 0.
       const float den_tot = f2_lo(den2) + f2_hi(den2);
+      const float l_eff = kc > 0 ? l_run : 1.f;
+      const float c_lin = den_tot > 0.f ? l_eff / den_tot : 0.f;
+      // Pass 2: P_lin = (l / den) phi(q), rounded to bf16 in place.
+      if (ok) {
+        tmem_wait_st();
+        const uint64_t c2 = f2_make(c_lin, c_lin);
+#pragma unroll 1
+        for (int g = 0; g < D / 64; ++g) {
+          uint32_t w[32];
+          tmem_ld32(pl + 32 * g, w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint64_t g2 = f2_mul(c2, static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32));
+            w[e] = pack_bf16x2(f2_lo(g2), f2_hi(g2));
+          }
+          tmem_st32(pl + 32 * g, w);
+        }
+        tmem_wait_st();
+      }
       tc_fence_before();
-      mbar_arrive(&phiq_full);
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, k & 1, a.err, &abort_flag));
+      mbar_arrive(&plin_full);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&lin_done, k & 1, a.err, &abort_flag));
       if (!(ok = named_barrier_and(1, 128, ok))) break;
 
-      // Epilogue: O = alpha * O_s / l + (1 - alpha) * O_l / den, bf16, straight to global memory.
+      // Epilogue: O = alpha acc / l in bf16, staged row by row in the H~_i slot (the linear MMA
+      // has read it) in the 128-byte swizzle and written by TMA stores of block_q rows (rows
+      // past N are clipped by the tensor map; with block_q = 64 the tile's upper 64 rows belong
+      // to the next query block and are not stored); the loads of the next 32 columns overlap
+      // the arithmetic and shared-memory writes of the current ones.
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      const float inv_d = den_tot > 0.f ? 1.f / den_tot : 0.f;
-      const int tok = i * a.block_q + r;
-      const bool store = r < a.block_q && tok < a.N;
-      __nv_bfloat16* orow = a.out + (static_cast<size_t>(bh) * a.N + tok) * D;
-      // per column pair: y = (alpha inv_l) O_s + ((1 - alpha) inv_d) O_l in paired arithmetic;
-      // O_s is not read when the critical set is empty (its TMEM columns were never written)
-      const uint64_t il2 = f2_make(inv_l, inv_l), id2 = f2_make(inv_d, inv_d);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t os[16], ol[16];
-        if (kc > 0) tmem_ld16(lane_addr + OS + c0, os);
-        tmem_ld16(lane_addr + OL + c0, ol);
-        tmem_wait_ld();
-        uint32_t pk[8];
+      const float inv_l = 1.f / l_eff;
+      uint8_t* stage = sRing + hs * L::SLOT;  // DB boxes of 128 rows x 64 columns
+      const uint64_t il2 = f2_make(inv_l, inv_l);
+      uint32_t ob[2][32];
+      tmem_ld32(lane_addr + OS, ob[0]);
+      tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-          const uint64_t al2 = *reinterpret_cast<const uint64_t*>(&sAlpha[c0 + c]);
-          const uint64_t wl = f2_fma(al2 ^ 0x8000000080000000ull, id2, id2);  // (1 - alpha) inv_d
-          uint64_t y = f2_mul(wl, static_cast<uint64_t>(ol[c]) | (static_cast<uint64_t>(ol[c + 1]) << 32));
-          if (kc > 0)
-            y = f2_fma(f2_mul(al2, il2), static_cast<uint64_t>(os[c]) | (static_cast<uint64_t>(os[c + 1]) << 32), y);
+      for (int q = 0; q < D / 32; ++q) {
+        if (q + 1 < D / 32) tmem_ld32(lane_addr + OS + 32 * (q + 1), ob[(q + 1) & 1]);
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const uint64_t al2 = *reinterpret_cast<const uint64_t*>(&sAlpha[32 * q + c]);
+          const uint64_t y = f2_mul(f2_mul(al2, il2), static_cast<uint64_t>(ob[q & 1][c]) |
+                                                          (static_cast<uint64_t>(ob[q & 1][c + 1]) << 32));
           pk[c >> 1] = pack_bf16x2(f2_lo(y), f2_hi(y));
         }
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
+        uint8_t* box = stage + (q >> 1) * 16384;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(box + sw128_offset(r, ((q & 1) * 4 + v) * 16)) =
+              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        if (q + 1 < D / 32) tmem_wait_ld();
+      }
+      fence_proxy_async_smem();
+      named_barrier(1, 128);
+      if (wt == 0) {
+        for (int b = 0; b < DB; ++b) tma_store_3d(&map_o, stage + b * 16384, b * 64, i * a.block_q, bh);
+        tma_store_commit();
+        tma_store_wait_read();  // the slot may take the next K/V block
+        mbar_arrive(&k_empty[hs]);
+        mbar_arrive(&v_empty[hs]);
       }
       tc_fence_before();
-      mbar_arrive(&tmem_free);  // O_s and O_l have left TMEM: the next tile may overwrite them
+      mbar_arrive(&tmem_free);  // the accumulator has left TMEM: the next tile may overwrite it
     }
   }
+  if (tid == 64) tma_store_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -373,7 +373,7 @@ sla_status launch_router(const Shape& s, const Workspace& w, double* scores64, i
 }
 
 template <int D>
-sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
+sla_status launch_agg(const Shape& s, const Workspace& w, const float* alpha, cudaStream_t st) {
   CUtensorMap mw, mh;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
@@ -397,7 +397,7 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
   }
   const int smem = sla::kAggStages * sla::kAggStageBytes + sla::kAggStagingBytes + 1024;
   SLA_TRY(allow_smem(sla::agg_kernel<D>, smem));
-  AggArgs a{s.Nq, s.Nk, s.LD, s.BH, w.Hagg, w.Zagg, w.err};
+  AggArgs a{s.Nq, s.Nk, s.LD, s.BH, w.Hagg, w.Zagg, w.err, alpha, s.H};
   const long long tiles = static_cast<long long>(s.LD / 128) * ((s.Nq + 255) / 256) * s.BH;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   return launch_dependent(sla::agg_kernel<D>, dim3(grid), dim3(224), smem, st, "agg_kernel", mw, mh, mo, a);
@@ -406,8 +406,11 @@ sla_status launch_agg(const Shape& s, const Workspace& w, cudaStream_t st) {
 template <int D>
 sla_status launch_attn(const Shape& s, const void* q, const void* k, const void* v, const float* alpha, void* out,
                        const Workspace& w, int crit_ld, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mh;
+  CUtensorMap mq, mk, mv, mh, mo;
   SLA_TRY(act_map(&mq, q, s, 128));
+  // output boxes of block_q rows: the staged 128-row tile holds the next query block's rows
+  // past block_q when block_q = 64, and those must not be written
+  SLA_TRY(act_map(&mo, out, s, static_cast<uint32_t>(s.bq)));
   SLA_TRY(act_map(&mk, k, s, 64));
   SLA_TRY(act_map(&mv, v, s, 64));
   {
@@ -434,7 +437,7 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.err = w.err;
   // persistent: two CTAs per SM walk the tiles
   const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
-  return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, a);
+  return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, mo, a);
 }
 
 template <int D>
@@ -539,7 +542,9 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
     SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
   }
   SLA_TRY(ev.mark(2, st));
-  SLA_TRY(launch_agg<D>(s, w, st));
+  // the bf16 attention adds the linear branch into its accumulator and takes H_i scaled per
+  // channel by (1 - alpha) / alpha; the low-bit kernel takes H_i as it is
+  SLA_TRY(launch_agg<D>(s, w, fp8 ? nullptr : alpha, st));
   SLA_TRY(ev.mark(3, st));
   if (fp8) {
     if constexpr (D == 128) {

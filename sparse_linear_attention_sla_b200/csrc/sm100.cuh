@@ -51,6 +51,11 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Smallest alpha the blend O = alpha O_s + (1 - alpha) O_l divides by when the linear branch
+// is folded into the sparse branch's accumulator: an alpha of 0 acts as 2^-24 (the sparse
+// branch then carries a weight of 6e-8 instead of 0).
+constexpr float kAlphaFloor = 5.9604644775390625e-8f;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
