@@ -113,7 +113,10 @@ sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const
  * between the stages, waits for the last one, and writes stage_ms[4] (host):
  * [0] per-block precompute (pooling, KV states), [1] routing (scores and
  * selection, or the caller-mask lists), [2] marginal-state aggregation,
- * [3] fused attention. Synchronises the stream; meant for measurement. */
+ * [3] fused attention. Each stage runs as one launch over every head here, so
+ * that it can be timed alone; sla_forward runs the first three in groups of
+ * heads (see sla_forward_launches), with the same results. Synchronises the
+ * stream; meant for measurement. */
 sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k, const void* v,
                              const float* alpha, const int8_t* mask, void* out, void* ws,
                              size_t ws_bytes, void* stream, float* stage_ms);
@@ -163,6 +166,94 @@ sla_status sla_forward_fp8_timed(const sla_problem* p, const void* q, const void
  * D = 64 or 128. Asynchronous on the stream; writes nothing on an argument error. */
 sla_status sla_quantize_kv(const sla_problem* p, const void* k, const void* v, uint8_t* k8_out,
                            uint8_t* v8_out, int32_t* kexp_out, int32_t* vexp_out, void* stream);
+
+/* Marginal-state aggregation on its own (SLA Abstract: the O(N) linear branch over the
+ * marginal blocks): for each (b, h) and query block i,
+ *   H_i = sum of h_j, Z_i = sum of z_j over the KV blocks j labelled marginal (1) in row i,
+ * with h_j = phi(K_j)^T V_j and z_j = colsum phi(K_j) over the block's valid tokens.
+ * The forward computes the same sums (there H_i is written scaled per channel for its blend).
+ * Precision: phi(k) enters the tensor core in bf16, h_j and z_j are rounded to bf16, the sums
+ * accumulate in fp32, H_i is rounded to bf16.
+ *   k, v    [B,H,N,D] bf16 device, 16-byte aligned
+ *   mask    [B,H,Nq,Nk] int8 device labels (e.g. from sla_route); values outside {0,1,2}
+ *           are reported by sla_check
+ *   H_out   [B,H,Nq,D,D] bf16 device (row-major D x D per query block), 16-byte aligned
+ *   Z_out   [B,H,Nq,D] fp32 device, 16-byte aligned
+ *   ws      workspace of at least sla_workspace_size(p) bytes
+ * Asynchronous on the stream; writes nothing on an argument error. */
+sla_status sla_aggregate_states(const sla_problem* p, const void* k, const void* v, const int8_t* mask,
+                                void* H_out, float* Z_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Number of kernel launches sla_forward (low_bit = 0) or sla_forward_fp8 (low_bit = 1)
+ * enqueues for this problem, with (with_mask = 1) or without a caller mask: the precompute,
+ * labels and aggregation run in groups of heads sized so that a group's per-block states
+ * stay in L2. Host only; -1 for an invalid problem. For measurement. */
+int sla_forward_launches(const sla_problem* p, int with_mask, int low_bit);
+
+/* ---------------------------------------------------------------- backward
+ *
+ * "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable Sparse-Linear Attention",
+ * Abstract: one kernel covers the forward and the backward pass. The pages give no backward
+ * formulas; this is the exact derivative of sla_forward's output with respect to q, k, v
+ * and alpha with the block labels held fixed (the hard top-k passes no gradient):
+ *   sparse branch  softmax attention renormalised over the critical keys, with
+ *                  G_s = alpha dO: dV += P^T G_s, dS = P (G_s V^T - rowsum(G_s O_s)),
+ *                  dQ += dS K / sqrt(D), dK += dS^T Q / sqrt(D)
+ *   linear branch  with u = phi(q), den = u . Z_i, G_l = (1 - alpha) dO:
+ *                  dQ += (G_l H_i^T / den - (G_l . O_l) Z_i / den) phi'(q), and through
+ *                  dH_i = u^T G_l / den, dZ_i = -u^T (G_l . O_l) / den summed into every
+ *                  marginal block's h_j, z_j: dV += phi(K_j) dh_j, dK += (V_j dh_j^T + dz_j) phi'(K_j)
+ *   blend          dalpha[h, :] = sum over rows of dO (O_s - O_l)
+ * phi'(x) = 1 for x > 0, e^x otherwise. Operands enter the tensor cores in bf16 (G_s, the
+ * softmax P and dS, phi(q), dnum = G_l / den, the per-block states and their gradients);
+ * accumulation is fp32. The sparse branch's dK and dV are summed over query tiles with
+ * fp32 global reductions (their order, and so the last bits, vary between runs).
+ *   q, k, v, dO   [B,H,N,D] bf16 device, 16-byte aligned
+ *   alpha         [H,D] fp32 device
+ *   mask          [B,H,Nq,Nk] int8 device labels of the forward (nullable: the router runs)
+ *   dQ, dK, dV    [B,H,N,D] fp32 device outputs, 16-byte aligned
+ *   dalpha        [H,D] fp32 device output
+ *   ws            workspace of sla_workspace_size_backward(p) bytes
+ * Supported: D = 128 and block_q = 128 (else SLA_ERR_UNSUPPORTED). Asynchronous on the
+ * stream; writes nothing on an argument error. */
+
+/* Workspace bytes for sla_backward (0 for an invalid problem). */
+size_t sla_workspace_size_backward(const sla_problem* p);
+
+sla_status sla_backward(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                        const int8_t* mask, const void* dO, float* dQ, float* dK, float* dV, float* dalpha,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- variants
+ *
+ * Variants of the router and of the linear branch's feature map from "SPLA - Atención de
+ * Bloque Dispersa más Lineal para el Modelado de Contexto Largo":
+ *   feature_map  0: phi(x) = elu(x) + 1 (SLA, as sla_forward);
+ *                1: phi(x) = e^x on the raw q and k (§2.3, the parameter-free exponential
+ *                   map), in h_j, z_j and phi(q) of the linear branch;
+ *   block_score  0: S_ij = qbar_i . kbar_j / sqrt(D) (SLA2 §2.B, as sla_route);
+ *                1: the second-order block score (§2.1, diagonal covariance), ranked as its
+ *                   log: S2_ij = qbar_i . kbar_j / sqrt(D) + log1p(sum_d qbar_i,d^2 var_j,d / (2 D)),
+ *                   var_j,d the population variance of channel d over the block's valid
+ *                   keys; labels from S2 with the same total order and counts.
+ * The sparse branch and the blend are those of sla_forward. */
+typedef struct {
+  int feature_map;
+  int block_score;
+} sla_variant;
+
+/* sla_route with a variant's block score. scores_out (nullable) receives the variant's
+ * scores (S2 for block_score = 1). Other arguments as for sla_route; SLA_ERR_INVALID_ARG
+ * for a variant field outside {0, 1}. */
+sla_status sla_route_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
+                             int8_t* mask_out, int32_t* crit_idx_out, double* scores_out, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* sla_forward with a variant's block score (when mask is NULL) and feature map. Arguments as
+ * for sla_forward; the workspace of sla_workspace_size serves. */
+sla_status sla_forward_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
+                               const void* v, const float* alpha, const int8_t* mask, void* out, void* ws,
+                               size_t ws_bytes, void* stream);
 
 /* Synchronise the stream, read and clear the workspace's device error word.
  * Returns SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_BAD_MASK (or SLA_ERR_CUDA). */

@@ -29,13 +29,19 @@ _STATUS = {
 EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sla_forward",
            "sla_forward_timed", "sla_check", "sla_last_error", "sla_version", "sla_route_noalloc",
            "sla_selftest_wait_timeout", "sla_workspace_size_fp8", "sla_forward_fp8", "sla_forward_fp8_timed",
-           "sla_quantize_kv")
+           "sla_quantize_kv", "sla_aggregate_states", "sla_forward_launches", "sla_route_variant",
+           "sla_forward_variant", "sla_workspace_size_backward", "sla_backward")
 
 
 class SlaError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{_STATUS.get(status, status)}: {message}")
         self.status = status
+
+
+class Variant(ctypes.Structure):
+    """sla_variant: feature_map 0 (elu + 1) or 1 (exp); block_score 0 (first order) or 1 (second order)."""
+    _fields_ = [("feature_map", ctypes.c_int), ("block_score", ctypes.c_int)]
 
 
 class Problem(ctypes.Structure):
@@ -77,6 +83,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_quantize_kv.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         lib.sla_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint, vp]
         lib.sla_selftest_wait_timeout.restype = ctypes.c_int
+        lib.sla_aggregate_states.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_workspace_size_backward.argtypes = [P]
+        lib.sla_workspace_size_backward.restype = sz
+        lib.sla_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        V = ctypes.POINTER(Variant)
+        lib.sla_route_variant.argtypes = [P, V, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_forward_variant.argtypes = [P, V, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_forward_launches.argtypes = [P, ctypes.c_int, ctypes.c_int]
+        lib.sla_forward_launches.restype = ctypes.c_int
         lib.sla_last_error.restype = ctypes.c_char_p
         lib.sla_version.restype = ctypes.c_char_p
         for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check",
@@ -181,6 +196,105 @@ def kv_states(k, v, block_kv=64, ws=None):
                                ctypes.c_size_t(ws.numel()), _stream_handle(dev))
     _raise(st)
     return h, z
+
+
+def aggregate_states(k, v, mask, block_q, block_kv=64, ws=None):
+    """Per-query-block sums of the marginal blocks' states: H [B,H,Nq,D,D] bf16, Z [B,H,Nq,D] fp32."""
+    B, H, N, D = k.shape
+    _check_act("k", k, B, H, N, D, k.device)
+    _check_act("v", v, B, H, N, D, k.device)
+    p = problem(B, H, N, D, block_q, block_kv)
+    Nq, Nk, _, _ = counts(p)
+    dev = k.device
+    if mask.dtype != torch.int8 or tuple(mask.shape) != (B, H, Nq, Nk) or not mask.is_contiguous() \
+            or mask.device != dev:
+        raise ValueError(f"mask must be contiguous int8 [{B}, {H}, {Nq}, {Nk}] on {dev}")
+    Hs = torch.empty(B, H, Nq, D, D, dtype=torch.bfloat16, device=dev)
+    Zs = torch.empty(B, H, Nq, D, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = new_workspace(p, dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_aggregate_states(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(mask), _ptr(Hs), _ptr(Zs), _ptr(ws),
+                                      ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+    _raise(st)
+    return Hs, Zs, ws
+
+
+def route_variant(q, k, block_q, block_kv, kh, kl, feature_map=0, block_score=0, want_scores=False,
+                  want_crit=False, ws=None):
+    """sla_route_variant: labels [B,H,Nq,Nk] int8 (and crit_idx, scores when asked)."""
+    B, H, N, D = q.shape
+    _check_act("q", q, B, H, N, D, q.device)
+    _check_act("k", k, B, H, N, D, q.device)
+    p = problem(B, H, N, D, block_q, block_kv, kh, kl)
+    Nq, Nk, kc, _ = counts(p)
+    dev = q.device
+    mask = torch.empty(B, H, Nq, Nk, dtype=torch.int8, device=dev)
+    crit = torch.empty(B, H, Nq, kc, dtype=torch.int32, device=dev) if want_crit else None
+    scores = torch.empty(B, H, Nq, Nk, dtype=torch.float64, device=dev) if want_scores else None
+    if ws is None:
+        ws = new_workspace(p, dev)
+    var = Variant(feature_map, block_score)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_route_variant(ctypes.byref(p), ctypes.byref(var), _ptr(q), _ptr(k), _ptr(mask), _ptr(crit),
+                                   _ptr(scores), _ptr(ws), ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+    _raise(st)
+    return mask, crit, scores
+
+
+def forward_variant(q, k, v, alpha, block_q, block_kv, kh, kl, feature_map=0, block_score=0, mask=None, out=None,
+                    ws=None):
+    """sla_forward_variant: O [B,H,N,D] bf16."""
+    p, out, ws = _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws)
+    var = Variant(feature_map, block_score)
+    lib = load_library()
+    dev = q.device
+    with torch.cuda.device(dev):
+        st = lib.sla_forward_variant(ctypes.byref(p), ctypes.byref(var), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                     _ptr(mask), _ptr(out), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                                     _stream_handle(dev))
+    _raise(st)
+    return out
+
+
+def backward(q, k, v, alpha, dO, block_q=128, block_kv=64, kh=0.05, kl=0.10, mask=None, ws=None):
+    """sla_backward: (dQ, dK, dV [B,H,N,D] fp32, dalpha [H,D] fp32) of sum(dO * O)."""
+    B, H, N, D = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("dO", dO)):
+        _check_act(name, t, B, H, N, D, dev)
+    if alpha.dtype != torch.float32 or tuple(alpha.shape) != (H, D) or not alpha.is_contiguous():
+        raise ValueError(f"alpha must be contiguous fp32 [{H}, {D}]")
+    p = problem(B, H, N, D, block_q, block_kv, kh, kl)
+    Nq, Nk, _, _ = counts(p)
+    if mask is not None and (mask.dtype != torch.int8 or tuple(mask.shape) != (B, H, Nq, Nk)
+                             or not mask.is_contiguous()):
+        raise ValueError(f"mask must be contiguous int8 [{B}, {H}, {Nq}, {Nk}]")
+    lib = load_library()
+    if ws is None:
+        n = lib.sla_workspace_size_backward(ctypes.byref(p))
+        if n == 0:
+            counts(p)
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+        ws[:256].zero_()
+    dQ, dK, dV = (torch.empty(B, H, N, D, dtype=torch.float32, device=dev) for _ in range(3))
+    dalpha = torch.empty(H, D, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = lib.sla_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(mask), _ptr(dO),
+                              _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dalpha), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                              _stream_handle(dev))
+    _raise(st)
+    return dQ, dK, dV, dalpha, ws
+
+
+def forward_launches(p, with_mask=False, low_bit=False) -> int:
+    """Kernel launches one sla_forward (or sla_forward_fp8) call enqueues for problem p."""
+    n = load_library().sla_forward_launches(ctypes.byref(p), int(bool(with_mask)), int(bool(low_bit)))
+    if n < 0:
+        raise SlaError(1, "invalid problem")
+    return n
 
 
 def _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws, fp8=False):

@@ -80,7 +80,7 @@ struct AttnSmem {
   static constexpr uint32_t total() { return Q + 2 * SLOT + 1024; }
 };
 
-template <int D>
+template <int D, int FM = 0>  // FM: feature map of the linear branch, 0 elu + 1, 1 e^x
 __global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(192, 2)
   using L = AttnSmem<D>;
   constexpr int DB = D / 64;  // 64-column boxes per row
   constexpr uint32_t TMEM_COLS = 256;
-  constexpr uint32_t OS = 128, OL = 0;
+  constexpr uint32_t OS = 128;  // the accumulator's first TMEM column
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
@@ -287,6 +287,7 @@ __global__ void __launch_bounds__(192, 2)
     const float sc = a.scale_log2;
     uint32_t ns = 0;   // S/P blocks so far
     uint32_t nbw = 0;  // ring uses so far (K/V blocks and H~_i pseudo-blocks)
+    int release_slot = -1;  // (thread 0 of the warpgroup) ring slot still held by an output store
     bool ok = true;
     int k = 0;
     // This thread's entries of Z_i and alpha for the tile after the current one, loaded
@@ -310,6 +311,15 @@ __global__ void __launch_bounds__(192, 2)
         sAlpha[wt] = fmaxf(a_next, kAlphaFloor);
       }
       if (!named_barrier_and(1, 128, ok)) break;  // sZ / sAlpha of this tile are visible
+      // The previous tile's output, staged in its H~_i slot, has been read out by the TMA
+      // store once this thread's bulk group is done reading: the slot may take a K/V block
+      // again (the next one needed there is this tile's second block, or a later one).
+      if (release_slot >= 0) {
+        tma_store_wait_read();
+        mbar_arrive(&k_empty[release_slot]);
+        mbar_arrive(&v_empty[release_slot]);
+        release_slot = -1;
+      }
       if (wt < D && t + static_cast<int>(gridDim.x) < a.n_tiles) {
         const int tn = t + gridDim.x;
         z_next = a.Zagg[static_cast<size_t>(tn) * D + wt];
@@ -425,7 +435,7 @@ __global__ void __launch_bounds__(192, 2)
       // Pass 1: phi(q) (bf16, as the tensor core takes it) into the P_lin columns, 32
       // elements at a time, and den = phi(q) . Z_i from those rounded values; then the Q tile
       // is released (the next tile's Q may land). Column pairs in paired arithmetic:
-      // phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e).
+      // phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e) (with FM = 1, e^x throughout).
       const uint32_t pl = lane_addr + (ns & 1) * 64;
       uint64_t den2 = 0ull;
       if (ok) {
@@ -448,8 +458,8 @@ __global__ void __launch_bounds__(192, 2)
             const uint64_t x2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
             const uint64_t pos2 = f2_add(x2, one2);
             const uint64_t t2 = f2_mul(x2, log2e2);
-            const float g0 = f2_lo(x2) > 0.f ? f2_lo(pos2) : fast_exp2(f2_lo(t2));
-            const float g1 = f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
+            const float g0 = FM == 0 && f2_lo(x2) > 0.f ? f2_lo(pos2) : fast_exp2(f2_lo(t2));
+            const float g1 = FM == 0 && f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
             w[e] = pack_bf16x2(g0, g1);
             const uint64_t gr2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
             den2 = f2_fma(gr2, *reinterpret_cast<const uint64_t*>(&sZ[32 * g + 2 * e]), den2);
@@ -523,9 +533,7 @@ __global__ void __launch_bounds__(192, 2)
       if (wt == 0) {
         for (int b = 0; b < DB; ++b) tma_store_3d(&map_o, stage + b * 16384, b * 64, i * a.block_q, bh);
         tma_store_commit();
-        tma_store_wait_read();  // the slot may take the next K/V block
-        mbar_arrive(&k_empty[hs]);
-        mbar_arrive(&v_empty[hs]);
+        release_slot = static_cast<int>(hs);  // released at the next tile's start (see there)
       }
       tc_fence_before();
       mbar_arrive(&tmem_free);  // the accumulator has left TMEM: the next tile may overwrite it

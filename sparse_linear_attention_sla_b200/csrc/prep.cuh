@@ -6,7 +6,8 @@
 //       kbar_j = mean of the valid keys (fp64, router input),
 //       z_j    = colsum phi(K_j)            (linear-attention normaliser state),
 //       h_j    = phi(K_j)^T V_j (D x D)     (linear-attention state, tcgen05 MMA),
-//     with phi(x) = elu(x) + 1; per query block i, qbar_i = mean of the valid queries.
+//     with phi(x) = elu(x) + 1 (or e^x, the exponential feature map variant); per query
+//     block i, qbar_i = mean of the valid queries.
 //
 // Sources: "SLA2: Sparse-Linear Attention with Learnable Routing and QAT" §2.B
 // (pooling adjacent Q/K tokens for the router); "SLA: Beyond Sparsity in
@@ -19,7 +20,38 @@
 
 namespace sla {
 
-__device__ __forceinline__ float phi_f(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+// Feature map of the linear branch: FM = 0 is elu(x) + 1 (x + 1 for x > 0, e^x otherwise);
+// FM = 1 is the exponential map e^x ("SPLA - Atención de Bloque Dispersa más Lineal para el
+// Modelado de Contexto Largo", §2.3).
+template <int FM>
+__device__ __forceinline__ float phi_f(float x) {
+  if constexpr (FM == 1) return __expf(x);
+  return x > 0.f ? x + 1.f : __expf(x);
+}
+
+// Exact fp64 value of a bf16 without the conversion unit. For a normal bf16 (exponent field
+// E in 1..254, 7 mantissa bits M) the fp64 has exponent field E + 896 and M as its top
+// mantissa bits, so its high word is (magnitude << 13) + (896 << 20) with the sign on top
+// and its low word is 0. bf16_lo_f64 takes the bf16 in bits 0..15 of a packed pair,
+// bf16_hi_f64 the one in bits 16..31.
+__device__ __forceinline__ double bf16_lo_f64(uint32_t w) {
+  const uint32_t hi = (((w & 0x7FFFu) << 13) + 0x38000000u) | ((w & 0x8000u) << 16);
+  return __hiloint2double(static_cast<int>(hi), 0);
+}
+__device__ __forceinline__ double bf16_hi_f64(uint32_t w) {
+  const uint32_t hi = (((w & 0x7FFF0000u) >> 3) + 0x38000000u) | (w & 0x80000000u);
+  return __hiloint2double(static_cast<int>(hi), 0);
+}
+// True if either bf16 of a packed pair has exponent field 0 (zero or subnormal) or 255
+// (infinity or NaN): those take the conversion instruction instead. Per 16-bit half, with
+// t the exponent bits in place: t + 0x80 carries into bit 15 only for 0xFF, and
+// (t | 0x8000) - 0x80 clears bit 15 only for 0.
+__device__ __forceinline__ bool bf16x2_not_normal(uint32_t w) {
+  const uint32_t t = w & 0x7F807F80u;
+  const uint32_t all_ones = (t + 0x00800080u) & 0x80008000u;
+  const uint32_t zero = ~((t | 0x80008000u) - 0x00800080u) & 0x80008000u;
+  return (all_ones | zero) != 0u;
+}
 
 // ---------------------------------------------------------------- pooling
 // grid: (nblocks, BH); block: 128 threads. x: [BH, N, D] bf16; out: [BH, nblocks, D] fp64.
@@ -40,11 +72,18 @@ __global__ void __launch_bounds__(128) pool_mean_kernel(const __nv_bfloat16* __r
   for (int r = r0 + rr; r < r1; r += RSTEP) {
     uint4 u = *reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * D);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    const bool rare = bf16x2_not_normal(w[0]) | bf16x2_not_normal(w[1]) | bf16x2_not_normal(w[2]) |
+                      bf16x2_not_normal(w[3]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 f = unpack_bf16x2(w[e]);
-      acc[2 * e] += static_cast<double>(f.x);
-      acc[2 * e + 1] += static_cast<double>(f.y);
+      if (!rare) {
+        acc[2 * e] += bf16_lo_f64(w[e]);
+        acc[2 * e + 1] += bf16_hi_f64(w[e]);
+      } else {
+        const float2 f = unpack_bf16x2(w[e]);
+        acc[2 * e] += static_cast<double>(f.x);
+        acc[2 * e + 1] += static_cast<double>(f.y);
+      }
     }
   }
 #pragma unroll
@@ -84,7 +123,7 @@ struct PrepSmem {
 // rows in fp64 and, for a K tile (PHI), sums phi(k) in fp32 and rewrites the tile in
 // place as phi(k) (zero past the sequence end). The row groups of a warp are summed with
 // shuffles; the warp's partial sums go to part_d / part_f[wq] (wq = warp within the group).
-template <int D, int ROWS, bool PHI>
+template <int D, int ROWS, bool PHI, int FM = 0>
 __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int wq, int valid, double (*part_d)[D],
                                             float (*part_f)[D]) {
   constexpr int RG = 128 / (D / 8);
@@ -104,16 +143,23 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
     const uint4 u = *p;
     uint32_t w[4] = {u.x, u.y, u.z, u.w};
     const bool in = rr < valid;
+    const bool rare = bf16x2_not_normal(w[0]) | bf16x2_not_normal(w[1]) | bf16x2_not_normal(w[2]) |
+                      bf16x2_not_normal(w[3]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 x = unpack_bf16x2(w[e]);
       float f0 = 0.f, f1 = 0.f;
       if (in) {
-        ks[2 * e] += static_cast<double>(x.x);
-        ks[2 * e + 1] += static_cast<double>(x.y);
+        if (!rare) {  // exact either way; the integer form keeps the conversion unit free
+          ks[2 * e] += bf16_lo_f64(w[e]);
+          ks[2 * e + 1] += bf16_hi_f64(w[e]);
+        } else {
+          ks[2 * e] += static_cast<double>(x.x);
+          ks[2 * e + 1] += static_cast<double>(x.y);
+        }
         if (PHI) {
-          f0 = phi_f(x.x);
-          f1 = phi_f(x.y);
+          f0 = phi_f<FM>(x.x);
+          f1 = phi_f<FM>(x.y);
           zs[2 * e] += f0;
           zs[2 * e + 1] += f1;
         }
@@ -154,7 +200,7 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
 //               or TMEM -> fp32 straight to global memory (state export)
 // For D = 64 the second half of phi(K)^T (rows 64..127 of the M=128 MMA) points
 // at a zero tile, so the result rows 64..127 are zero and ignored.
-template <int D>
+template <int D, int FM = 0>
 __global__ void __launch_bounds__(576, 1)
     prep_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_hout, PrepArgs a) {
@@ -300,7 +346,7 @@ __global__ void __launch_bounds__(576, 1)
         else
           column_pass<D, 64, false>(slotp, cc, rg, wq, valid, part_d[cw], part_f[cw]);
       } else {
-        column_pass<D, 64, true>(slotp, cc, rg, wq, valid, part_d[cw], part_f[cw]);
+        column_pass<D, 64, true, FM>(slotp, cc, rg, wq, valid, part_d[cw], part_f[cw]);
       }
       if (!isq) fence_proxy_async_smem();
       named_barrier(bar_id, 128);

@@ -14,9 +14,12 @@
 #include "aggregate.cuh"
 #include "attention.cuh"
 #include "attention_fp8.cuh"
+#include "backward.cuh"
+#include "backward_states.cuh"
 #include "fp8.cuh"
 #include "prep.cuh"
 #include "route.cuh"
+#include "variants.cuh"
 
 namespace {
 
@@ -94,6 +97,7 @@ struct Workspace {
   uint32_t* err;
   double* qbar;
   double* kbar;
+  double* var;  // per-block channel variances of K (the second-order block score)
   double* S;    // fp64 scores (the long-row selection)
   float* S32;   // fp32 scores (the certified selection), aliases S
   float* nq;    // fp32 norms of the pooled queries
@@ -105,6 +109,13 @@ struct Workspace {
   __nv_bfloat16* hst;
   __nv_bfloat16* Hagg;
   float* Zagg;
+  // backward only
+  __nv_bfloat16* gs;    // alpha * dO [BH, N, D]
+  __nv_bfloat16* dHst;  // [BH, Nq, LD]: dH_i row-major, then dZ_i, then zero pad
+  __nv_bfloat16* WT;    // marginal indicator transposed [BH, Nk, wt_ld]
+  __nv_bfloat16* dh;    // [BH, Nk, D*D] gradients of the per-block states
+  float* dz;            // [BH, Nk, D]
+  int wt_ld;
   // low-bit sparse branch only
   uint8_t* k8;     // e4m3 codes of K [BH, N, D]
   uint8_t* v8;     // e4m3 codes of V [BH, N, D]
@@ -115,7 +126,7 @@ struct Workspace {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false) {
+Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false, bool bwd = false) {
   Workspace w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -127,6 +138,7 @@ Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false) {
   w.err = reinterpret_cast<uint32_t*>(take(256));
   w.qbar = reinterpret_cast<double*>(take(BH * s.Nq * s.D * sizeof(double)));
   w.kbar = reinterpret_cast<double*>(take(BH * s.Nk * s.D * sizeof(double)));
+  w.var = reinterpret_cast<double*>(take(BH * s.Nk * s.D * sizeof(double)));
   w.S = reinterpret_cast<double*>(take(BH * s.Nq * s.Nk * sizeof(double)));
   w.S32 = reinterpret_cast<float*>(w.S);
   w.nq = reinterpret_cast<float*>(take(BH * s.Nq * sizeof(float)));
@@ -138,6 +150,14 @@ Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false) {
   w.hst = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(s.LD) * 2));
   w.Hagg = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nq * static_cast<size_t>(s.D) * s.D * 2));
   w.Zagg = reinterpret_cast<float*>(take(BH * s.Nq * s.D * sizeof(float)));
+  if (bwd) {
+    w.wt_ld = (s.Nq + 63) / 64 * 64;
+    w.gs = reinterpret_cast<__nv_bfloat16*>(take(BH * s.N * static_cast<size_t>(s.D) * 2));
+    w.dHst = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nq * static_cast<size_t>(s.LD) * 2));
+    w.WT = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(w.wt_ld) * 2));
+    w.dh = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(s.D) * s.D * 2));
+    w.dz = reinterpret_cast<float*>(take(BH * s.Nk * s.D * sizeof(float)));
+  }
   if (fp8) {
     w.k8 = take(BH * s.N * static_cast<size_t>(s.D));
     w.v8 = take(BH * s.N * static_cast<size_t>(s.D));
@@ -148,10 +168,10 @@ Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false) {
   return w;
 }
 
-sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w, bool fp8 = false) {
+sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w, bool fp8 = false, bool bwd = false) {
   if (!ws) return fail(SLA_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(SLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  *w = layout(s, static_cast<uint8_t*>(ws), fp8);
+  *w = layout(s, static_cast<uint8_t*>(ws), fp8, bwd);
   if (ws_bytes < w->bytes)
     return fail(SLA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, w->bytes);
   return SLA_OK;
@@ -267,7 +287,7 @@ sla_status launch_pool(const void* x, double* out, const Shape& s, int block, in
 }
 
 // Fused precompute: query-block means (when qbar is set), KV-block means, z_j and h_j.
-template <int D>
+template <int D, int FM = 0>
 sla_status launch_prep(const void* q, const void* k, const void* v, const Shape& s, const sla::PrepArgs& args,
                        cudaStream_t st) {
   CUtensorMap mq, mk, mv, mh;
@@ -285,10 +305,10 @@ sla_status launch_prep(const void* q, const void* k, const void* v, const Shape&
     SLA_TRY(make_map(&mh, args.hst, 3, dims, strides, box));
   }
   constexpr int smem = sla::PrepSmem<D>::total();
-  SLA_TRY(allow_smem(sla::prep_kernel<D>, smem));
+  SLA_TRY(allow_smem(sla::prep_kernel<D, FM>, smem));
   const long long items = static_cast<long long>(s.BH) * s.Nk + (args.qbar ? static_cast<long long>(s.BH) * s.Nq : 0);
   const int grid = static_cast<int>(items < sm_count() ? items : sm_count());
-  sla::prep_kernel<D><<<grid, 576, smem, st>>>(mq, mk, mv, mh, args);
+  sla::prep_kernel<D, FM><<<grid, 576, smem, st>>>(mq, mk, mv, mh, args);
   return launched("prep_kernel");
 }
 
@@ -317,6 +337,9 @@ sla_status launch_cert(const CertArgs& a, cudaStream_t st) {
 // Rows of up to kCertMaxNk blocks are selected from fp32 scores with fp64 resolution of
 // the uncertain band (keys in registers); longer rows from fp64 scores in shared memory.
 constexpr int kCertMaxNk = 32 * 64;
+
+sla_status launch_select64(const Shape& s, const Workspace& w, const double* S, int8_t* mask, int32_t* crit,
+                           int crit_ld, __nv_bfloat16* W, cudaStream_t st);
 
 // Labels, critical lists and the marginal indicator from the pooled means in w.qbar and
 // w.kbar. scores64 (nullable) receives the fp64 scores whenever it is given.
@@ -351,6 +374,12 @@ sla_status launch_router(const Shape& s, const Workspace& w, double* scores64, i
   }
   double* S = scores64 ? scores64 : w.S;
   SLA_TRY(launch_scores<D>(w.qbar, w.kbar, S, s, st));
+  return launch_select64(s, w, S, mask, crit, crit_ld, W, st);
+}
+
+// Labels, critical lists and the marginal indicator from fp64 scores S [BH, Nq, Nk].
+sla_status launch_select64(const Shape& s, const Workspace& w, const double* S, int8_t* mask, int32_t* crit,
+                           int crit_ld, __nv_bfloat16* W, cudaStream_t st) {
   SelectArgs a{};
   a.S = S;
   a.rows = s.BH * s.Nq;
@@ -372,38 +401,49 @@ sla_status launch_router(const Shape& s, const Workspace& w, double* scores64, i
   return launch_dependent(sla::select_kernel, dim3(grid), dim3(wpc * 32), smem, st, "select_kernel", a);
 }
 
+// C[m, :] = sum_k A[m, k] Bst[k, :] per head (the aggregation GEMM): A [BH, M, a_ld] bf16 0/1,
+// Bst [BH, K, LD] bf16 stacked states, C split into its first D*D columns (bf16, Cd) and the
+// next D (fp32, Cz). Run forwards (A = W, M = Nq, K = Nk) and, for the backward, with the
+// indicator transposed (A = W^T, M = Nk, K = Nq).
 template <int D>
-sla_status launch_agg(const Shape& s, const Workspace& w, const float* alpha, cudaStream_t st) {
+sla_status launch_agg_gemm(int M, int K, int BH, int LD, const __nv_bfloat16* A, int a_ld, const __nv_bfloat16* Bst,
+                           __nv_bfloat16* Cd, float* Cz, uint32_t* err, const float* alpha, int H, int bh0,
+                           cudaStream_t st) {
   CUtensorMap mw, mh;
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
-    const uint64_t strides[2] = {static_cast<uint64_t>(s.w_ld), static_cast<uint64_t>(s.Nq) * s.w_ld};
+    const uint64_t dims[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(BH)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(a_ld), static_cast<uint64_t>(M) * a_ld};
     const uint32_t box[3] = {64, 128, 1};
-    SLA_TRY(make_map(&mw, w.W, 3, dims, strides, box));
+    SLA_TRY(make_map(&mw, A, 3, dims, strides, box));
   }
   {
-    const uint64_t dims[3] = {static_cast<uint64_t>(s.LD), static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.BH)};
-    const uint64_t strides[2] = {static_cast<uint64_t>(s.LD), static_cast<uint64_t>(s.Nk) * s.LD};
+    const uint64_t dims[3] = {static_cast<uint64_t>(LD), static_cast<uint64_t>(K), static_cast<uint64_t>(BH)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(LD), static_cast<uint64_t>(K) * LD};
     const uint32_t box[3] = {64, 64, 1};
-    SLA_TRY(make_map(&mh, w.hst, 3, dims, strides, box));
+    SLA_TRY(make_map(&mh, Bst, 3, dims, strides, box));
   }
   CUtensorMap mo;
   {
-    const uint64_t DD = static_cast<uint64_t>(s.D) * s.D;
-    const uint64_t dims[3] = {DD, static_cast<uint64_t>(s.Nq), static_cast<uint64_t>(s.BH)};
-    const uint64_t strides[2] = {DD, static_cast<uint64_t>(s.Nq) * DD};
+    const uint64_t DD = static_cast<uint64_t>(D) * D;
+    const uint64_t dims[3] = {DD, static_cast<uint64_t>(M), static_cast<uint64_t>(BH)};
+    const uint64_t strides[2] = {DD, static_cast<uint64_t>(M) * DD};
     const uint32_t box[3] = {64, 128, 1};
-    SLA_TRY(make_map(&mo, w.Hagg, 3, dims, strides, box));
+    SLA_TRY(make_map(&mo, Cd, 3, dims, strides, box));
   }
   const int smem = sla::kAggStages * sla::kAggStageBytes + sla::kAggStagingBytes + 1024;
   SLA_TRY(allow_smem(sla::agg_kernel<D>, smem));
-  AggArgs a{s.Nq, s.Nk, s.LD, s.BH, w.Hagg, w.Zagg, w.err, alpha, s.H};
-  const long long tiles = static_cast<long long>(s.LD / 128) * ((s.Nq + 255) / 256) * s.BH;
+  AggArgs a{M, K, LD, BH, Cd, Cz, err, alpha, H, bh0};
+  const long long tiles = static_cast<long long>(LD / 128) * ((M + 255) / 256) * BH;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   return launch_dependent(sla::agg_kernel<D>, dim3(grid), dim3(224), smem, st, "agg_kernel", mw, mh, mo, a);
 }
 
 template <int D>
+sla_status launch_agg(const Shape& s, const Workspace& w, const float* alpha, cudaStream_t st, int bh0 = 0) {
+  return launch_agg_gemm<D>(s.Nq, s.Nk, s.BH, s.LD, w.W, s.w_ld, w.hst, w.Hagg, w.Zagg, w.err, alpha, s.H, bh0, st);
+}
+
+template <int D, int FM = 0>
 sla_status launch_attn(const Shape& s, const void* q, const void* k, const void* v, const float* alpha, void* out,
                        const Workspace& w, int crit_ld, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mh, mo;
@@ -420,7 +460,7 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
     SLA_TRY(make_map(&mh, w.Hagg, 2, dims, strides, box));
   }
   constexpr int smem = sla::AttnSmem<D>::total();
-  SLA_TRY(allow_smem(sla::attn_kernel<D>, smem));
+  SLA_TRY(allow_smem(sla::attn_kernel<D, FM>, smem));
   AttnArgs a;
   a.H = s.H;
   a.N = s.N;
@@ -437,7 +477,8 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.err = w.err;
   // persistent: two CTAs per SM walk the tiles
   const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
-  return launch_dependent(sla::attn_kernel<D>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, mo, a);
+  return launch_dependent(sla::attn_kernel<D, FM>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, mo,
+                          a);
 }
 
 template <int D>
@@ -500,6 +541,181 @@ sla_status route_impl(const Shape& s, const void* q, const void* k, int8_t* mask
                           st);
 }
 
+// ------------------------------------------------------------------ backward
+
+sla_status backward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
+                         const int8_t* mask, const void* dO, float* dQ, float* dK, float* dV, float* dalpha,
+                         const Workspace& w, cudaStream_t st) {
+  constexpr int D = 128;
+  const size_t act_f32 = static_cast<size_t>(s.BH) * s.N * D * sizeof(float);
+  SLA_CUDA(cudaMemsetAsync(dK, 0, act_f32, st));
+  SLA_CUDA(cudaMemsetAsync(dV, 0, act_f32, st));
+  SLA_CUDA(cudaMemsetAsync(dalpha, 0, static_cast<size_t>(s.H) * D * sizeof(float), st));
+  // states, labels and H_i, Z_i as in the forward (H_i unscaled)
+  sla::PrepArgs pa{};
+  pa.BH = s.BH;
+  pa.N = s.N;
+  pa.Nq = s.Nq;
+  pa.Nk = s.Nk;
+  pa.block_q = s.bq;
+  pa.qbar = mask ? nullptr : w.qbar;
+  pa.kbar = mask ? nullptr : w.kbar;
+  pa.hst = w.hst;
+  pa.LD = s.LD;
+  pa.err = w.err;
+  SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
+  if (mask) {
+    MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
+    sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+    SLA_TRY(launched("mask_lists_kernel"));
+  } else {
+    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+  }
+  SLA_TRY(launch_agg<D>(s, w, nullptr, st));
+  // G_s = alpha dO
+  const size_t chunks = static_cast<size_t>(s.BH) * s.N * D / 8;
+  sla::gs_kernel<<<4 * sm_count(), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO), alpha, w.gs, s.H, s.N, D,
+                                                  chunks);
+  SLA_TRY(launched("gs_kernel"));
+  // per query tile: dQ, dalpha, dH_i / dZ_i, and the sparse branch's dK, dV
+  {
+    CUtensorMap mq, mg, mk, mv, mh;
+    SLA_TRY(act_map(&mq, q, s, 128));
+    SLA_TRY(act_map(&mg, w.gs, s, 128));
+    SLA_TRY(act_map(&mk, k, s, 64));
+    SLA_TRY(act_map(&mv, v, s, 64));
+    const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(s.BH) * s.Nq * D};
+    const uint64_t strides[1] = {static_cast<uint64_t>(D)};
+    const uint32_t box[2] = {64, 64};
+    SLA_TRY(make_map(&mh, w.Hagg, 2, dims, strides, box));
+    sla::BwdArgs a{};
+    a.H = s.H;
+    a.N = s.N;
+    a.Nq = s.Nq;
+    a.n_tiles = s.BH * s.Nq;
+    a.LD = s.LD;
+    a.crit = w.crit;
+    a.crit_ld = s.Nk;
+    a.crit_cnt = w.crit_cnt;
+    a.Zagg = w.Zagg;
+    a.alpha = alpha;
+    a.dO = static_cast<const __nv_bfloat16*>(dO);
+    a.dQ = dQ;
+    a.dK = dK;
+    a.dV = dV;
+    a.dalpha = dalpha;
+    a.dHst = w.dHst;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    a.err = w.err;
+    const int smem = 6 * 32768 + 1024;
+    SLA_TRY(allow_smem(sla::bwd_kernel, smem));
+    const int grid = a.n_tiles < sm_count() ? a.n_tiles : sm_count();
+    SLA_TRY(launch_dependent(sla::bwd_kernel, dim3(grid), dim3(192), smem, st, "bwd_kernel", mq, mg, mk, mv, mh, a));
+  }
+  // dh_j, dz_j = sums of dH_i, dZ_i over the rows i where j is marginal
+  sla::w_transpose_kernel<<<dim3((s.Nk + 31) / 32, w.wt_ld / 32, s.BH), dim3(32, 8), 0, st>>>(w.W, s.Nq, s.Nk, s.w_ld,
+                                                                                           w.WT, w.wt_ld);
+  SLA_TRY(launched("w_transpose_kernel"));
+  SLA_TRY(launch_agg_gemm<D>(s.Nk, s.Nq, s.BH, s.LD, w.WT, w.wt_ld, w.dHst, w.dh, w.dz, w.err, nullptr, s.H, 0, st));
+  // the states' part of dK, dV
+  {
+    CUtensorMap mk, mv, mdh;
+    SLA_TRY(act_map(&mk, k, s, 64));
+    SLA_TRY(act_map(&mv, v, s, 64));
+    const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(D), static_cast<uint64_t>(s.BH) * s.Nk};
+    const uint64_t strides[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(D) * D};
+    const uint32_t box[3] = {64, 128, 1};
+    SLA_TRY(make_map(&mdh, w.dh, 3, dims, strides, box));
+    sla::BwdStatesArgs a{s.BH, s.N, s.Nk, w.dz, dK, dV, w.err};
+    const int smem = 65536 + 1024;
+    SLA_TRY(allow_smem(sla::bwd_states_kernel, smem));
+    SLA_TRY(launch_dependent(sla::bwd_states_kernel, dim3(s.BH * s.Nk), dim3(192), smem, st, "bwd_states_kernel", mk,
+                             mv, mdh, a));
+  }
+  return SLA_OK;
+}
+
+// ------------------------------------------------------------------ variants (SPLA §2.1, §2.3)
+
+struct Variant {
+  int fm;      // feature map: 0 elu + 1, 1 e^x
+  int score2;  // block score: 0 first order, 1 second order
+};
+
+sla_status read_variant(const sla_variant* v, Variant* out) {
+  if (!v) return fail(SLA_ERR_INVALID_ARG, "variant is NULL");
+  if (v->feature_map != 0 && v->feature_map != 1)
+    return fail(SLA_ERR_INVALID_ARG, "feature_map must be 0 (elu + 1) or 1 (exp), got %d", v->feature_map);
+  if (v->block_score != 0 && v->block_score != 1)
+    return fail(SLA_ERR_INVALID_ARG, "block_score must be 0 (first order) or 1 (second order), got %d", v->block_score);
+  out->fm = v->feature_map;
+  out->score2 = v->block_score;
+  return SLA_OK;
+}
+
+template <int D>
+sla_status launch_block_var(const void* k, const Shape& s, const Workspace& w, cudaStream_t st) {
+  sla::block_var_kernel<D><<<dim3(s.Nk, s.BH), 128, 0, st>>>(static_cast<const __nv_bfloat16*>(k), w.kbar, w.var, s.N);
+  return launched("block_var_kernel");
+}
+
+template <int D>
+sla_status launch_score2(const Shape& s, const Workspace& w, double* S2, cudaStream_t st) {
+  sla::score2_kernel<D><<<dim3((s.Nk + 31) / 32, (s.Nq + 31) / 32, s.BH), 256, 0, st>>>(w.qbar, w.kbar, w.var, S2,
+                                                                                           s.Nq, s.Nk);
+  return launched("score2_kernel");
+}
+
+// Second-order labels from w.qbar (already pooled) and K: block means and variances, S2,
+// the fp64 selection. S2 goes to scores64 when given, else to the workspace.
+template <int D>
+sla_status route_second_order(const Shape& s, const void* k, const Workspace& w, double* scores64, int8_t* mask,
+                              int32_t* crit, int crit_ld, __nv_bfloat16* W, cudaStream_t st) {
+  SLA_TRY(launch_block_var<D>(k, s, w, st));
+  double* S2 = scores64 ? scores64 : w.S;
+  SLA_TRY(launch_score2<D>(s, w, S2, st));
+  return launch_select64(s, w, S2, mask, crit, crit_ld, W, st);
+}
+
+template <int D>
+sla_status route_variant_impl(const Shape& s, const Variant& var, const void* q, const void* k, int8_t* mask_out,
+                              int32_t* crit_out, double* scores_out, const Workspace& w, cudaStream_t st) {
+  if (!var.score2) return route_impl<D>(s, q, k, mask_out, crit_out, scores_out, w, st);
+  SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
+  return route_second_order<D>(s, k, w, scores_out, mask_out, crit_out ? crit_out : w.crit, crit_out ? s.kc : s.Nk,
+                               nullptr, st);
+}
+
+// The forward with a variant: one launch per stage over every head.
+template <int D, int FM>
+sla_status forward_variant_impl(const Shape& s, const Variant& var, const void* q, const void* k, const void* v,
+                                const float* alpha, const int8_t* mask, void* out, const Workspace& w,
+                                cudaStream_t st) {
+  sla::PrepArgs pa{};
+  pa.BH = s.BH;
+  pa.N = s.N;
+  pa.Nq = s.Nq;
+  pa.Nk = s.Nk;
+  pa.block_q = s.bq;
+  pa.qbar = mask ? nullptr : w.qbar;
+  pa.kbar = mask ? nullptr : w.kbar;
+  pa.hst = w.hst;
+  pa.LD = s.LD;
+  pa.err = w.err;
+  SLA_TRY((launch_prep<D, FM>(q, k, v, s, pa, st)));
+  if (mask) {
+    MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
+    sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+    SLA_TRY(launched("mask_lists_kernel"));
+  } else if (var.score2) {
+    SLA_TRY(route_second_order<D>(s, k, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+  } else {
+    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+  }
+  SLA_TRY(launch_agg<D>(s, w, alpha, st));
+  return launch_attn<D, FM>(s, q, k, v, alpha, out, w, s.Nk, st);
+}
+
 // Stage boundaries for sla_forward_timed: ev[0] before the per-block precompute,
 // ev[1] after it, ev[2] after routing, ev[3] after aggregation, ev[4] after attention.
 // sla_forward_fp8_timed: ev[4] after the K/V quantiser, ev[5] after attention.
@@ -513,6 +729,41 @@ struct StageEvents {
     return SLA_OK;
   }
 };
+
+// The forward's per-head pieces of the workspace for heads h0, h0 + 1, ... (every piece is
+// head-major), except the per-block states: a group of heads always writes them at the start
+// of their buffer, so every group reuses the same lines of L2.
+Workspace group_view(const Workspace& w, const Shape& s, int h0) {
+  const size_t h = static_cast<size_t>(h0);
+  Workspace o = w;
+  o.qbar = w.qbar + h * s.Nq * s.D;
+  o.kbar = w.kbar + h * s.Nk * s.D;
+  o.S = w.S + h * s.Nq * s.Nk;
+  o.S32 = w.S32 + h * s.Nq * s.Nk;
+  o.nq = w.nq + h * s.Nq;
+  o.nk = w.nk + h * s.Nk;
+  o.mask = w.mask + h * s.Nq * s.Nk;
+  o.crit = w.crit + h * s.Nq * s.Nk;
+  o.crit_cnt = w.crit_cnt + h * s.Nq;
+  o.W = w.W + h * s.Nq * s.w_ld;
+  o.Hagg = w.Hagg + h * s.Nq * static_cast<size_t>(s.D) * s.D;
+  o.Zagg = w.Zagg + h * s.Nq * s.D;
+  return o;
+}
+
+// Heads per group of the grouped precompute -> route -> aggregation: as many as keep a
+// group's bf16 per-block states within kGroupStateBytes of L2 (so the aggregation reads them
+// from L2 right after the precompute wrote them), and no more than kMaxGroups groups.
+constexpr size_t kGroupStateBytes = size_t(48) << 20;
+constexpr int kMaxGroups = 16;
+int heads_per_group(const Shape& s) {
+  const size_t per_head = static_cast<size_t>(s.Nk) * s.LD * 2;
+  int g = static_cast<int>(kGroupStateBytes / per_head);
+  const int min_g = (s.BH + kMaxGroups - 1) / kMaxGroups;
+  if (g < min_g) g = min_g;
+  if (g < 1) g = 1;
+  return g > s.BH ? s.BH : g;
+}
 
 template <int D>
 sla_status forward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
@@ -529,23 +780,52 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
   pa.hst = w.hst;
   pa.LD = s.LD;
   pa.err = w.err;
-  SLA_TRY(ev.mark(0, st));
-  if (mask) {
-    SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
-    SLA_TRY(ev.mark(1, st));
-    MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
-    sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
-    SLA_TRY(launched("mask_lists_kernel"));
-  } else {
-    SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
-    SLA_TRY(ev.mark(1, st));
-    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
-  }
-  SLA_TRY(ev.mark(2, st));
   // the bf16 attention adds the linear branch into its accumulator and takes H_i scaled per
   // channel by (1 - alpha) / alpha; the low-bit kernel takes H_i as it is
-  SLA_TRY(launch_agg<D>(s, w, fp8 ? nullptr : alpha, st));
-  SLA_TRY(ev.mark(3, st));
+  const float* agg_alpha = fp8 ? nullptr : alpha;
+  const int G = heads_per_group(s);
+  SLA_TRY(ev.mark(0, st));
+  if (ev.on || G >= s.BH) {
+    // One launch of each stage over every head (the timed entry point reports the stages
+    // separately this way).
+    SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
+    SLA_TRY(ev.mark(1, st));
+    if (mask) {
+      MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
+      sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+      SLA_TRY(launched("mask_lists_kernel"));
+    } else {
+      SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+    }
+    SLA_TRY(ev.mark(2, st));
+    SLA_TRY(launch_agg<D>(s, w, agg_alpha, st));
+    SLA_TRY(ev.mark(3, st));
+  } else {
+    // Groups of G heads: each group's states stay in L2 between its precompute and its
+    // aggregation, and the next group overwrites the same lines.
+    const size_t per_head = static_cast<size_t>(s.N) * s.D;
+    for (int h0 = 0; h0 < s.BH; h0 += G) {
+      Shape sg = s;
+      sg.BH = s.BH - h0 < G ? s.BH - h0 : G;
+      const Workspace wg = group_view(w, s, h0);
+      sla::PrepArgs pg = pa;
+      pg.BH = sg.BH;
+      pg.qbar = mask ? nullptr : wg.qbar;
+      pg.kbar = mask ? nullptr : wg.kbar;
+      const size_t off = static_cast<size_t>(h0) * per_head;
+      SLA_TRY(launch_prep<D>(static_cast<const __nv_bfloat16*>(q) + off, static_cast<const __nv_bfloat16*>(k) + off,
+                             static_cast<const __nv_bfloat16*>(v) + off, sg, pg, st));
+      if (mask) {
+        MaskListArgs m{mask + static_cast<size_t>(h0) * s.Nq * s.Nk, sg.BH * s.Nq, s.Nk, wg.crit, s.Nk,
+                       wg.crit_cnt, wg.W, s.w_ld, w.err};
+        sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+        SLA_TRY(launched("mask_lists_kernel"));
+      } else {
+        SLA_TRY(launch_router<D>(sg, wg, nullptr, wg.mask, wg.crit, s.Nk, wg.W, st));
+      }
+      SLA_TRY(launch_agg<D>(sg, wg, agg_alpha, st, h0));
+    }
+  }
   if (fp8) {
     if constexpr (D == 128) {
       SLA_TRY(launch_quant<D>(s, k, v, w.k8, w.v8, w.kexp, w.vexp, st, true));
@@ -739,6 +1019,118 @@ sla_status sla_quantize_kv(const sla_problem* p, const void* k, const void* v, u
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.D == 64) return launch_quant<64>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st, false);
   return launch_quant<128>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st, false);
+}
+
+sla_status sla_aggregate_states(const sla_problem* p, const void* k, const void* v, const int8_t* mask,
+                                void* H_out, float* Z_out, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(k) || !aligned16(v)) return fail(SLA_ERR_INVALID_ARG, "k and v must be non-NULL and 16-byte aligned");
+  if (!mask) return fail(SLA_ERR_INVALID_ARG, "mask is NULL");
+  if (!aligned16(H_out) || !aligned16(Z_out))
+    return fail(SLA_ERR_INVALID_ARG, "H_out and Z_out must be non-NULL and 16-byte aligned");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  w.Hagg = static_cast<__nv_bfloat16*>(H_out);
+  w.Zagg = Z_out;
+  sla::PrepArgs pa{};
+  pa.BH = s.BH;
+  pa.N = s.N;
+  pa.Nq = s.Nq;
+  pa.Nk = s.Nk;
+  pa.block_q = s.bq;
+  pa.hst = w.hst;
+  pa.LD = s.LD;
+  pa.err = w.err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
+  if (s.D == 64) {
+    SLA_TRY(launch_prep<64>(nullptr, k, v, s, pa, st));
+  } else {
+    SLA_TRY(launch_prep<128>(nullptr, k, v, s, pa, st));
+  }
+  sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+  SLA_TRY(launched("mask_lists_kernel"));
+  if (s.D == 64) return launch_agg<64>(s, w, nullptr, st);
+  return launch_agg<128>(s, w, nullptr, st);
+}
+
+int sla_forward_launches(const sla_problem* p, int with_mask, int low_bit) {
+  Shape s;
+  if (make_shape(p, &s) != SLA_OK) return -1;
+  const int per_group = 1 + (with_mask ? 1 : 2) + 1;  // precompute, labels (router: scores + selection), aggregation
+  const int G = heads_per_group(s);
+  const int groups = G >= s.BH ? 1 : (s.BH + G - 1) / G;
+  return groups * per_group + 1 + (low_bit ? 1 : 0);  // + attention (+ the K/V quantiser)
+}
+
+sla_status sla_route_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
+                             int8_t* mask_out, int32_t* crit_idx_out, double* scores_out, void* ws, size_t ws_bytes,
+                             void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  Variant var;
+  SLA_TRY(read_variant(variant, &var));
+  if (!aligned16(q) || !aligned16(k)) return fail(SLA_ERR_INVALID_ARG, "q and k must be non-NULL and 16-byte aligned");
+  if (!mask_out) return fail(SLA_ERR_INVALID_ARG, "mask_out is NULL");
+  if (crit_idx_out && (reinterpret_cast<uintptr_t>(crit_idx_out) % 4))
+    return fail(SLA_ERR_INVALID_ARG, "crit_idx_out must be 4-byte aligned");
+  if (scores_out && (reinterpret_cast<uintptr_t>(scores_out) % 8))
+    return fail(SLA_ERR_INVALID_ARG, "scores_out must be 8-byte aligned");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) return route_variant_impl<64>(s, var, q, k, mask_out, crit_idx_out, scores_out, w, st);
+  return route_variant_impl<128>(s, var, q, k, mask_out, crit_idx_out, scores_out, w, st);
+}
+
+sla_status sla_forward_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
+                               const void* v, const float* alpha, const int8_t* mask, void* out, void* ws,
+                               size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  Variant var;
+  SLA_TRY(read_variant(variant, &var));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SLA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
+  if (!alpha || reinterpret_cast<uintptr_t>(alpha) % 4) return fail(SLA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
+  const size_t act = static_cast<size_t>(s.BH) * s.N * s.D * 2;
+  if (overlaps(out, q, act) || overlaps(out, k, act) || overlaps(out, v, act))
+    return fail(SLA_ERR_INVALID_ARG, "out must not alias q, k or v");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) {
+    if (var.fm) return forward_variant_impl<64, 1>(s, var, q, k, v, alpha, mask, out, w, st);
+    return forward_variant_impl<64, 0>(s, var, q, k, v, alpha, mask, out, w, st);
+  }
+  if (var.fm) return forward_variant_impl<128, 1>(s, var, q, k, v, alpha, mask, out, w, st);
+  return forward_variant_impl<128, 0>(s, var, q, k, v, alpha, mask, out, w, st);
+}
+
+size_t sla_workspace_size_backward(const sla_problem* p) {
+  Shape s;
+  if (make_shape(p, &s) != SLA_OK) return 0;
+  return layout(s, nullptr, false, true).bytes;
+}
+
+sla_status sla_backward(const sla_problem* p, const void* q, const void* k, const void* v, const float* alpha,
+                        const int8_t* mask, const void* dO, float* dQ, float* dK, float* dV, float* dalpha, void* ws,
+                        size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (s.D != 128) return fail(SLA_ERR_UNSUPPORTED, "the backward needs D=128 (got %d)", s.D);
+  if (s.bq != 128) return fail(SLA_ERR_UNSUPPORTED, "the backward needs block_q=128 (got %d)", s.bq);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO))
+    return fail(SLA_ERR_INVALID_ARG, "q, k, v and dO must be non-NULL and 16-byte aligned");
+  if (!aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return fail(SLA_ERR_INVALID_ARG, "dQ, dK and dV must be non-NULL and 16-byte aligned");
+  if (!alpha || reinterpret_cast<uintptr_t>(alpha) % 4) return fail(SLA_ERR_INVALID_ARG, "alpha must be 4-byte aligned");
+  if (!dalpha || reinterpret_cast<uintptr_t>(dalpha) % 4)
+    return fail(SLA_ERR_INVALID_ARG, "dalpha must be non-NULL and 4-byte aligned");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w, false, true));
+  return backward_impl(s, q, k, v, alpha, mask, dO, dQ, dK, dV, dalpha, w, static_cast<cudaStream_t>(stream));
 }
 
 sla_status sla_check(void* ws, void* stream) {

@@ -25,7 +25,7 @@ def _declared_symbols():
     for path in os.listdir(os.path.join(ROOT, "include")):
         if path.endswith(".h"):
             text = open(os.path.join(ROOT, "include", path)).read()
-            names |= set(re.findall(r"^\s*(?:sla_status|size_t|const char\*)\s+(sla_\w+)\s*\(", text, re.M))
+            names |= set(re.findall(r"^\s*(?:sla_status|size_t|int|const char\*)\s+(sla_\w+)\s*\(", text, re.M))
     return names
 
 
@@ -160,3 +160,62 @@ def test_route_noalloc_refuses_oversize_problem(lib):
     assert "maximum" in lib.sla_last_error().decode()
     # the same problem with both outputs given by the caller still needs more than the array holds
     assert fn(ctypes.byref(p), fake, fake, fake, fake, ctypes.c_void_p(2 << 20), null) == 3
+
+
+def test_forward_launch_counts(lib):
+    """Groups of heads for the precompute, labels and aggregation: as many heads as keep a
+    group's bf16 per-block states within 48 MiB, at most 16 groups; four launches per group
+    (three with a caller mask) plus the attention (and the quantiser for the low-bit call)."""
+    # Wan2.1-1.3B shape: 512 blocks x (128*128 + 128) bf16 = 16.9 MB of states per head -> 2 heads
+    p = binding.problem(1, 12, 32760, 128, 128, 64, 0.05, 0.1)
+    assert binding.forward_launches(p) == 6 * 4 + 1
+    assert binding.forward_launches(p, with_mask=True) == 6 * 3 + 1
+    assert binding.forward_launches(p, low_bit=True) == 6 * 4 + 2
+    # small problem: one group
+    assert binding.forward_launches(binding.problem(1, 2, 1024, 64, 64, 64, 0.25, 0.25)) == 5
+    # Wan2.1-14B 720p: 39 MB per head -> 1 head, but at most 16 groups -> 5 heads per group
+    assert binding.forward_launches(binding.problem(2, 40, 75600, 128, 128, 64, 0.05, 0.15)) == 16 * 4 + 1
+    assert lib.sla_forward_launches(ctypes.byref(binding.problem(1, 1, 64, 96, 64, 64, 0.1, 0.1)), 0, 0) == -1
+
+
+def test_aggregate_states_host_checks(lib):
+    p = binding.problem(1, 1, 128, 64, 64, 64, 0.25, 0.25)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(16 << 20)
+    size = binding.workspace_size(p)
+    assert lib.sla_aggregate_states(ctypes.byref(p), fake, fake, null, fake, fake, ws, size, null) == 1  # no mask
+    assert lib.sla_aggregate_states(ctypes.byref(p), fake, fake, fake, ctypes.c_void_p((1 << 20) + 8), fake, ws,
+                                    size, null) == 1  # H_out misaligned
+    assert lib.sla_aggregate_states(ctypes.byref(p), fake, fake, fake, fake, fake, ws, size - 1, null) == 3
+
+
+def test_variant_entry_points_reject_bad_variants(lib):
+    p = binding.problem(1, 1, 128, 64, 64, 64, 0.25, 0.25)
+    fake = ctypes.c_void_p(1 << 20)
+    null = ctypes.c_void_p(0)
+    ws = ctypes.c_void_p(16 << 20)
+    size = binding.workspace_size(p)
+    for bad in (binding.Variant(2, 0), binding.Variant(0, -1)):
+        assert lib.sla_route_variant(ctypes.byref(p), ctypes.byref(bad), fake, fake, fake, null, null, ws, size,
+                                     null) == 1
+        assert lib.sla_forward_variant(ctypes.byref(p), ctypes.byref(bad), fake, fake, fake, fake, null,
+                                       ctypes.c_void_p(8 << 20), ws, size, null) == 1
+    assert lib.sla_route_variant(ctypes.byref(p), None, fake, fake, fake, null, null, ws, size, null) == 1
+
+
+def test_backward_host_checks(lib):
+    p = binding.problem(1, 1, 256, 128, 128, 64, 0.25, 0.25)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(32 << 20)
+    size = lib.sla_workspace_size_backward(ctypes.byref(p))
+    assert size > binding.workspace_size(p)
+    # only calls the host rejects before any CUDA call (unsupported shape, NULL pointer, small workspace)
+    args = [fake, fake, fake, fake, null, fake, fake, fake, fake, fake]
+    p64 = binding.problem(1, 1, 256, 64, 64, 64, 0.25, 0.25)
+    assert lib.sla_backward(ctypes.byref(p64), *args, ws, size, null) == 2
+    pbq = binding.problem(1, 1, 256, 128, 64, 64, 0.25, 0.25)
+    assert lib.sla_backward(ctypes.byref(pbq), *args, ws, size, null) == 2
+    assert lib.sla_backward(ctypes.byref(p), null, *args[1:], ws, size, null) == 1
+    assert lib.sla_backward(ctypes.byref(p), *args, ws, size - 1, null) == 3

@@ -107,7 +107,7 @@ def test_kv_states_match_oracle(cuda_device):
         h, z = binding.kv_states(k, v)
         kc_, vc = _to_cpu(k, v)
         rh, rz = oracle.kv_states(kc_, vc, 64)
-        # phi(k) enters the tensor core in bf16 (relative rounding 2^-9) with fp32 accumulation
+        # phi(k) enters the tensor core in bf16 (relative rounding 2^-8) with fp32 accumulation
         scale_h = np.abs(rh).max()
         assert np.abs(h.cpu().numpy() - rh).max() <= 8e-3 * scale_h
         np.testing.assert_allclose(z.cpu().numpy(), rz, rtol=1e-5, atol=1e-4)
@@ -278,3 +278,46 @@ def test_long_rows_use_the_fp64_selection(cuda_device):
     qb = [0, 1, Nq // 2, Nq - 1]
     ref = _oracle_rows(q, k, v, alpha, bq, mask, [(0, 0)], query_blocks=qb)
     assert_outputs_close(out_ext.float().cpu().numpy(), ref, "long rows")
+
+
+@pytest.mark.parametrize("B, H, N, D, bq, kh, kl", [(1, 2, 1000, 128, 128, 0.2, 0.3), (2, 1, 333, 64, 64, 0.25, 0.25),
+                                                     (1, 3, 4113, 128, 128, 0.0, 0.0)])
+def test_aggregate_states_match_oracle(cuda_device, B, H, N, D, bq, kh, kl):
+    """H_i, Z_i after the aggregation against the oracle's sums over the marginal blocks.
+
+    Bound per entry: phi(k) enters the tensor core in bf16, h_j and z_j are stored in bf16 and
+    H_i is rounded to bf16 (three roundings, each at most 2^-8 relative: bf16 carries 8
+    significant bits); the sums accumulate in fp32. So |H - H_ref| <= 3 * 2^-8 * sum over
+    marginal j of (phi(K_j)^T |V_j|) and |Z - Z_ref| <= 2^-8 * Z_ref (phi > 0), plus fp32
+    slack."""
+    q, k, v, _ = random_inputs(B, H, N, D, seed=N + D, device=cuda_device)
+    mask, _, _ = binding.route(q, k, bq, 64, kh, kl)
+    Hs, Zs, ws = binding.aggregate_states(k, v, mask, bq)
+    binding.check(ws)
+    kc_, vc = _to_cpu(k, v)
+    h, z = oracle.kv_states(kc_, vc, 64)
+    h_abs, _ = oracle.kv_states(kc_, vc.abs(), 64)
+    m = mask.cpu().numpy()
+    Hg, Zg = Hs.float().cpu().numpy(), Zs.cpu().numpy()
+    for b in range(B):
+        for hh in range(H):
+            Hr, Zr = oracle.marginal_sums(m[b, hh], h[b, hh], z[b, hh])
+            Ha, _ = oracle.marginal_sums(m[b, hh], h_abs[b, hh], z[b, hh])
+            tol_h = 3 * 2.0 ** -8 * Ha + 1e-6 * (Ha.max() + 1)
+            assert np.all(np.abs(Hg[b, hh] - Hr) <= tol_h), float((np.abs(Hg[b, hh] - Hr) - tol_h).max())
+            np.testing.assert_allclose(Zg[b, hh], Zr, rtol=2.0 ** -8 + 1e-6, atol=1e-5)
+    if kh == 0 and kl == 0:  # every block marginal: H_i is the sum over all blocks for every row
+        assert np.allclose(Hg[0, 0, 0], Hg[0, 0, -1]) and np.allclose(Zg[0, 0, 0], Zg[0, 0, -1])
+
+
+def test_alpha_at_zero_and_one(cuda_device):
+    """Channels with alpha exactly 0 (linear branch only) and 1 (sparse branch only) next to
+    ordinary ones: the fused blend floors alpha at 2^-24, which stays within the tolerances."""
+    B, H, N, D, bq, kh, kl = 1, 2, 1000, 128, 128, 0.25, 0.25
+    q, k, v, alpha = random_inputs(B, H, N, D, seed=77, device=cuda_device)
+    alpha[:, 0::4] = 0.0
+    alpha[:, 1::4] = 1.0
+    gmask, omask, nmis = _route_parity(q, k, bq, kh, kl)
+    out = binding.forward(q, k, v, alpha, bq, 64, kh, kl, mask=omask)
+    ref = _oracle_rows(q, k, v, alpha, bq, omask, [(0, 0), (0, 1)])
+    assert_outputs_close(out.float().cpu().numpy(), ref, "alpha in {0, 1}")
