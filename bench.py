@@ -51,6 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the low-bit (e4m3) sparse-branch measurement")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-configuration table (the other workloads, the kh sweep and its tail)")
     ap.add_argument("--config-steps", type=int, default=10, help="timed calls per configuration of that table")
@@ -105,8 +106,12 @@ def algorithmic_work(w, mask):
     f_elem = 3.0 * N * D * BH
     f_alg = f_sparse + f_states + f_apply + f_agg + f_router + f_elem
     bytes_alg = 8.0 * N * D * BH + Nq * Nk * BH + H * D * 4
+    # backward with the labels fixed: five products per critical pair (S recomputed, dP, dV, dQ,
+    # dK), four D x D products per row in the linear branch (G H^T, u^T G, phi(K) dh, V dh^T),
+    # the transposed aggregation, and the row terms
+    f_bwd = 2.5 * f_sparse + 4.0 * N * D * D * BH + f_agg + 8.0 * N * D * BH
     return {"flops": f_alg, "bytes": bytes_alg, "f_sparse": f_sparse, "f_attn_kernel": f_sparse + f_apply,
-            "f_states": f_states, "f_agg": f_agg, "f_router": f_router}
+            "f_states": f_states, "f_agg": f_agg, "f_router": f_router, "f_bwd": f_bwd}
 
 
 def max_over_ranks(x, dist=None, device="cpu"):
@@ -537,6 +542,34 @@ def run_ours(args):
                "timed_calls": n_f}
         del wsf
 
+    # the backward (dQ, dK, dV, dalpha with the forward's labels held fixed), same timing rules
+    bwd = None
+    if not args.no_bwd and w.D == 128 and w.block_q == 128:
+        mask_b = binding.route(q, k, w.block_q, w.block_kv, w.kh, w.kl)[0]
+        g = torch.Generator(device=dev).manual_seed(1234)
+        dO = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        wsb, times = None, []
+        n_b = min(args.steps, 10)
+        for it in range(3 + n_b):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            _, _, _, _, wsb = binding.backward(q, k, v, alpha, dO, w.block_q, w.block_kv, w.kh, w.kl, mask=mask_b,
+                                               ws=wsb)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        binding.check(wsb)
+        ms_b = rank_max(sum(times) / len(times))
+        f_b = work["f_bwd"]
+        ach_b = f_b / (ms_b * 1e-3) / 1e12
+        bwd = {"call": "sla_backward", "ms_per_call": round(ms_b, 4), "algorithmic_tflop": round(f_b / 1e12, 4),
+               "achieved_tflops": round(ach_b, 2), "frac_of_bf16_peak": round(ach_b / peaks["bf16_tflops"], 4),
+               "peak_source": "measured bf16 burst", "labels": "the router's, held fixed", "dO": "seeded normal",
+               "timed_calls": n_b, "ratio_to_forward": round(ms_b / ms_step, 3)}
+        del wsb, dO
+
     # the other configurations: one table, same timing rules (c3 stays the headline value)
     configs = None
     if not args.no_configs:
@@ -568,12 +601,11 @@ def run_ours(args):
         "stage_ms": {"precompute": round(stage_ms[0], 4), "route": round(stage_ms[1], 4),
                      "aggregate": round(stage_ms[2], 4), "attention": round(stage_ms[3], 4),
                      "sum": round(sum(stage_ms), 4),
-                     "how": "sla_forward_timed after the timed loop: each stage as one launch over every head, "
-                            "timed alone (sla_forward itself runs precompute, labels and aggregation in groups of "
-                            "heads whose states stay in L2)"},
+                     "how": "sla_forward_timed after the timed loop: events between the stages of the same "
+                            "launches sla_forward makes"},
         "roofline": roofline, "path_roofline": path_roofline,
         "clocks": clock_info, "e2e": e2e, "gpu_launches": binding.forward_launches(p) * args.steps,
-        "dense_reference": dense, "low_bit": low, "configs": configs, "cpu_baseline": cpu,
+        "dense_reference": dense, "low_bit": low, "backward": bwd, "configs": configs, "cpu_baseline": cpu,
         "wall_s_timed": round(wall, 3),
     }
     print(json.dumps(line), flush=True)

@@ -113,10 +113,8 @@ sla_status sla_forward(const sla_problem* p, const void* q, const void* k, const
  * between the stages, waits for the last one, and writes stage_ms[4] (host):
  * [0] per-block precompute (pooling, KV states), [1] routing (scores and
  * selection, or the caller-mask lists), [2] marginal-state aggregation,
- * [3] fused attention. Each stage runs as one launch over every head here, so
- * that it can be timed alone; sla_forward runs the first three in groups of
- * heads (see sla_forward_launches), with the same results. Synchronises the
- * stream; meant for measurement. */
+ * [3] fused attention. The launches are those of sla_forward, with the same
+ * results. Synchronises the stream; meant for measurement. */
 sla_status sla_forward_timed(const sla_problem* p, const void* q, const void* k, const void* v,
                              const float* alpha, const int8_t* mask, void* out, void* ws,
                              size_t ws_bytes, void* stream, float* stage_ms);
@@ -185,9 +183,10 @@ sla_status sla_aggregate_states(const sla_problem* p, const void* k, const void*
                                 void* H_out, float* Z_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernel launches sla_forward (low_bit = 0) or sla_forward_fp8 (low_bit = 1)
- * enqueues for this problem, with (with_mask = 1) or without a caller mask: the precompute,
- * labels and aggregation run in groups of heads sized so that a group's per-block states
- * stay in L2. Host only; -1 for an invalid problem. For measurement. */
+ * enqueues for this problem, with (with_mask = 1) or without a caller mask: one per stage
+ * (precompute; labels: the caller mask's lists, or the router's scores and selection;
+ * aggregation; the K/V quantiser for low_bit; attention). Host only; -1 for an invalid
+ * problem. For measurement. */
 int sla_forward_launches(const sla_problem* p, int with_mask, int low_bit);
 
 /* ---------------------------------------------------------------- backward
@@ -254,6 +253,46 @@ sla_status sla_route_variant(const sla_problem* p, const sla_variant* variant, c
 sla_status sla_forward_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
                                const void* v, const float* alpha, const int8_t* mask, void* out, void* ws,
                                size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- PISA
+ *
+ * "PISA - Atención Dispersa por Tramos para Transformers de Difusión Eficientes" §2: the
+ * blocks that are not critical stay inside the softmax through a Taylor expansion of their
+ * exponentials around the block's centroid, in the numerator and the denominator. Per query
+ * token t of query block i with critical set S_i and the other blocks U_i:
+ *   o_t = N_t / D_t
+ *   N_t = sum_{j in S_i} sum_n e^{s_tn} v_n + sum_{j in U_i} a_tj Vsum_j
+ *         + (q_t / sqrt(D)) Hbar sum_{j in U_i} a_tj
+ *   D_t = sum_{j in S_i} sum_n e^{s_tn} + sum_{j in U_i} a_tj n_j
+ * s_tn = q_t . k_n / sqrt(D), a_tj = e^{q_t . kbar_j / sqrt(D)}, kbar_j the mean of block
+ * j's valid keys, n_j their count, Vsum_j the sum of its value rows, Hbar the mean over all
+ * KV blocks of H_j = sum_n (k_n - kbar_j) v_n^T. Readings: every exponent carries 1 / sqrt(D)
+ * (the first-order term's q_t / sqrt(D) follows); the denominator keeps the zero-order term
+ * (the first-order one sums to zero); the critical sets are SLA's (label 2), every other
+ * block is in U_i; the covariance-aware top-k the page mentions is not built. No alpha.
+ * Precision: the critical blocks as sla_forward; kbar_j and Vsum_j enter the tensor cores
+ * in bf16, Hbar in bf16 (summed in fp32 in a fixed order), the first-order operand
+ * (sum_j a_tj / sqrt(D)) q_t in bf16. */
+
+/* Workspace bytes for sla_forward_pisa and sla_pisa_hbar (0 for an invalid problem). */
+size_t sla_workspace_size_pisa(const sla_problem* p);
+
+/* The PISA output.
+ *   q, k, v   [B,H,N,D] bf16 device, 16-byte aligned
+ *   labels    [B,H,Nq,Nk] int8 device (nullable): the critical blocks are those labelled 2,
+ *             labels outside {0, 1, 2} are reported by sla_check; NULL runs the router
+ *             with p->kh, p->kl
+ *   out       [B,H,N,D] bf16 device, 16-byte aligned, not aliasing q, k or v
+ *   ws        workspace of sla_workspace_size_pisa(p) bytes
+ * Asynchronous on the stream; writes nothing on an argument error. */
+sla_status sla_forward_pisa(const sla_problem* p, const void* q, const void* k, const void* v, const int8_t* labels,
+                            void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Hbar of every head, [B,H,D,D] fp32 device (row d: key channel, column e: value channel),
+ * as the PISA forward computes it before rounding it to bf16. k, v as for sla_forward_pisa;
+ * ws of sla_workspace_size_pisa(p) bytes. For tests and inspection. */
+sla_status sla_pisa_hbar(const sla_problem* p, const void* k, const void* v, float* hbar_out, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /* Synchronise the stream, read and clear the workspace's device error word.
  * Returns SLA_OK, SLA_ERR_TIMEOUT or SLA_ERR_BAD_MASK (or SLA_ERR_CUDA). */

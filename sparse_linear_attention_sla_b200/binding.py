@@ -30,7 +30,8 @@ EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sl
            "sla_forward_timed", "sla_check", "sla_last_error", "sla_version", "sla_route_noalloc",
            "sla_selftest_wait_timeout", "sla_workspace_size_fp8", "sla_forward_fp8", "sla_forward_fp8_timed",
            "sla_quantize_kv", "sla_aggregate_states", "sla_forward_launches", "sla_route_variant",
-           "sla_forward_variant", "sla_workspace_size_backward", "sla_backward")
+           "sla_forward_variant", "sla_workspace_size_backward", "sla_backward", "sla_workspace_size_pisa",
+           "sla_forward_pisa", "sla_pisa_hbar")
 
 
 class SlaError(RuntimeError):
@@ -87,6 +88,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_workspace_size_backward.argtypes = [P]
         lib.sla_workspace_size_backward.restype = sz
         lib.sla_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_workspace_size_pisa.argtypes = [P]
+        lib.sla_workspace_size_pisa.restype = sz
+        lib.sla_forward_pisa.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        lib.sla_pisa_hbar.argtypes = [P, vp, vp, vp, vp, sz, vp]
         V = ctypes.POINTER(Variant)
         lib.sla_route_variant.argtypes = [P, V, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_forward_variant.argtypes = [P, V, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -95,7 +100,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_last_error.restype = ctypes.c_char_p
         lib.sla_version.restype = ctypes.c_char_p
         for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check",
-                     "sla_forward_fp8", "sla_forward_fp8_timed", "sla_quantize_kv"):
+                     "sla_forward_fp8", "sla_forward_fp8_timed", "sla_quantize_kv", "sla_forward_pisa",
+                     "sla_pisa_hbar", "sla_aggregate_states", "sla_backward", "sla_route_variant",
+                     "sla_forward_variant"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -287,6 +294,57 @@ def backward(q, k, v, alpha, dO, block_q=128, block_kv=64, kh=0.05, kl=0.10, mas
                               _stream_handle(dev))
     _raise(st)
     return dQ, dK, dV, dalpha, ws
+
+
+def new_workspace_pisa(p: Problem, device) -> torch.Tensor:
+    """A zero-headed workspace of sla_workspace_size_pisa(p) bytes on device."""
+    n = int(load_library().sla_workspace_size_pisa(ctypes.byref(p)))
+    if n == 0:
+        counts(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def forward_pisa(q, k, v, block_q=128, block_kv=64, kh=0.05, kl=0.10, labels=None, out=None, ws=None):
+    """sla_forward_pisa: O [B,H,N,D] bf16. labels [B,H,Nq,Nk] int8 (2 = critical) or None (the router)."""
+    B, H, N, D = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_act(name, t, B, H, N, D, dev)
+    p = problem(B, H, N, D, block_q, block_kv, kh, kl)
+    Nq, Nk, _, _ = counts(p)
+    if labels is not None and (labels.dtype != torch.int8 or tuple(labels.shape) != (B, H, Nq, Nk)
+                               or not labels.is_contiguous() or labels.device != dev):
+        raise ValueError(f"labels must be contiguous int8 [{B}, {H}, {Nq}, {Nk}] on {dev}")
+    if out is None:
+        out = torch.empty_like(q)
+    if ws is None:
+        ws = new_workspace_pisa(p, dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_forward_pisa(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(labels), _ptr(out), _ptr(ws),
+                                  ctypes.c_size_t(ws.numel()), _stream_handle(dev))
+    _raise(st)
+    return out
+
+
+def pisa_hbar(k, v, block_kv=64, ws=None):
+    """sla_pisa_hbar: Hbar [B,H,D,D] fp32, the mean over KV blocks of (K_j - kbar_j)^T V_j."""
+    B, H, N, D = k.shape
+    dev = k.device
+    for name, t in (("k", k), ("v", v)):
+        _check_act(name, t, B, H, N, D, dev)
+    p = problem(B, H, N, D, 128, block_kv)
+    if ws is None:
+        ws = new_workspace_pisa(p, dev)
+    out = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        st = lib.sla_pisa_hbar(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(out), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                               _stream_handle(dev))
+    _raise(st)
+    return out
 
 
 def forward_launches(p, with_mask=False, low_bit=False) -> int:

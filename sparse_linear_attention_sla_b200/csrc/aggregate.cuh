@@ -28,7 +28,6 @@ struct AggArgs {
   // the linear branch into the sparse branch's accumulator (see attn_kernel). Z_i is unscaled.
   const float* alpha;    // [H, D]
   int H;
-  int bh0;               // (batch, head) index of this launch's first head: head = (bh0 + bh) % H
 };
 
 
@@ -169,7 +168,7 @@ __global__ void __launch_bounds__(224, 1) agg_kernel(const __grid_constant__ CUt
       tc_fence_after();
       const bool z_tile = n0 >= D * D;
       if (a.alpha && !z_tile) {  // column c of the tile is channel (n0 + c) % D of h_j's rows
-        const float al = a.alpha[((a.bh0 + bh) % a.H) * D + (n0 + et) % D];
+        const float al = a.alpha[(bh % a.H) * D + (n0 + et) % D];
         sGamma[et] = (1.f - al) / fmaxf(al, kAlphaFloor);
       } else {
         sGamma[et] = 1.f;

@@ -46,6 +46,16 @@
 // of acc waits for this tile's epilogue.
 // An empty critical set gives O_s = 0 (l taken as 1); an empty marginal set gives Z_i = 0
 // and no linear term.
+//
+// PISA (template flag; "PISA - Atención Dispersa por Tramos para Transformers de Difusión
+// Eficientes" §2): no alpha and no linear branch. Every block that is not critical enters
+// the softmax through its centroid: after the critical blocks the tile runs ceil(Nk / 64)
+// pseudo-blocks whose keys are the block means kbar_j and whose values are the block sums
+// Vsum_j, the centroid of a critical block (and of a block past Nk) masked out. With
+// p_j = 2^(q . kbar_j log2(e) / sqrt(D) - m) the pseudo-block adds p_j Vsum_j to the
+// accumulator (the MMA), n_j p_j to the normaliser and p_j to A = sum_j p_j; the tail writes
+// P_lin = (A / sqrt(D)) q and H~ = Hbar, the mean first-order matrix of the head, so that
+// O = (acc + (q / sqrt(D)) Hbar A) / l.
 #pragma once
 
 #include "sm100.cuh"
@@ -54,6 +64,8 @@ namespace sla {
 
 struct AttnArgs {
   int H, N, Nq, block_q, n_tiles;
+  int Nk, nc, n_last;       // PISA: KV blocks, centroid pseudo-blocks (ceil(Nk / 64)), keys of the last block
+  float inv_sqrt_d;         // PISA: 1 / sqrt(D)
   const int32_t* crit;      // [BH*Nq, crit_ld] critical KV block indices, ascending
   int crit_ld;
   const int32_t* crit_cnt;  // [BH*Nq]
@@ -80,11 +92,14 @@ struct AttnSmem {
   static constexpr uint32_t total() { return Q + 2 * SLOT + 1024; }
 };
 
-template <int D, int FM = 0>  // FM: feature map of the linear branch, 0 elu + 1, 1 e^x
+// FM: feature map of the linear branch, 0 elu + 1, 1 e^x. PISA: the piecewise variant (see
+// the end of the header comment); map_kc / map_vc are read only then.
+template <int D, int FM = 0, bool PISA = false>
 __global__ void __launch_bounds__(192, 2)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_h,
-                const __grid_constant__ CUtensorMap map_o, AttnArgs a) {
+                const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_kc,
+                const __grid_constant__ CUtensorMap map_vc, AttnArgs a) {
   using L = AttnSmem<D>;
   constexpr int DB = D / 64;  // 64-column boxes per row
   constexpr uint32_t TMEM_COLS = 256;
@@ -139,6 +154,10 @@ __global__ void __launch_bounds__(192, 2)
       prefetch_tmap(&map_k);
       prefetch_tmap(&map_v);
       prefetch_tmap(&map_h);
+      if constexpr (PISA) {
+        prefetch_tmap(&map_kc);
+        prefetch_tmap(&map_vc);
+      }
       int k_round[2] = {-1, -1}, v_round[2] = {-1, -1};
       int q_loads = 0;
       uint32_t nb = 0;  // ring uses so far (K/V blocks and H_i pseudo-blocks)
@@ -147,37 +166,41 @@ __global__ void __launch_bounds__(192, 2)
       for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
         const int bh = t / a.Nq, i = t % a.Nq;
         const int kc = a.crit_cnt[t];
+        const int nblk = kc + (PISA ? a.nc : 0);  // blocks of the softmax: critical, then centroid
         const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
+        const int h_row = (PISA ? bh : t) * D;   // first row of this tile's H~ (per head for PISA)
         if (k > 0 && !(ok = mbar_wait(&q_free, (k - 1) & 1, a.err, &abort_flag))) break;
         mbar_arrive_expect_tx(&q_full, L::Q);
         for (int b = 0; b < DB; ++b) tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * a.block_q, bh);
         ++q_loads;
-        for (int n = 0; n <= kc; ++n, ++nb) {  // n == kc is the H_i pseudo-block
+        for (int n = 0; n <= nblk; ++n, ++nb) {  // n == nblk is the H~ pseudo-block
           const int s = nb & 1, r = nb >> 1;
           uint8_t* slot = sRing + s * L::SLOT;
           // The K half is refilled as soon as S of its previous block is done, the V half
           // once P*V of its previous block is done.
           if (r > 0 && !(ok = mbar_wait(&k_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
-          const int j = n < kc ? clist[n] : 0;
-          if (n < kc) {
+          const int j = n < kc ? clist[n] : n - kc;  // KV block, or centroid pseudo-block
+          const CUtensorMap* mk = n < kc ? &map_k : &map_kc;
+          const CUtensorMap* mv = n < kc ? &map_v : &map_vc;
+          if (n < nblk) {
             mbar_arrive_expect_tx(&k_full[s], L::KV);
-            for (int b = 0; b < DB; ++b) tma_load_3d(slot + b * 8192, &map_k, &k_full[s], b * 64, j * 64, bh);
-          } else if (D == 128) {  // H_i rows 0..63 land in the K half, rows 64..127 in the V half
+            for (int b = 0; b < DB; ++b) tma_load_3d(slot + b * 8192, mk, &k_full[s], b * 64, j * 64, bh);
+          } else if (D == 128) {  // H~ rows 0..63 land in the K half, rows 64..127 in the V half
             mbar_arrive_expect_tx(&k_full[s], L::KV);
-            for (int eh = 0; eh < 2; ++eh) tma_load_2d(slot + eh * 8192, &map_h, &k_full[s], eh * 64, t * D);
+            for (int eh = 0; eh < 2; ++eh) tma_load_2d(slot + eh * 8192, &map_h, &k_full[s], eh * 64, h_row);
           } else {
             mbar_arrive_expect_tx(&k_full[s], L::HT);
-            tma_load_2d(slot, &map_h, &k_full[s], 0, t * D);
+            tma_load_2d(slot, &map_h, &k_full[s], 0, h_row);
           }
           k_round[s] = r;
           if (r > 0 && !(ok = mbar_wait(&v_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
-          if (n < kc) {
+          if (n < nblk) {
             mbar_arrive_expect_tx(&v_full[s], L::KV);
-            for (int b = 0; b < DB; ++b) tma_load_3d(slot + L::KV + b * 8192, &map_v, &v_full[s], b * 64, j * 64, bh);
+            for (int b = 0; b < DB; ++b) tma_load_3d(slot + L::KV + b * 8192, mv, &v_full[s], b * 64, j * 64, bh);
           } else if (D == 128) {
             mbar_arrive_expect_tx(&v_full[s], L::KV);
             for (int eh = 0; eh < 2; ++eh)
-              tma_load_2d(slot + L::KV + eh * 8192, &map_h, &v_full[s], eh * 64, t * D + 64);
+              tma_load_2d(slot + L::KV + eh * 8192, &map_h, &v_full[s], eh * 64, h_row + 64);
           } else {
             mbar_arrive(&v_full[s]);
           }
@@ -230,7 +253,7 @@ __global__ void __launch_bounds__(192, 2)
       return true;
     };
     for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
-      const int kc = a.crit_cnt[t];
+      const int kc = a.crit_cnt[t] + (PISA ? a.nc : 0);  // blocks of the softmax
       if (!(ok = wait_all(&q_full, k & 1))) break;
       for (int n = 0; n < kc; ++n, ++nb, ++ns) {
         const int s = nb & 1, b = ns & 1;
@@ -292,8 +315,8 @@ __global__ void __launch_bounds__(192, 2)
     int k = 0;
     // This thread's entries of Z_i and alpha for the tile after the current one, loaded
     // during the current tile so that their latency stays off the tile boundary.
-    float z_next = 0.f, a_next = 0.f;
-    if (wt < D && static_cast<int>(blockIdx.x) < a.n_tiles) {
+    float z_next = 0.f, a_next = 1.f;
+    if (!PISA && wt < D && static_cast<int>(blockIdx.x) < a.n_tiles) {
       z_next = a.Zagg[static_cast<size_t>(blockIdx.x) * D + wt];
       a_next = a.alpha[(blockIdx.x / a.Nq % a.H) * D + wt];
     }
@@ -302,9 +325,10 @@ __global__ void __launch_bounds__(192, 2)
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++k) {
       const int bh = t / a.Nq, i = t % a.Nq;
       const int kc = a.crit_cnt[t];
+      const int nblk = kc + (PISA ? a.nc : 0);  // blocks of the softmax: critical, then centroid
       const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
-      const uint32_t hs = (nbw + kc) & 1;  // ring slot of this tile's H~_i, reused to stage O
-      nbw += kc + 1;
+      const uint32_t hs = (nbw + nblk) & 1;  // ring slot of this tile's H~, reused to stage O
+      nbw += nblk + 1;
       if (!named_barrier_and(1, 128, ok)) break;  // the previous tile's epilogue is done with sZ / sAlpha
       if (wt < D) {
         sZ[wt] = z_next;
@@ -320,15 +344,17 @@ __global__ void __launch_bounds__(192, 2)
         mbar_arrive(&v_empty[release_slot]);
         release_slot = -1;
       }
-      if (wt < D && t + static_cast<int>(gridDim.x) < a.n_tiles) {
+      if (!PISA && wt < D && t + static_cast<int>(gridDim.x) < a.n_tiles) {
         const int tn = t + gridDim.x;
         z_next = a.Zagg[static_cast<size_t>(tn) * D + wt];
         a_next = a.alpha[(tn / a.Nq % a.H) * D + wt];
       }
       float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and row sum
+      float a_run = 0.f;                     // PISA: sum of the centroid weights p_j
+      int cp = 0;                            // PISA: first critical entry not yet met by a pseudo-block
       uint32_t sa[32], sb[32];               // S columns [0, 32) and [32, 64) of the current block
       int j_cur = kc > 0 ? clist[0] : 0;
-      if (kc > 0) {
+      if (nblk > 0) {
         ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[ns & 1], (ns >> 1) & 1, a.err, &abort_flag));
         if (ok) {
           tc_fence_after();
@@ -337,15 +363,36 @@ __global__ void __launch_bounds__(192, 2)
           tmem_wait_ld();
         }
       }
-      for (int n = 0; ok && n < kc; ++n, ++ns) {
+      for (int n = 0; ok && n < nblk; ++n, ++ns) {
         const int b = ns & 1;
         const int j_next = n + 1 < kc ? clist[n + 1] : 0;
-        const int valid = min(64, a.N - j_cur * 64);  // valid key columns of this block
-        if (valid < 64) {
+        const bool centroid = PISA && n >= kc;
+        uint64_t keep = ~0ull;  // PISA: the centroids of this pseudo-block that take part
+        if (!centroid) {
+          const int valid = min(64, a.N - j_cur * 64);  // valid key columns of this block
+          if (valid < 64) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (c >= valid) sa[c] = __float_as_uint(-INFINITY);
-            if (c + 32 >= valid) sb[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 32; ++c) {
+              if (c >= valid) sa[c] = __float_as_uint(-INFINITY);
+              if (c + 32 >= valid) sb[c] = __float_as_uint(-INFINITY);
+            }
+          }
+        } else {
+          // centroids 64 pb .. 64 pb + 63: drop those of critical blocks (the ascending list
+          // is walked once over the tile's pseudo-blocks) and those past Nk
+          const int pb = n - kc;
+          while (cp < kc && clist[cp] < 64 * (pb + 1)) {
+            keep &= ~(1ull << (clist[cp] - 64 * pb));
+            ++cp;
+          }
+          const int nv = min(64, a.Nk - 64 * pb);
+          if (nv < 64) keep &= (1ull << nv) - 1ull;
+          if (keep != ~0ull) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (!((keep >> c) & 1ull)) sa[c] = __float_as_uint(-INFINITY);
+              if (!((keep >> (c + 32)) & 1ull)) sb[c] = __float_as_uint(-INFINITY);
+            }
           }
         }
         // row maximum: four independent chains of 3-input maxima
@@ -389,6 +436,7 @@ __global__ void __launch_bounds__(192, 2)
           }
           tmem_wait_st();
           l_run *= f;
+          a_run *= f;
           m_run = m_new;
         }
         // p = 2^(s * scale - m): one paired FMA per two elements and one exponential per
@@ -408,14 +456,32 @@ __global__ void __launch_bounds__(192, 2)
           pk[16 + (c >> 1)] = pack_bf16x2(e2, e3);
         }
         const uint64_t pst = f2_add(ps2, ps2b);
-        l_run += f2_lo(pst) + f2_hi(pst);
+        const float psum = f2_lo(pst) + f2_hi(pst);
+        if (!centroid) {
+          l_run += psum;
+        } else {
+          // centroid j weighs n_j in the normaliser: 64, except a short last block
+          float wsum = 64.f * psum;
+          const int cl = a.Nk - 1 - 64 * (a.nc - 1);  // column of block Nk - 1 in the last pseudo-block
+          if (a.n_last < 64 && n + 1 == nblk && ((keep >> cl) & 1ull)) {
+            float s_l = 0.f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              if (c == cl) s_l = __uint_as_float(sa[c]);
+              if (c + 32 == cl) s_l = __uint_as_float(sb[c]);
+            }
+            wsum -= static_cast<float>(64 - a.n_last) * fast_exp2(fmaf(s_l, sc, -m_run));
+          }
+          l_run += wsum;
+          a_run += psum;
+        }
         tmem_st32(lane_addr + b * 64, pk);  // P over the first 32 columns of its S
         // Publish P_n before waiting for S_{n+1}: P*V of this block, and the S two blocks on
         // (which reuses these columns), can then be issued while S_{n+1} is still in flight.
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
-        if (n + 1 < kc) {
+        if (n + 1 < nblk) {
           ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b ^ 1], ((ns + 1) >> 1) & 1, a.err, &abort_flag));
           if (ok) {
             tc_fence_after();
@@ -429,7 +495,7 @@ __global__ void __launch_bounds__(192, 2)
       // Linear branch. P_lin goes into the S columns the next block would have used
       // (ns & 1); their last reader is the P*V two blocks back (with one block or none, an
       // MMA of an earlier tile, finished before this tile's lin_done was seen).
-      if (ok && kc >= 2)
+      if (ok && nblk >= 2)
         ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 2) & 1], ((ns - 2) >> 1) & 1, a.err, &abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full, k & 1, a.err, &abort_flag));
       // Pass 1: phi(q) (bf16, as the tensor core takes it) into the P_lin columns, 32
@@ -437,61 +503,93 @@ __global__ void __launch_bounds__(192, 2)
       // is released (the next tile's Q may land). Column pairs in paired arithmetic:
       // phi(x) = x + 1 for x > 0, else e^x = 2^(x log2 e) (with FM = 1, e^x throughout).
       const uint32_t pl = lane_addr + (ns & 1) * 64;
-      uint64_t den2 = 0ull;
-      if (ok) {
-        const uint64_t one2 = f2_make(1.f, 1.f), log2e2 = f2_make(1.4426950408889634f, 1.4426950408889634f);
+      float l_eff;
+      if constexpr (PISA) {
+        // First-order term: P_lin = (A / sqrt(D)) q in bf16 against H~ = Hbar; l > 0 always
+        // (the row maximum is a key or a centroid that takes part).
+        l_eff = l_run;
+        if (ok) {
+          const float cq = a_run * a.inv_sqrt_d;
+          const uint64_t c2 = f2_make(cq, cq);
 #pragma unroll 1
-        for (int g = 0; g < D / 32; ++g) {
-          uint32_t w[16];
+          for (int g = 0; g < D / 32; ++g) {
+            uint32_t w[16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int c8 = 4 * g + c;
-            const uint4 u = *reinterpret_cast<const uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
-            w[4 * c] = u.x;
-            w[4 * c + 1] = u.y;
-            w[4 * c + 2] = u.z;
-            w[4 * c + 3] = u.w;
-          }
+            for (int c = 0; c < 4; ++c) {
+              const int c8 = 4 * g + c;
+              const uint4 u = *reinterpret_cast<const uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
+              w[4 * c] = u.x;
+              w[4 * c + 1] = u.y;
+              w[4 * c + 2] = u.z;
+              w[4 * c + 3] = u.w;
+            }
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            // bf16 -> fp32 is a shift into the high half-word
-            const uint64_t x2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
-            const uint64_t pos2 = f2_add(x2, one2);
-            const uint64_t t2 = f2_mul(x2, log2e2);
-            const float g0 = FM == 0 && f2_lo(x2) > 0.f ? f2_lo(pos2) : fast_exp2(f2_lo(t2));
-            const float g1 = FM == 0 && f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
-            w[e] = pack_bf16x2(g0, g1);
-            const uint64_t gr2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
-            den2 = f2_fma(gr2, *reinterpret_cast<const uint64_t*>(&sZ[32 * g + 2 * e]), den2);
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t y2 = f2_mul(c2, static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32));
+              w[e] = pack_bf16x2(f2_lo(y2), f2_hi(y2));
+            }
+            tmem_st16(pl + 16 * g, w);
           }
-          tmem_st16(pl + 16 * g, w);
+          tmem_wait_st();
         }
-      }
-      mbar_arrive(&q_free);
-      // The blend O = alpha O_s / l + (1 - alpha) O_l / den, with the accumulator holding
-      // l O_s and H~_i = H_i (1 - alpha) / alpha, is alpha (acc + (l / den) phi(q) H~_i) / l.
-      // With no critical block l is taken as 1 (acc starts at 0); with no marginal block
-      // (den = 0) the linear term is 0.
-      const float den_tot = f2_lo(den2) + f2_hi(den2);
-      const float l_eff = kc > 0 ? l_run : 1.f;
-      const float c_lin = den_tot > 0.f ? l_eff / den_tot : 0.f;
-      // Pass 2: P_lin = (l / den) phi(q), rounded to bf16 in place.
-      if (ok) {
-        tmem_wait_st();
-        const uint64_t c2 = f2_make(c_lin, c_lin);
+        mbar_arrive(&q_free);
+      } else {
+        uint64_t den2 = 0ull;
+        if (ok) {
+          const uint64_t one2 = f2_make(1.f, 1.f), log2e2 = f2_make(1.4426950408889634f, 1.4426950408889634f);
 #pragma unroll 1
-        for (int g = 0; g < D / 64; ++g) {
-          uint32_t w[32];
-          tmem_ld32(pl + 32 * g, w);
-          tmem_wait_ld();
+          for (int g = 0; g < D / 32; ++g) {
+            uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const uint64_t g2 = f2_mul(c2, static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32));
-            w[e] = pack_bf16x2(f2_lo(g2), f2_hi(g2));
+            for (int c = 0; c < 4; ++c) {
+              const int c8 = 4 * g + c;
+              const uint4 u = *reinterpret_cast<const uint4*>(sQ + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
+              w[4 * c] = u.x;
+              w[4 * c + 1] = u.y;
+              w[4 * c + 2] = u.z;
+              w[4 * c + 3] = u.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              // bf16 -> fp32 is a shift into the high half-word
+              const uint64_t x2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
+              const uint64_t pos2 = f2_add(x2, one2);
+              const uint64_t t2 = f2_mul(x2, log2e2);
+              const float g0 = FM == 0 && f2_lo(x2) > 0.f ? f2_lo(pos2) : fast_exp2(f2_lo(t2));
+              const float g1 = FM == 0 && f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
+              w[e] = pack_bf16x2(g0, g1);
+              const uint64_t gr2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
+              den2 = f2_fma(gr2, *reinterpret_cast<const uint64_t*>(&sZ[32 * g + 2 * e]), den2);
+            }
+            tmem_st16(pl + 16 * g, w);
           }
-          tmem_st32(pl + 32 * g, w);
         }
-        tmem_wait_st();
+        mbar_arrive(&q_free);
+        // The blend O = alpha O_s / l + (1 - alpha) O_l / den, with the accumulator holding
+        // l O_s and H~_i = H_i (1 - alpha) / alpha, is alpha (acc + (l / den) phi(q) H~_i) / l.
+        // With no critical block l is taken as 1 (acc starts at 0); with no marginal block
+        // (den = 0) the linear term is 0.
+        const float den_tot = f2_lo(den2) + f2_hi(den2);
+        l_eff = kc > 0 ? l_run : 1.f;
+        const float c_lin = den_tot > 0.f ? l_eff / den_tot : 0.f;
+        // Pass 2: P_lin = (l / den) phi(q), rounded to bf16 in place.
+        if (ok) {
+          tmem_wait_st();
+          const uint64_t c2 = f2_make(c_lin, c_lin);
+#pragma unroll 1
+          for (int g = 0; g < D / 64; ++g) {
+            uint32_t w[32];
+            tmem_ld32(pl + 32 * g, w);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const uint64_t g2 = f2_mul(c2, static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32));
+              w[e] = pack_bf16x2(f2_lo(g2), f2_hi(g2));
+            }
+            tmem_st32(pl + 32 * g, w);
+          }
+          tmem_wait_st();
+        }
       }
       tc_fence_before();
       mbar_arrive(&plin_full);

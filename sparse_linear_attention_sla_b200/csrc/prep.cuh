@@ -29,30 +29,6 @@ __device__ __forceinline__ float phi_f(float x) {
   return x > 0.f ? x + 1.f : __expf(x);
 }
 
-// Exact fp64 value of a bf16 without the conversion unit. For a normal bf16 (exponent field
-// E in 1..254, 7 mantissa bits M) the fp64 has exponent field E + 896 and M as its top
-// mantissa bits, so its high word is (magnitude << 13) + (896 << 20) with the sign on top
-// and its low word is 0. bf16_lo_f64 takes the bf16 in bits 0..15 of a packed pair,
-// bf16_hi_f64 the one in bits 16..31.
-__device__ __forceinline__ double bf16_lo_f64(uint32_t w) {
-  const uint32_t hi = (((w & 0x7FFFu) << 13) + 0x38000000u) | ((w & 0x8000u) << 16);
-  return __hiloint2double(static_cast<int>(hi), 0);
-}
-__device__ __forceinline__ double bf16_hi_f64(uint32_t w) {
-  const uint32_t hi = (((w & 0x7FFF0000u) >> 3) + 0x38000000u) | (w & 0x80000000u);
-  return __hiloint2double(static_cast<int>(hi), 0);
-}
-// True if either bf16 of a packed pair has exponent field 0 (zero or subnormal) or 255
-// (infinity or NaN): those take the conversion instruction instead. Per 16-bit half, with
-// t the exponent bits in place: t + 0x80 carries into bit 15 only for 0xFF, and
-// (t | 0x8000) - 0x80 clears bit 15 only for 0.
-__device__ __forceinline__ bool bf16x2_not_normal(uint32_t w) {
-  const uint32_t t = w & 0x7F807F80u;
-  const uint32_t all_ones = (t + 0x00800080u) & 0x80008000u;
-  const uint32_t zero = ~((t | 0x80008000u) - 0x00800080u) & 0x80008000u;
-  return (all_ones | zero) != 0u;
-}
-
 // ---------------------------------------------------------------- pooling
 // grid: (nblocks, BH); block: 128 threads. x: [BH, N, D] bf16; out: [BH, nblocks, D] fp64.
 template <int D>
@@ -72,18 +48,11 @@ __global__ void __launch_bounds__(128) pool_mean_kernel(const __nv_bfloat16* __r
   for (int r = r0 + rr; r < r1; r += RSTEP) {
     uint4 u = *reinterpret_cast<const uint4*>(base + static_cast<size_t>(r) * D);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    const bool rare = bf16x2_not_normal(w[0]) | bf16x2_not_normal(w[1]) | bf16x2_not_normal(w[2]) |
-                      bf16x2_not_normal(w[3]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      if (!rare) {
-        acc[2 * e] += bf16_lo_f64(w[e]);
-        acc[2 * e + 1] += bf16_hi_f64(w[e]);
-      } else {
-        const float2 f = unpack_bf16x2(w[e]);
-        acc[2 * e] += static_cast<double>(f.x);
-        acc[2 * e + 1] += static_cast<double>(f.y);
-      }
+      const float2 f = unpack_bf16x2(w[e]);
+      acc[2 * e] += static_cast<double>(f.x);
+      acc[2 * e + 1] += static_cast<double>(f.y);
     }
   }
 #pragma unroll
@@ -143,20 +112,13 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
     const uint4 u = *p;
     uint32_t w[4] = {u.x, u.y, u.z, u.w};
     const bool in = rr < valid;
-    const bool rare = bf16x2_not_normal(w[0]) | bf16x2_not_normal(w[1]) | bf16x2_not_normal(w[2]) |
-                      bf16x2_not_normal(w[3]);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const float2 x = unpack_bf16x2(w[e]);
       float f0 = 0.f, f1 = 0.f;
       if (in) {
-        if (!rare) {  // exact either way; the integer form keeps the conversion unit free
-          ks[2 * e] += bf16_lo_f64(w[e]);
-          ks[2 * e + 1] += bf16_hi_f64(w[e]);
-        } else {
-          ks[2 * e] += static_cast<double>(x.x);
-          ks[2 * e + 1] += static_cast<double>(x.y);
-        }
+        ks[2 * e] += static_cast<double>(x.x);
+        ks[2 * e + 1] += static_cast<double>(x.y);
         if (PHI) {
           f0 = phi_f<FM>(x.x);
           f1 = phi_f<FM>(x.y);

@@ -631,7 +631,7 @@ struct MaskListArgs {
   int32_t* crit;
   int crit_ld;
   int32_t* crit_cnt;
-  __nv_bfloat16* W;
+  __nv_bfloat16* W;     // marginal indicator [rows, w_ld] (nullable)
   int w_ld;
   uint32_t* err;
 };
@@ -657,12 +657,13 @@ __global__ void __launch_bounds__(256) mask_lists_kernel(MaskListArgs a) {
     const bool is_c = in && lab == 2;
     const uint32_t bcrit = __ballot_sync(0xffffffffu, is_c);
     if (in) {
-      a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(lab == 1 ? 1.f : 0.f);
+      if (a.W) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(lab == 1 ? 1.f : 0.f);
       if (is_c) a.crit[static_cast<size_t>(row) * a.crit_ld + crit_before + __popc(bcrit & lt_mask)] = j;
     }
     crit_before += __popc(bcrit);
   }
-  for (int j = a.Nk + lane; j < a.w_ld; j += 32) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(0.f);
+  if (a.W)
+    for (int j = a.Nk + lane; j < a.w_ld; j += 32) a.W[static_cast<size_t>(row) * a.w_ld + j] = __float2bfloat16_rn(0.f);
   if (lane == 0) a.crit_cnt[row] = crit_before;
   if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(a.err, SLA_DEVERR_BAD_MASK);
 }

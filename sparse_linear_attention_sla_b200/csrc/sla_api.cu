@@ -17,6 +17,7 @@
 #include "backward.cuh"
 #include "backward_states.cuh"
 #include "fp8.cuh"
+#include "pisa.cuh"
 #include "prep.cuh"
 #include "route.cuh"
 #include "variants.cuh"
@@ -121,12 +122,17 @@ struct Workspace {
   uint8_t* v8;     // e4m3 codes of V [BH, N, D]
   int32_t* kexp;   // K block scale exponents [BH, Nk]
   int32_t* vexp;   // V block scale exponents [BH, Nk]
+  // PISA only
+  __nv_bfloat16* kcen;  // centroid keys: block means of K [BH, Nk, D]
+  __nv_bfloat16* vsum;  // centroid values: block sums of V [BH, Nk, D]
+  float* hpart;         // per-part sums of the centred first-order matrices [BH * P, D, D]
+  __nv_bfloat16* hbar;  // mean first-order matrix per head [BH, D, D]
   size_t bytes;
 };
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false, bool bwd = false) {
+Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false, bool bwd = false, bool pisa = false) {
   Workspace w{};
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -164,14 +170,22 @@ Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false, bool bwd = fal
     w.kexp = reinterpret_cast<int32_t*>(take(BH * s.Nk * sizeof(int32_t)));
     w.vexp = reinterpret_cast<int32_t*>(take(BH * s.Nk * sizeof(int32_t)));
   }
+  if (pisa) {
+    const size_t DD = static_cast<size_t>(s.D) * s.D;
+    w.kcen = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * s.D * 2));
+    w.vsum = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * s.D * 2));
+    w.hpart = reinterpret_cast<float*>(take(BH * sla::pisa_parts(s.BH, s.Nk) * DD * sizeof(float)));
+    w.hbar = reinterpret_cast<__nv_bfloat16*>(take(BH * DD * 2));
+  }
   w.bytes = off;
   return w;
 }
 
-sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w, bool fp8 = false, bool bwd = false) {
+sla_status check_ws(const Shape& s, void* ws, size_t ws_bytes, Workspace* w, bool fp8 = false, bool bwd = false,
+                    bool pisa = false) {
   if (!ws) return fail(SLA_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(SLA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
-  *w = layout(s, static_cast<uint8_t*>(ws), fp8, bwd);
+  *w = layout(s, static_cast<uint8_t*>(ws), fp8, bwd, pisa);
   if (ws_bytes < w->bytes)
     return fail(SLA_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, w->bytes);
   return SLA_OK;
@@ -407,7 +421,7 @@ sla_status launch_select64(const Shape& s, const Workspace& w, const double* S, 
 // indicator transposed (A = W^T, M = Nk, K = Nq).
 template <int D>
 sla_status launch_agg_gemm(int M, int K, int BH, int LD, const __nv_bfloat16* A, int a_ld, const __nv_bfloat16* Bst,
-                           __nv_bfloat16* Cd, float* Cz, uint32_t* err, const float* alpha, int H, int bh0,
+                           __nv_bfloat16* Cd, float* Cz, uint32_t* err, const float* alpha, int H,
                            cudaStream_t st) {
   CUtensorMap mw, mh;
   {
@@ -432,21 +446,22 @@ sla_status launch_agg_gemm(int M, int K, int BH, int LD, const __nv_bfloat16* A,
   }
   const int smem = sla::kAggStages * sla::kAggStageBytes + sla::kAggStagingBytes + 1024;
   SLA_TRY(allow_smem(sla::agg_kernel<D>, smem));
-  AggArgs a{M, K, LD, BH, Cd, Cz, err, alpha, H, bh0};
+  AggArgs a{M, K, LD, BH, Cd, Cz, err, alpha, H};
   const long long tiles = static_cast<long long>(LD / 128) * ((M + 255) / 256) * BH;
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   return launch_dependent(sla::agg_kernel<D>, dim3(grid), dim3(224), smem, st, "agg_kernel", mw, mh, mo, a);
 }
 
 template <int D>
-sla_status launch_agg(const Shape& s, const Workspace& w, const float* alpha, cudaStream_t st, int bh0 = 0) {
-  return launch_agg_gemm<D>(s.Nq, s.Nk, s.BH, s.LD, w.W, s.w_ld, w.hst, w.Hagg, w.Zagg, w.err, alpha, s.H, bh0, st);
+sla_status launch_agg(const Shape& s, const Workspace& w, const float* alpha, cudaStream_t st) {
+  return launch_agg_gemm<D>(s.Nq, s.Nk, s.BH, s.LD, w.W, s.w_ld, w.hst, w.Hagg, w.Zagg, w.err, alpha, s.H, st);
 }
 
-template <int D, int FM = 0>
+// PISA: the centroid pseudo-blocks from w.kcen / w.vsum and H~ = w.hbar (one per head).
+template <int D, int FM = 0, bool PISA = false>
 sla_status launch_attn(const Shape& s, const void* q, const void* k, const void* v, const float* alpha, void* out,
                        const Workspace& w, int crit_ld, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mh, mo;
+  CUtensorMap mq, mk, mv, mh, mo, mkc, mvc;
   SLA_TRY(act_map(&mq, q, s, 128));
   // output boxes of block_q rows: the staged 128-row tile holds the next query block's rows
   // past block_q when block_q = 64, and those must not be written
@@ -454,13 +469,25 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   SLA_TRY(act_map(&mk, k, s, 64));
   SLA_TRY(act_map(&mv, v, s, 64));
   {
-    const uint64_t dims[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.BH) * s.Nq * s.D};
+    const uint64_t rows = static_cast<uint64_t>(s.BH) * (PISA ? 1 : s.Nq) * s.D;
+    const uint64_t dims[2] = {static_cast<uint64_t>(s.D), rows};
     const uint64_t strides[1] = {static_cast<uint64_t>(s.D)};
     const uint32_t box[2] = {64, 64};
-    SLA_TRY(make_map(&mh, w.Hagg, 2, dims, strides, box));
+    SLA_TRY(make_map(&mh, PISA ? w.hbar : w.Hagg, 2, dims, strides, box));
+  }
+  if (PISA) {
+    // [BH, Nk, D]: the last pseudo-block's rows past Nk read as zeros
+    const uint64_t dims[3] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.Nk), static_cast<uint64_t>(s.BH)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(s.D), static_cast<uint64_t>(s.Nk) * s.D};
+    const uint32_t box[3] = {64, 64, 1};
+    SLA_TRY(make_map(&mkc, w.kcen, 3, dims, strides, box));
+    SLA_TRY(make_map(&mvc, w.vsum, 3, dims, strides, box));
+  } else {
+    mkc = mk;
+    mvc = mv;
   }
   constexpr int smem = sla::AttnSmem<D>::total();
-  SLA_TRY(allow_smem(sla::attn_kernel<D, FM>, smem));
+  SLA_TRY(allow_smem(sla::attn_kernel<D, FM, PISA>, smem));
   AttnArgs a;
   a.H = s.H;
   a.N = s.N;
@@ -470,15 +497,19 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.crit = w.crit;
   a.crit_ld = crit_ld;
   a.crit_cnt = w.crit_cnt;
-  a.Zagg = w.Zagg;
-  a.alpha = alpha;
+  a.Zagg = PISA ? nullptr : w.Zagg;
+  a.alpha = PISA ? nullptr : alpha;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  a.Nk = s.Nk;
+  a.nc = (s.Nk + 63) / 64;
+  a.n_last = s.N - (s.Nk - 1) * 64;
+  a.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   a.err = w.err;
   // persistent: two CTAs per SM walk the tiles
   const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
-  return launch_dependent(sla::attn_kernel<D, FM>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv, mh, mo,
-                          a);
+  return launch_dependent(sla::attn_kernel<D, FM, PISA>, dim3(grid), dim3(192), smem, st, "attn_kernel", mq, mk, mv,
+                          mh, mo, mkc, mvc, a);
 }
 
 template <int D>
@@ -616,7 +647,7 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
   sla::w_transpose_kernel<<<dim3((s.Nk + 31) / 32, w.wt_ld / 32, s.BH), dim3(32, 8), 0, st>>>(w.W, s.Nq, s.Nk, s.w_ld,
                                                                                            w.WT, w.wt_ld);
   SLA_TRY(launched("w_transpose_kernel"));
-  SLA_TRY(launch_agg_gemm<D>(s.Nk, s.Nq, s.BH, s.LD, w.WT, w.wt_ld, w.dHst, w.dh, w.dz, w.err, nullptr, s.H, 0, st));
+  SLA_TRY(launch_agg_gemm<D>(s.Nk, s.Nq, s.BH, s.LD, w.WT, w.wt_ld, w.dHst, w.dh, w.dz, w.err, nullptr, s.H, st));
   // the states' part of dK, dV
   {
     CUtensorMap mk, mv, mdh;
@@ -716,6 +747,50 @@ sla_status forward_variant_impl(const Shape& s, const Variant& var, const void* 
   return launch_attn<D, FM>(s, q, k, v, alpha, out, w, s.Nk, st);
 }
 
+// ------------------------------------------------------------------ PISA
+
+// Centroid keys and values, the per-part first-order sums and (with_kbar) the fp64 block
+// means for the router.
+template <int D>
+sla_status launch_pisa_stats(const void* k, const void* v, const Shape& s, const Workspace& w, bool with_kbar,
+                             cudaStream_t st) {
+  CUtensorMap mk, mv;
+  SLA_TRY(act_map(&mk, k, s, 64));
+  SLA_TRY(act_map(&mv, v, s, 64));
+  sla::PisaStatsArgs a{s.BH, s.N, s.Nk, sla::pisa_parts(s.BH, s.Nk), with_kbar ? w.kbar : nullptr, w.kcen, w.vsum,
+                       w.hpart, w.err};
+  constexpr int smem = sla::PisaSmem<D>::total();
+  SLA_TRY(allow_smem(sla::pisa_stats_kernel<D>, smem));
+  const int parts = s.BH * a.P;
+  const int grid = parts < sm_count() ? parts : sm_count();
+  sla::pisa_stats_kernel<D><<<grid, 576, smem, st>>>(mk, mv, a);
+  return launched("pisa_stats_kernel");
+}
+
+template <int D>
+sla_status launch_hbar(const Shape& s, const Workspace& w, __nv_bfloat16* h16, float* h32, cudaStream_t st) {
+  sla::hbar_kernel<D><<<dim3(D, s.BH), D, 0, st>>>(w.hpart, h16, h32, sla::pisa_parts(s.BH, s.Nk), s.Nk);
+  return launched("hbar_kernel");
+}
+
+// The PISA forward: statistics, critical sets (the router's label 2, or the caller's labels),
+// Hbar, the fused pass.
+template <int D>
+sla_status forward_pisa_impl(const Shape& s, const void* q, const void* k, const void* v, const int8_t* labels,
+                             void* out, const Workspace& w, cudaStream_t st) {
+  SLA_TRY(launch_pisa_stats<D>(k, v, s, w, labels == nullptr, st));
+  if (labels) {
+    MaskListArgs m{labels, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, nullptr, s.w_ld, w.err};
+    sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+    SLA_TRY(launched("mask_lists_kernel"));
+  } else {
+    SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
+    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, nullptr, st));
+  }
+  SLA_TRY(launch_hbar<D>(s, w, w.hbar, nullptr, st));
+  return launch_attn<D, 0, true>(s, q, k, v, nullptr, out, w, s.Nk, st);
+}
+
 // Stage boundaries for sla_forward_timed: ev[0] before the per-block precompute,
 // ev[1] after it, ev[2] after routing, ev[3] after aggregation, ev[4] after attention.
 // sla_forward_fp8_timed: ev[4] after the K/V quantiser, ev[5] after attention.
@@ -729,41 +804,6 @@ struct StageEvents {
     return SLA_OK;
   }
 };
-
-// The forward's per-head pieces of the workspace for heads h0, h0 + 1, ... (every piece is
-// head-major), except the per-block states: a group of heads always writes them at the start
-// of their buffer, so every group reuses the same lines of L2.
-Workspace group_view(const Workspace& w, const Shape& s, int h0) {
-  const size_t h = static_cast<size_t>(h0);
-  Workspace o = w;
-  o.qbar = w.qbar + h * s.Nq * s.D;
-  o.kbar = w.kbar + h * s.Nk * s.D;
-  o.S = w.S + h * s.Nq * s.Nk;
-  o.S32 = w.S32 + h * s.Nq * s.Nk;
-  o.nq = w.nq + h * s.Nq;
-  o.nk = w.nk + h * s.Nk;
-  o.mask = w.mask + h * s.Nq * s.Nk;
-  o.crit = w.crit + h * s.Nq * s.Nk;
-  o.crit_cnt = w.crit_cnt + h * s.Nq;
-  o.W = w.W + h * s.Nq * s.w_ld;
-  o.Hagg = w.Hagg + h * s.Nq * static_cast<size_t>(s.D) * s.D;
-  o.Zagg = w.Zagg + h * s.Nq * s.D;
-  return o;
-}
-
-// Heads per group of the grouped precompute -> route -> aggregation: as many as keep a
-// group's bf16 per-block states within kGroupStateBytes of L2 (so the aggregation reads them
-// from L2 right after the precompute wrote them), and no more than kMaxGroups groups.
-constexpr size_t kGroupStateBytes = size_t(48) << 20;
-constexpr int kMaxGroups = 16;
-int heads_per_group(const Shape& s) {
-  const size_t per_head = static_cast<size_t>(s.Nk) * s.LD * 2;
-  int g = static_cast<int>(kGroupStateBytes / per_head);
-  const int min_g = (s.BH + kMaxGroups - 1) / kMaxGroups;
-  if (g < min_g) g = min_g;
-  if (g < 1) g = 1;
-  return g > s.BH ? s.BH : g;
-}
 
 template <int D>
 sla_status forward_impl(const Shape& s, const void* q, const void* k, const void* v, const float* alpha,
@@ -783,49 +823,19 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
   // the bf16 attention adds the linear branch into its accumulator and takes H_i scaled per
   // channel by (1 - alpha) / alpha; the low-bit kernel takes H_i as it is
   const float* agg_alpha = fp8 ? nullptr : alpha;
-  const int G = heads_per_group(s);
   SLA_TRY(ev.mark(0, st));
-  if (ev.on || G >= s.BH) {
-    // One launch of each stage over every head (the timed entry point reports the stages
-    // separately this way).
-    SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
-    SLA_TRY(ev.mark(1, st));
-    if (mask) {
-      MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
-      sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
-      SLA_TRY(launched("mask_lists_kernel"));
-    } else {
-      SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
-    }
-    SLA_TRY(ev.mark(2, st));
-    SLA_TRY(launch_agg<D>(s, w, agg_alpha, st));
-    SLA_TRY(ev.mark(3, st));
+  SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
+  SLA_TRY(ev.mark(1, st));
+  if (mask) {
+    MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, w.W, s.w_ld, w.err};
+    sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+    SLA_TRY(launched("mask_lists_kernel"));
   } else {
-    // Groups of G heads: each group's states stay in L2 between its precompute and its
-    // aggregation, and the next group overwrites the same lines.
-    const size_t per_head = static_cast<size_t>(s.N) * s.D;
-    for (int h0 = 0; h0 < s.BH; h0 += G) {
-      Shape sg = s;
-      sg.BH = s.BH - h0 < G ? s.BH - h0 : G;
-      const Workspace wg = group_view(w, s, h0);
-      sla::PrepArgs pg = pa;
-      pg.BH = sg.BH;
-      pg.qbar = mask ? nullptr : wg.qbar;
-      pg.kbar = mask ? nullptr : wg.kbar;
-      const size_t off = static_cast<size_t>(h0) * per_head;
-      SLA_TRY(launch_prep<D>(static_cast<const __nv_bfloat16*>(q) + off, static_cast<const __nv_bfloat16*>(k) + off,
-                             static_cast<const __nv_bfloat16*>(v) + off, sg, pg, st));
-      if (mask) {
-        MaskListArgs m{mask + static_cast<size_t>(h0) * s.Nq * s.Nk, sg.BH * s.Nq, s.Nk, wg.crit, s.Nk,
-                       wg.crit_cnt, wg.W, s.w_ld, w.err};
-        sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
-        SLA_TRY(launched("mask_lists_kernel"));
-      } else {
-        SLA_TRY(launch_router<D>(sg, wg, nullptr, wg.mask, wg.crit, s.Nk, wg.W, st));
-      }
-      SLA_TRY(launch_agg<D>(sg, wg, agg_alpha, st, h0));
-    }
+    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
   }
+  SLA_TRY(ev.mark(2, st));
+  SLA_TRY(launch_agg<D>(s, w, agg_alpha, st));
+  SLA_TRY(ev.mark(3, st));
   if (fp8) {
     if constexpr (D == 128) {
       SLA_TRY(launch_quant<D>(s, k, v, w.k8, w.v8, w.kexp, w.vexp, st, true));
@@ -1058,10 +1068,8 @@ sla_status sla_aggregate_states(const sla_problem* p, const void* k, const void*
 int sla_forward_launches(const sla_problem* p, int with_mask, int low_bit) {
   Shape s;
   if (make_shape(p, &s) != SLA_OK) return -1;
-  const int per_group = 1 + (with_mask ? 1 : 2) + 1;  // precompute, labels (router: scores + selection), aggregation
-  const int G = heads_per_group(s);
-  const int groups = G >= s.BH ? 1 : (s.BH + G - 1) / G;
-  return groups * per_group + 1 + (low_bit ? 1 : 0);  // + attention (+ the K/V quantiser)
+  // precompute, labels (router: scores + selection), aggregation, attention (+ the K/V quantiser)
+  return 1 + (with_mask ? 1 : 2) + 1 + 1 + (low_bit ? 1 : 0);
 }
 
 sla_status sla_route_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
@@ -1106,6 +1114,46 @@ sla_status sla_forward_variant(const sla_problem* p, const sla_variant* variant,
   }
   if (var.fm) return forward_variant_impl<128, 1>(s, var, q, k, v, alpha, mask, out, w, st);
   return forward_variant_impl<128, 0>(s, var, q, k, v, alpha, mask, out, w, st);
+}
+
+size_t sla_workspace_size_pisa(const sla_problem* p) {
+  Shape s;
+  if (make_shape(p, &s) != SLA_OK) return 0;
+  return layout(s, nullptr, false, false, true).bytes;
+}
+
+sla_status sla_forward_pisa(const sla_problem* p, const void* q, const void* k, const void* v, const int8_t* labels,
+                            void* out, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SLA_ERR_INVALID_ARG, "q, k, v and out must be non-NULL and 16-byte aligned");
+  const size_t act = static_cast<size_t>(s.BH) * s.N * s.D * 2;
+  if (overlaps(out, q, act) || overlaps(out, k, act) || overlaps(out, v, act))
+    return fail(SLA_ERR_INVALID_ARG, "out must not alias q, k or v");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w, false, false, true));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) return forward_pisa_impl<64>(s, q, k, v, labels, out, w, st);
+  return forward_pisa_impl<128>(s, q, k, v, labels, out, w, st);
+}
+
+sla_status sla_pisa_hbar(const sla_problem* p, const void* k, const void* v, float* hbar_out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!aligned16(k) || !aligned16(v)) return fail(SLA_ERR_INVALID_ARG, "k and v must be non-NULL and 16-byte aligned");
+  if (!hbar_out || reinterpret_cast<uintptr_t>(hbar_out) % 4)
+    return fail(SLA_ERR_INVALID_ARG, "hbar_out must be non-NULL and 4-byte aligned");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w, false, false, true));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.D == 64) {
+    SLA_TRY(launch_pisa_stats<64>(k, v, s, w, false, st));
+    return launch_hbar<64>(s, w, nullptr, hbar_out, st);
+  }
+  SLA_TRY(launch_pisa_stats<128>(k, v, s, w, false, st));
+  return launch_hbar<128>(s, w, nullptr, hbar_out, st);
 }
 
 size_t sla_workspace_size_backward(const sla_problem* p) {

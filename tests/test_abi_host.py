@@ -163,18 +163,13 @@ def test_route_noalloc_refuses_oversize_problem(lib):
 
 
 def test_forward_launch_counts(lib):
-    """Groups of heads for the precompute, labels and aggregation: as many heads as keep a
-    group's bf16 per-block states within 48 MiB, at most 16 groups; four launches per group
-    (three with a caller mask) plus the attention (and the quantiser for the low-bit call)."""
-    # Wan2.1-1.3B shape: 512 blocks x (128*128 + 128) bf16 = 16.9 MB of states per head -> 2 heads
+    """One launch per stage: precompute, labels (the router's scores and selection, or the
+    caller mask's lists), aggregation, attention (and the quantiser for the low-bit call)."""
     p = binding.problem(1, 12, 32760, 128, 128, 64, 0.05, 0.1)
-    assert binding.forward_launches(p) == 6 * 4 + 1
-    assert binding.forward_launches(p, with_mask=True) == 6 * 3 + 1
-    assert binding.forward_launches(p, low_bit=True) == 6 * 4 + 2
-    # small problem: one group
-    assert binding.forward_launches(binding.problem(1, 2, 1024, 64, 64, 64, 0.25, 0.25)) == 5
-    # Wan2.1-14B 720p: 39 MB per head -> 1 head, but at most 16 groups -> 5 heads per group
-    assert binding.forward_launches(binding.problem(2, 40, 75600, 128, 128, 64, 0.05, 0.15)) == 16 * 4 + 1
+    assert binding.forward_launches(p) == 5
+    assert binding.forward_launches(p, with_mask=True) == 4
+    assert binding.forward_launches(p, low_bit=True) == 6
+    assert binding.forward_launches(binding.problem(2, 40, 75600, 128, 128, 64, 0.05, 0.15)) == 5
     assert lib.sla_forward_launches(ctypes.byref(binding.problem(1, 1, 64, 96, 64, 64, 0.1, 0.1)), 0, 0) == -1
 
 
@@ -219,3 +214,26 @@ def test_backward_host_checks(lib):
     assert lib.sla_backward(ctypes.byref(pbq), *args, ws, size, null) == 2
     assert lib.sla_backward(ctypes.byref(p), null, *args[1:], ws, size, null) == 1
     assert lib.sla_backward(ctypes.byref(p), *args, ws, size - 1, null) == 3
+
+
+def test_pisa_host_checks(lib):
+    p = binding.problem(1, 2, 1000, 128, 128, 64, 0.25, 0.25)
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(64 << 20)
+    size = lib.sla_workspace_size_pisa(ctypes.byref(p))
+    # the forward's workspace plus centroid keys and values, per-part first-order sums and Hbar
+    a256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    BH, Nk, D = 2, 16, 128
+    parts = min(Nk, max(1, 148 // BH))
+    assert size == binding.workspace_size(p) + 2 * a256(BH * Nk * D * 2) + a256(BH * parts * D * D * 4) + \
+        a256(BH * D * D * 2)
+    out = ctypes.c_void_p(8 << 20)
+    assert lib.sla_forward_pisa(ctypes.byref(p), null, fake, fake, null, out, ws, size, null) == 1
+    assert lib.sla_forward_pisa(ctypes.byref(p), fake, fake, fake, null, fake, ws, size, null) == 1  # out aliases q
+    assert lib.sla_forward_pisa(ctypes.byref(p), fake, fake, fake, null, out, ws, size - 1, null) == 3
+    assert lib.sla_pisa_hbar(ctypes.byref(p), fake, fake, null, ws, size, null) == 1
+    assert lib.sla_pisa_hbar(ctypes.byref(p), fake, fake, out, ws, size - 1, null) == 3
+    bad = binding.problem(1, 2, 1000, 96, 128, 64, 0.25, 0.25)
+    assert lib.sla_workspace_size_pisa(ctypes.byref(bad)) == 0
+    assert lib.sla_forward_pisa(ctypes.byref(bad), fake, fake, fake, null, out, ws, size, null) == 2
