@@ -52,6 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the low-bit (e4m3) sparse-branch measurement")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
+    ap.add_argument("--no-pisa", action="store_true", help="skip the PISA variant measurement")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-configuration table (the other workloads, the kh sweep and its tail)")
     ap.add_argument("--config-steps", type=int, default=10, help="timed calls per configuration of that table")
@@ -110,8 +111,14 @@ def algorithmic_work(w, mask):
     # dK), four D x D products per row in the linear branch (G H^T, u^T G, phi(K) dh, V dh^T),
     # the transposed aggregation, and the row terms
     f_bwd = 2.5 * f_sparse + 4.0 * N * D * D * BH + f_agg + 8.0 * N * D * BH
+    # PISA with the same critical sets: the critical pairs, two D-products per row and
+    # non-critical block (its centroid's score and value sum), the first-order term per row, and
+    # the centred first-order matrices of the blocks
+    noncrit = (Nk - (mask == 2).sum(-1)).double().reshape(BH, Nq)
+    f_pisa = f_sparse + 4.0 * D * float(torch.einsum("i,bi->", qsize, noncrit).item()) + \
+        2.0 * N * D * D * BH + 2.0 * N * D * D * BH
     return {"flops": f_alg, "bytes": bytes_alg, "f_sparse": f_sparse, "f_attn_kernel": f_sparse + f_apply,
-            "f_states": f_states, "f_agg": f_agg, "f_router": f_router, "f_bwd": f_bwd}
+            "f_states": f_states, "f_agg": f_agg, "f_router": f_router, "f_bwd": f_bwd, "f_pisa": f_pisa}
 
 
 def max_over_ranks(x, dist=None, device="cpu"):
@@ -570,6 +577,30 @@ def run_ours(args):
                "timed_calls": n_b, "ratio_to_forward": round(ms_b / ms_step, 3)}
         del wsb, dO
 
+    # the PISA variant with the router's critical sets, same timing rules
+    pisa = None
+    if not args.no_pisa:
+        wsp = binding.new_workspace_pisa(p, dev)
+        times = []
+        n_p = min(args.steps, 20)
+        for it in range(3 + n_p):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            binding.forward_pisa(q, k, v, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=wsp)
+            e1.record(stream)
+            e1.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        binding.check(wsp)
+        ms_p = rank_max(sum(times) / len(times))
+        ach_p = work["f_pisa"] / (ms_p * 1e-3) / 1e12
+        pisa = {"call": "sla_forward_pisa", "ms_per_call": round(ms_p, 4),
+                "algorithmic_tflop": round(work["f_pisa"] / 1e12, 4), "achieved_tflops": round(ach_p, 2),
+                "frac_of_bf16_peak": round(ach_p / peaks["bf16_tflops"], 4), "labels": "the router's",
+                "timed_calls": n_p, "ratio_to_sla_forward": round(ms_p / ms_step, 3)}
+        del wsp
+
     # the other configurations: one table, same timing rules (c3 stays the headline value)
     configs = None
     if not args.no_configs:
@@ -605,7 +636,7 @@ def run_ours(args):
                             "launches sla_forward makes"},
         "roofline": roofline, "path_roofline": path_roofline,
         "clocks": clock_info, "e2e": e2e, "gpu_launches": binding.forward_launches(p) * args.steps,
-        "dense_reference": dense, "low_bit": low, "backward": bwd, "configs": configs, "cpu_baseline": cpu,
+        "dense_reference": dense, "low_bit": low, "backward": bwd, "pisa": pisa, "configs": configs, "cpu_baseline": cpu,
         "wall_s_timed": round(wall, 3),
     }
     print(json.dumps(line), flush=True)

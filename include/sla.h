@@ -155,7 +155,14 @@ sla_status sla_forward_fp8_timed(const sla_problem* p, const void* q, const void
                                  const float* alpha, const int8_t* mask, void* out, void* ws,
                                  size_t ws_bytes, void* stream, float* stage_ms);
 
-/* The K/V block quantiser of the low-bit branch on its own.
+/* Device addresses inside ws (sla_workspace_size_fp8(p) bytes) of the e4m3 codes of K and V
+ * ([B,H,N,D] uint8) and of their block exponents ([B,H,Nk] int32) that the last
+ * sla_forward_fp8 on this workspace wrote. Host only, nothing is enqueued. For tests and
+ * inspection. */
+sla_status sla_lowbit_codes(const sla_problem* p, void* ws, size_t ws_bytes, void** k8, void** v8, void** kexp,
+                            void** vexp);
+
+/* The K/V block quantiser of the low-bit branch on its own (the kernel sla_forward_fp8 runs).
  *   k, v                [B,H,N,D] bf16 device, 16-byte aligned
  *   k8_out, v8_out      [B,H,N,D] uint8 device e4m3 codes (8-byte aligned): sign bit 7,
  *                       exponent bits 3..6 (bias 7), mantissa bits 0..2; code * 2^exp
@@ -205,8 +212,9 @@ int sla_forward_launches(const sla_problem* p, int with_mask, int low_bit);
  *   blend          dalpha[h, :] = sum over rows of dO (O_s - O_l)
  * phi'(x) = 1 for x > 0, e^x otherwise. Operands enter the tensor cores in bf16 (G_s, the
  * softmax P and dS, phi(q), dnum = G_l / den, the per-block states and their gradients);
- * accumulation is fp32. The sparse branch's dK and dV are summed over query tiles with
- * fp32 global reductions (their order, and so the last bits, vary between runs).
+ * accumulation is fp32. Every sum runs in a fixed order (the sparse branch's dK and dV per KV
+ * block over the query tiles that hold it as critical, in ascending order; dalpha over the
+ * tiles), so two calls give identical results.
  *   q, k, v, dO   [B,H,N,D] bf16 device, 16-byte aligned
  *   alpha         [H,D] fp32 device
  *   mask          [B,H,Nq,Nk] int8 device labels of the forward (nullable: the router runs)

@@ -31,7 +31,7 @@ EXPORTS = ("sla_counts", "sla_workspace_size", "sla_route", "sla_kv_states", "sl
            "sla_selftest_wait_timeout", "sla_workspace_size_fp8", "sla_forward_fp8", "sla_forward_fp8_timed",
            "sla_quantize_kv", "sla_aggregate_states", "sla_forward_launches", "sla_route_variant",
            "sla_forward_variant", "sla_workspace_size_backward", "sla_backward", "sla_workspace_size_pisa",
-           "sla_forward_pisa", "sla_pisa_hbar")
+           "sla_forward_pisa", "sla_pisa_hbar", "sla_lowbit_codes")
 
 
 class SlaError(RuntimeError):
@@ -92,6 +92,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sla_workspace_size_pisa.restype = sz
         lib.sla_forward_pisa.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_pisa_hbar.argtypes = [P, vp, vp, vp, vp, sz, vp]
+        pp = ctypes.POINTER(ctypes.c_void_p)
+        lib.sla_lowbit_codes.argtypes = [P, vp, sz, pp, pp, pp, pp]
         V = ctypes.POINTER(Variant)
         lib.sla_route_variant.argtypes = [P, V, vp, vp, vp, vp, vp, vp, sz, vp]
         lib.sla_forward_variant.argtypes = [P, V, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -102,7 +104,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         for name in ("sla_counts", "sla_route", "sla_kv_states", "sla_forward", "sla_forward_timed", "sla_check",
                      "sla_forward_fp8", "sla_forward_fp8_timed", "sla_quantize_kv", "sla_forward_pisa",
                      "sla_pisa_hbar", "sla_aggregate_states", "sla_backward", "sla_route_variant",
-                     "sla_forward_variant"):
+                     "sla_forward_variant", "sla_lowbit_codes"):
             getattr(lib, name).restype = ctypes.c_int
         _lib = lib
         return lib
@@ -294,6 +296,24 @@ def backward(q, k, v, alpha, dO, block_q=128, block_kv=64, kh=0.05, kl=0.10, mas
                               _stream_handle(dev))
     _raise(st)
     return dQ, dK, dV, dalpha, ws
+
+
+def lowbit_codes(ws: torch.Tensor, B, H, N, D, block_q=128, block_kv=64):
+    """Copies of the e4m3 codes of K and V ([B,H,N,D] uint8) and block exponents ([B,H,Nk] int32)
+    that the last forward_fp8 on workspace ws wrote."""
+    p = problem(B, H, N, D, block_q, block_kv)
+    _, Nk, _, _ = counts(p)
+    ptrs = [ctypes.c_void_p() for _ in range(4)]
+    _raise(load_library().sla_lowbit_codes(ctypes.byref(p), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                                           *[ctypes.byref(x) for x in ptrs]))
+    base = ws.data_ptr()
+    out = []
+    for x, n, dt in ((ptrs[0], B * H * N * D, torch.uint8), (ptrs[1], B * H * N * D, torch.uint8),
+                     (ptrs[2], B * H * Nk, torch.int32), (ptrs[3], B * H * Nk, torch.int32)):
+        off = x.value - base
+        nbytes = n * (4 if dt == torch.int32 else 1)
+        out.append(ws[off:off + nbytes].view(dt).clone())
+    return (out[0].view(B, H, N, D), out[1].view(B, H, N, D), out[2].view(B, H, Nk), out[3].view(B, H, Nk))
 
 
 def new_workspace_pisa(p: Problem, device) -> torch.Tensor:

@@ -76,12 +76,6 @@ struct AttnArgs {
   uint32_t* err;
 };
 
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 template <int D>
 struct AttnSmem {
   static constexpr uint32_t Q = 128 * D * 2;       // Q tile (rewritten as phi(Q) at the end of a tile)

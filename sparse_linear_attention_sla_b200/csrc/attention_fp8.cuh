@@ -22,18 +22,28 @@
 //       of block j contributes e4m3(2^(x - r) * 2^(ev_j - ev_max)) <= 256 < 448 with ev_max
 //       the largest V exponent of the tile's critical blocks; the normaliser l sums the
 //       unquantised 2^(x - r).
-//   O_s = 2^ev_max * acc / l.
+//   O_s = 2^c acc / l with c = ev_max - kP8RefExp.
+//
+// The linear branch shares the sparse branch's accumulator as in attn_kernel: with H~_i =
+// H_i diag((1 - alpha) / alpha) from the aggregation,
+//     O = alpha (2^c acc / l + phi(q) H~_i / den) = alpha 2^c (acc + (l 2^-c / den) phi(q) H~_i) / l,
+// so the warpgroup writes P_lin = (l 2^-c / den) phi(q) (bf16) into TMEM and one bf16 MMA
+// adds P_lin H~_i into acc; with no critical block l = 1 and c = 0.
 //
 // Persistent, two CTAs per SM (<= 100 KB shared memory, 256 TMEM columns each). Warp roles
 // (192 threads):
 //   warp 0      TMA producer: per tile the bf16 Q tile, then K8_j / V8_j of every critical
-//               block through a 3-slot ring, then H_i as two pseudo-blocks (rows 0..63 and
-//               64..127, each filling a whole slot).
+//               block through a 3-slot ring, then H~_i as two pseudo-blocks (rows 0..63 and
+//               64..127, each filling a whole slot). The next tile's Q is loaded once the
+//               warpgroup has read this one for phi(q).
 //   warp 1      TMEM owner and single-thread tcgen05 issuer.
 //   warps 2..5  softmax / epilogue warpgroup: a thread owns one query row (= TMEM lane).
+//               The output is staged in the two H~_i slots and written by TMA stores; the
+//               slots return to the ring when the stores have read them (next tile).
 //
 // TMEM columns: S ping-pong [0,64) [64,128) (P8, 16 columns, is written over the first
-// columns of its S), O_s [128,256); after the sparse loop O_l reuses [0,128).
+// columns of its S), acc [128,256); after the sparse loop P_lin (64 columns) takes the S
+// columns the next block would have used.
 #pragma once
 
 #include "attention.cuh"
@@ -70,19 +80,19 @@ struct AttnFp8Smem {
 __global__ void __launch_bounds__(192, 2)
     attn_fp8_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k8,
                     const __grid_constant__ CUtensorMap map_v8, const __grid_constant__ CUtensorMap map_h,
-                    AttnFp8Args a) {
+                    const __grid_constant__ CUtensorMap map_o, AttnFp8Args a) {
   using L = AttnFp8Smem;
   constexpr int D = 128;
   constexpr int NS = L::NSLOT;
   constexpr uint32_t TMEM_COLS = 256;
-  constexpr uint32_t OS = 128, OL = 0;
+  constexpr uint32_t OS = 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQb = base;
   uint8_t* sQ8 = sQb + L::QB;
   uint8_t* sRing = sQ8 + L::Q8;  // slot s at sRing + s * SLOT: K8 at +0, V8 at +KV
 
-  __shared__ uint64_t q_full, q8_full, q_free, phiq_full, ol_done, tmem_free, drain;
+  __shared__ uint64_t q_full, q8_full, q_free, plin_full, lin_done, tmem_free, drain;
   __shared__ uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
   __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
   __shared__ uint32_t tmem_base_sh;
@@ -97,9 +107,9 @@ __global__ void __launch_bounds__(192, 2)
   if (tid == 0) {
     mbar_init(&q_full, 1);
     mbar_init(&q8_full, 128);
-    mbar_init(&q_free, 1);
-    mbar_init(&phiq_full, 128);
-    mbar_init(&ol_done, 1);
+    mbar_init(&q_free, 128);     // every row read for phi(q)
+    mbar_init(&plin_full, 128);
+    mbar_init(&lin_done, 1);
     mbar_init(&tmem_free, 128);
     mbar_init(&drain, 1);
     for (int s = 0; s < NS; ++s) {
@@ -125,7 +135,7 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  grid_dep_wait();  // critical lists, H_i, Z_i and the K/V codes come from earlier kernels
+  grid_dep_wait();  // critical lists, H~_i, Z_i and the K/V codes come from earlier kernels
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -134,6 +144,7 @@ __global__ void __launch_bounds__(192, 2)
       prefetch_tmap(&map_k8);
       prefetch_tmap(&map_v8);
       prefetch_tmap(&map_h);
+      prefetch_tmap(&map_o);
       int k_round[NS], v_round[NS];
       for (int s = 0; s < NS; ++s) k_round[s] = v_round[s] = -1;
       int q_loads = 0;
@@ -189,13 +200,16 @@ __global__ void __launch_bounds__(192, 2)
       const uint32_t id_s = idesc_e4m3_f32(128, 64, 0, 0);
       const uint32_t id_pv = idesc_e4m3_f32(128, D, 0, 1);
       const uint32_t id_ol = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t qb0 = smem_u32(sQb), q80 = smem_u32(sQ8), ring0 = smem_u32(sRing);
+      const uint32_t q80 = smem_u32(sQ8), ring0 = smem_u32(sRing);
       uint32_t nb = 0, ns = 0;  // ring uses, S/P blocks
       bool ok = true;
-      // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites O_s. V8 is
-      // MN-major: rows of 128 codes (one swizzle atom wide), K = 32 rows = 4096 bytes a step.
+      int k = 0;
+      // P*V of the block at ring use nbm, S/P index nsm; `first` overwrites acc, which the
+      // previous tile's epilogue must have read (tile k > 0). V8 is MN-major: rows of 128
+      // codes (one swizzle atom wide), K = 32 rows = 4096 bytes a step.
       auto issue_pv = [&](uint32_t nbm, uint32_t nsm, bool first) -> bool {
         const int s = static_cast<int>(nbm % NS), b = nsm & 1;
+        if (first && k > 0 && !mbar_wait(&tmem_free, (k - 1) & 1, a.err, &abort_flag)) return false;
         if (!mbar_wait(&p_full[b], (nsm >> 1) & 1, a.err, &abort_flag)) return false;
         if (!mbar_wait(&v_full[s], (nbm / NS) & 1, a.err, &abort_flag)) return false;
         tc_fence_after();
@@ -209,13 +223,10 @@ __global__ void __launch_bounds__(192, 2)
         umma_commit(&v_empty[s]);
         return true;
       };
-      int k = 0;
       for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x, ++k) {
         const int kc = a.crit_cnt[t];
         // the warpgroup has written this tile's e4m3 Q
         if (!(ok = mbar_wait(&q8_full, k & 1, a.err, &abort_flag))) break;
-        // the epilogue of the previous tile has read O_s and O_l out of TMEM
-        if (k > 0 && !(ok = mbar_wait(&tmem_free, (k - 1) & 1, a.err, &abort_flag))) break;
         for (int n = 0; n < kc; ++n, ++nb, ++ns) {
           const int s = static_cast<int>(nb % NS), b = ns & 1;
           if (!(ok = mbar_wait(&k_full[s], (nb / NS) & 1, a.err, &abort_flag))) break;
@@ -233,28 +244,26 @@ __global__ void __launch_bounds__(192, 2)
         }
         if (!ok) break;
         if (kc > 0 && !(ok = issue_pv(nb - 1, ns - 1, kc == 1))) break;
-        // linear branch: O_l = phi(Q) H_i once both halves of H_i have landed and the
-        // warpgroup rewrote the bf16 Q tile as phi(Q)
+        // Linear branch, added into the sparse accumulator: acc += P_lin H~_i, P_lin written
+        // by the warpgroup into the S columns after the last block (ns & 1), H~_i in two ring
+        // slots (rows 0..63, 64..127). With no critical block this is the first write of acc.
+        // The slots are released by the warpgroup once the output staged there is stored.
         const int s0 = static_cast<int>(nb % NS), s1 = static_cast<int>((nb + 1) % NS);
+        if (kc == 0 && k > 0 && !(ok = mbar_wait(&tmem_free, (k - 1) & 1, a.err, &abort_flag))) break;
         if (!(ok = mbar_wait(&k_full[s0], (nb / NS) & 1, a.err, &abort_flag))) break;
         if (!(ok = mbar_wait(&v_full[s0], (nb / NS) & 1, a.err, &abort_flag))) break;
         if (!(ok = mbar_wait(&k_full[s1], ((nb + 1) / NS) & 1, a.err, &abort_flag))) break;
         if (!(ok = mbar_wait(&v_full[s1], ((nb + 1) / NS) & 1, a.err, &abort_flag))) break;
-        if (!(ok = mbar_wait(&phiq_full, k & 1, a.err, &abort_flag))) break;
+        if (!(ok = mbar_wait(&plin_full, k & 1, a.err, &abort_flag))) break;
         tc_fence_after();
+        const uint32_t pl = tmem + (ns & 1) * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(qb0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
           const uint32_t hb = ring0 + (kk < 4 ? s0 : s1) * L::SLOT;
           const uint64_t bd = smem_desc_sw128(hb + (kk & 3) * 2048, 8192, 1024);
-          umma_bf16_ss(tmem + OL, ad, bd, id_ol, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + OS, pl + kk * 8, bd, id_ol, (kc > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&ol_done);
-        umma_commit(&q_free);
-        umma_commit(&k_empty[s0]);
-        umma_commit(&v_empty[s0]);
-        umma_commit(&k_empty[s1]);
-        umma_commit(&v_empty[s1]);
+        umma_commit(&lin_done);
         nb += 2;
       }
       umma_commit(&drain);  // every MMA issued above has finished once this arrives
@@ -267,7 +276,9 @@ __global__ void __launch_bounds__(192, 2)
     const int r = quarter * 32 + lane;          // query row within the tile
     const int wt = tid - 64;                    // 0..127
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint32_t ns = 0;  // S/P blocks so far
+    uint32_t ns = 0;   // S/P blocks so far
+    uint32_t nbw = 0;  // ring uses so far (K/V blocks and H~_i halves)
+    int rel0 = -1, rel1 = -1;  // (thread 0 of the warpgroup) ring slots still held by an output store
     bool ok = true;
     int k = 0;
     // Every barrier of the warpgroup ANDs the threads' status, so a failed wait makes all
@@ -275,6 +286,9 @@ __global__ void __launch_bounds__(192, 2)
     for (int t = blockIdx.x; t < a.n_tiles; t += gridDim.x, ++k) {
       const int bh = t / a.Nq, i = t % a.Nq, h = bh % a.H;
       const int kc = a.crit_cnt[t];
+      // the ring slots of this tile's H~_i halves, reused to stage O
+      const int hs0 = static_cast<int>((nbw + kc) % NS), hs1 = static_cast<int>((nbw + kc + 1) % NS);
+      nbw += kc + 2;
       const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
       const int32_t* kexp = a.kexp + static_cast<size_t>(bh) * a.Nk;
       const int32_t* vexp = a.vexp + static_cast<size_t>(bh) * a.Nk;
@@ -282,6 +296,16 @@ __global__ void __launch_bounds__(192, 2)
       const bool row_valid = r < a.block_q && tok < a.N;
       // The previous tile is done with sZ, sAlpha and the parity-(k+1) reduction slots.
       if (!named_barrier_and(1, 128, ok)) break;
+      // The previous tile's output has been read out of its two slots once this thread's bulk
+      // group is done reading: the slots may take K8/V8 blocks again.
+      if (rel0 >= 0) {
+        tma_store_wait_read();
+        mbar_arrive(&k_empty[rel0]);
+        mbar_arrive(&v_empty[rel0]);
+        mbar_arrive(&k_empty[rel1]);
+        mbar_arrive(&v_empty[rel1]);
+        rel0 = rel1 = -1;
+      }
       const int par = k & 1;
       if (wt == 0) {
         sQmax[par ^ 1] = 0u;
@@ -310,7 +334,7 @@ __global__ void __launch_bounds__(192, 2)
         if (kc > 0) atomicMax(&sVmax[par], vmax_l);
       }
       sZ[wt] = z_in;
-      sAlpha[wt] = al_in;
+      sAlpha[wt] = fmaxf(al_in, kAlphaFloor);  // H~_i was scaled with the same floor
       if (!named_barrier_and(1, 128, ok)) break;
       const int eq = pow2_scale_exp(__uint_as_float(sQmax[par] << 16));
       const int vmax = sVmax[par];
@@ -454,28 +478,32 @@ __global__ void __launch_bounds__(192, 2)
         ek_cur = ek_next;
         ev_cur = ev_next;
       }
-      // Every MMA that reads the S/P columns has finished once the last PV has.
-      if (ok && kc > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
-
-      // phi(Q) in place over the bf16 tile, and the linear-branch denominator phi(q) . Z_i
-      // with the same rounded phi(q) the MMA sees (as in attn_kernel).
+      // Linear branch. P_lin goes into the S columns the next block would have used
+      // (ns & 1); their last reader is the P*V two blocks back (with one block or none, an
+      // MMA of an earlier tile, finished before that tile's lin_done was seen).
+      if (ok && kc >= 2)
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 2) & 1], ((ns - 2) >> 1) & 1, a.err, &abort_flag));
+      // Pass 1: phi(q) (bf16, as the tensor core takes it) into the P_lin columns, 32 elements
+      // at a time, and den = phi(q) . Z_i from those rounded values; then the bf16 Q tile is
+      // released (the next tile's Q may land).
+      const uint32_t pl = lane_addr + (ns & 1) * 64;
       uint64_t den2 = 0ull;
       if (ok) {
         const uint64_t one2 = f2_make(1.f, 1.f), log2e2 = f2_make(1.4426950408889634f, 1.4426950408889634f);
-#pragma unroll 2
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          uint4* p = reinterpret_cast<uint4*>(sQb + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
-          uint4 u = *p;
-          uint32_t w[4] = {u.x, u.y, u.z, u.w};
-          const uint4 z01 = *reinterpret_cast<const uint4*>(&sZ[c8 * 8]);
-          const uint4 z23 = *reinterpret_cast<const uint4*>(&sZ[c8 * 8 + 4]);
-          const uint64_t z2[4] = {static_cast<uint64_t>(z01.x) | (static_cast<uint64_t>(z01.y) << 32),
-                                  static_cast<uint64_t>(z01.z) | (static_cast<uint64_t>(z01.w) << 32),
-                                  static_cast<uint64_t>(z23.x) | (static_cast<uint64_t>(z23.y) << 32),
-                                  static_cast<uint64_t>(z23.z) | (static_cast<uint64_t>(z23.w) << 32)};
+#pragma unroll 1
+        for (int g = 0; g < D / 32; ++g) {
+          uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int c = 0; c < 4; ++c) {
+            const int c8 = 4 * g + c;
+            const uint4 u = *reinterpret_cast<const uint4*>(sQb + (c8 >> 3) * 16384 + sw128_offset(r, (c8 & 7) * 16));
+            w[4 * c] = u.x;
+            w[4 * c + 1] = u.y;
+            w[4 * c + 2] = u.z;
+            w[4 * c + 3] = u.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
             const uint64_t x2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
             const uint64_t pos2 = f2_add(x2, one2);
             const uint64_t t2 = f2_mul(x2, log2e2);
@@ -483,50 +511,83 @@ __global__ void __launch_bounds__(192, 2)
             const float g1 = f2_hi(x2) > 0.f ? f2_hi(pos2) : fast_exp2(f2_hi(t2));
             w[e] = pack_bf16x2(g0, g1);
             const uint64_t gr2 = static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32);
-            den2 = f2_fma(gr2, z2[e], den2);
+            den2 = f2_fma(gr2, *reinterpret_cast<const uint64_t*>(&sZ[32 * g + 2 * e]), den2);
           }
-          *p = make_uint4(w[0], w[1], w[2], w[3]);
+          tmem_st16(pl + 16 * g, w);
         }
-        fence_proxy_async_smem();
       }
+      mbar_arrive(&q_free);
+      // With no critical block l is taken as 1 and c as 0 (acc starts at 0); with no marginal
+      // block (den = 0) the linear term is 0.
       const float den_tot = f2_lo(den2) + f2_hi(den2);
+      const int cexp = kc > 0 ? vmax - kP8RefExp : 0;
+      const float l_eff = kc > 0 ? l_run : 1.f;
+      const float c_lin = den_tot > 0.f ? mul_pow2(l_eff, -cexp) / den_tot : 0.f;
+      // Pass 2: P_lin = (l 2^-c / den) phi(q), rounded to bf16 in place.
+      if (ok) {
+        tmem_wait_st();
+        const uint64_t c2 = f2_make(c_lin, c_lin);
+#pragma unroll 1
+        for (int g = 0; g < D / 64; ++g) {
+          uint32_t w[32];
+          tmem_ld32(pl + 32 * g, w);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const uint64_t g2 = f2_mul(c2, static_cast<uint64_t>(w[e] << 16) | (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32));
+            w[e] = pack_bf16x2(f2_lo(g2), f2_hi(g2));
+          }
+          tmem_st32(pl + 32 * g, w);
+        }
+        tmem_wait_st();
+      }
       tc_fence_before();
-      mbar_arrive(&phiq_full);
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, k & 1, a.err, &abort_flag));
+      mbar_arrive(&plin_full);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&lin_done, k & 1, a.err, &abort_flag));
       if (!(ok = named_barrier_and(1, 128, ok))) break;
 
-      // Epilogue: O = alpha * O_s + (1 - alpha) * O_l / den, with O_s = 2^(vmax - kP8RefExp) acc / l.
+      // Epilogue: O = alpha 2^c acc / l in bf16, staged row by row in the two H~_i slots (the
+      // linear MMA has read them; columns 0..63 in the first, 64..127 in the second) in the
+      // 128-byte swizzle and written by TMA stores of block_q rows (rows past N are clipped by
+      // the tensor map; with block_q = 64 the upper 64 rows belong to the next query block).
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? mul_pow2(1.f / l_run, vmax - kP8RefExp) : 0.f;
-      const float inv_d = den_tot > 0.f ? 1.f / den_tot : 0.f;
-      __nv_bfloat16* orow = a.out + (static_cast<size_t>(bh) * a.N + tok) * D;
-      const uint64_t il2 = f2_make(inv_l, inv_l), id2 = f2_make(inv_d, inv_d);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t os[16], ol[16];
-        if (kc > 0) tmem_ld16(lane_addr + OS + c0, os);
-        tmem_ld16(lane_addr + OL + c0, ol);
-        tmem_wait_ld();
-        uint32_t pk[8];
+      const float inv_l = mul_pow2(1.f / l_eff, cexp);
+      const uint64_t il2 = f2_make(inv_l, inv_l);
+      uint32_t ob[2][32];
+      tmem_ld32(lane_addr + OS, ob[0]);
+      tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; c += 2) {
-          const uint64_t al2 = *reinterpret_cast<const uint64_t*>(&sAlpha[c0 + c]);
-          const uint64_t wl = f2_fma(al2 ^ 0x8000000080000000ull, id2, id2);  // (1 - alpha) inv_d
-          uint64_t y = f2_mul(wl, static_cast<uint64_t>(ol[c]) | (static_cast<uint64_t>(ol[c + 1]) << 32));
-          if (kc > 0)
-            y = f2_fma(f2_mul(al2, il2), static_cast<uint64_t>(os[c]) | (static_cast<uint64_t>(os[c + 1]) << 32), y);
+      for (int q = 0; q < D / 32; ++q) {
+        if (q + 1 < D / 32) tmem_ld32(lane_addr + OS + 32 * (q + 1), ob[(q + 1) & 1]);
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const uint64_t al2 = *reinterpret_cast<const uint64_t*>(&sAlpha[32 * q + c]);
+          const uint64_t y = f2_mul(f2_mul(al2, il2), static_cast<uint64_t>(ob[q & 1][c]) |
+                                                          (static_cast<uint64_t>(ob[q & 1][c + 1]) << 32));
           pk[c >> 1] = pack_bf16x2(f2_lo(y), f2_hi(y));
         }
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
+        uint8_t* box = sRing + ((q >> 1) == 0 ? hs0 : hs1) * L::SLOT;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<uint4*>(box + sw128_offset(r, ((q & 1) * 4 + v) * 16)) =
+              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        if (q + 1 < D / 32) tmem_wait_ld();
+      }
+      fence_proxy_async_smem();
+      named_barrier(1, 128);
+      if (wt == 0) {
+        tma_store_3d(&map_o, sRing + hs0 * L::SLOT, 0, i * a.block_q, bh);
+        tma_store_3d(&map_o, sRing + hs1 * L::SLOT, 64, i * a.block_q, bh);
+        tma_store_commit();
+        rel0 = hs0;  // released at the next tile's start (see there)
+        rel1 = hs1;
       }
       tc_fence_before();
-      mbar_arrive(&tmem_free);  // O_s and O_l have left TMEM: the next tile may overwrite them
+      mbar_arrive(&tmem_free);  // the accumulator has left TMEM: the next tile may overwrite it
     }
   }
+  if (tid == 64) tma_store_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

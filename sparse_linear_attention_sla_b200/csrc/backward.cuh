@@ -10,11 +10,9 @@
 //            dH_i = u^T dnum  (tcgen05),  dZ_i = u^T dden   (written stacked, [dH_i | dZ_i],
 //            for the aggregation run backwards)
 //   pass 2 (the critical blocks again): P = 2^(S log2e - LSE), dP = G_s V_j^T,
-//            dS = P (dP - Delta) / sqrt(D);
-//            dQ += dS K_j (accumulated in TMEM over the blocks),
-//            dV_j += P^T G_s, dK_j += dS^T Q (tcgen05 into TMEM as dV_j^T, dK_j^T, then
-//            added into the fp32 gradients with coalesced global reductions: a KV block
-//            is critical for several query tiles)
+//            dS = P (dP - Delta) / sqrt(D); dQ += dS K_j (accumulated in TMEM over the
+//            blocks). LSE and Delta of every row are written out: the KV-block pass
+//            (bwd_kv_kernel) recomputes P and dS from them for dK_j and dV_j.
 //
 // Source: "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable Sparse-Linear
 // Attention", Abstract (one kernel covers forward and backward). The formulas are the exact
@@ -29,9 +27,9 @@
 //   warps 2..5  thread = query row = TMEM lane for the row-wise work; for dH_i the TMEM lane
 //               is a channel
 // TMEM (512 columns): pass 1 S [0,64) [64,128), acc [128,256); linear O_l [256,384),
-// dnum H^T [384,512), dH [0,128); pass 2 S [0,64), dP [64,128), dV^T [128,192),
-// dK^T [192,256), dQ [256,384).
-// Shared memory: Q, G_s, U (phi(Q); in pass 2 P and dS), dnum: 32 KB each; ring 2 x 32 KB.
+// dnum H^T [384,512), dH [0,128); pass 2 S / dP pairs [0,128) [128,256) (S at +0, dP at
+// +64), dQ [256,384).
+// Shared memory: Q, G_s, U (phi(Q); in pass 2 dS), dnum: 32 KB each; ring 2 x 32 KB.
 #pragma once
 
 #include "sm100.cuh"
@@ -47,17 +45,13 @@ struct BwdArgs {
   const float* alpha;       // [H, D]
   const __nv_bfloat16* dO;  // [BH, N, D]
   float* dQ;                // [BH, N, D]   written
-  float* dK;                // [BH, N, D]   added into (global reductions)
-  float* dV;                // [BH, N, D]   added into
-  float* dalpha;            // [H, D]       added into
+  float* lse;               // [BH, N]      written: log2-sum-exp of the row's critical scores
+  float* delta;             // [BH, N]      written: rowsum(G_s * O_s)
+  float* dalpha_part;       // [n_tiles, D] written: the tile's sum over rows of dO (O_s - O_l)
   __nv_bfloat16* dHst;      // [BH*Nq, LD]  written: dH_i row-major (D*D), then dZ_i (D), then 0
   float scale_log2;         // log2(e) / sqrt(D)
   uint32_t* err;
 };
-
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
 
 __global__ void __launch_bounds__(192, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_g,
@@ -69,16 +63,15 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = base;
   uint8_t* sG = base + TILE;
-  uint8_t* sU = base + 2 * TILE;   // phi(Q); in pass 2: P [128 x 64] at +0, dS [128 x 64] at +16384
+  uint8_t* sU = base + 2 * TILE;   // phi(Q); in pass 2: dS [128 x 64] at +16384
   uint8_t* sDn = base + 3 * TILE;  // dnum
   uint8_t* sRing = base + 4 * TILE;
-  uint8_t* sP = sU;
   uint8_t* sdS = sU + 16384;
 
   __shared__ uint64_t q_full, q_free, u_full, ol_done, dn_full, lin_done, t1_free, tile_done;
   __shared__ uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
   __shared__ uint64_t s_full[2], p_full[2], pv_done[2];
-  __shared__ uint64_t s2_full, ds_full, g2_done, dkv_free, drain;
+  __shared__ uint64_t s2_full[2], ds_full, g2_done, drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
   __shared__ __align__(16) float sZ[D];
@@ -105,10 +98,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&p_full[s], 128);
       mbar_init(&pv_done[s], 1);
     }
-    mbar_init(&s2_full, 1);
+    mbar_init(&s2_full[0], 1);
+    mbar_init(&s2_full[1], 1);
     mbar_init(&ds_full, 128);
     mbar_init(&g2_done, 1);
-    mbar_init(&dkv_free, 128);
     mbar_init(&drain, 1);
     abort_flag = 0;
     fence_mbar_init();
@@ -186,9 +179,8 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t id_s = idesc_bf16_f32(128, 64, 0, 0);   // A, B K-major, N = 64
     const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);    // A K-major, B MN-major, N = D
     const uint32_t id_t = idesc_bf16_f32(128, D, 1, 1);    // A, B MN-major, N = D
-    const uint32_t id_t64 = idesc_bf16_f32(128, 64, 1, 1); // A, B MN-major, N = 64
     const uint32_t q0 = smem_u32(sQ), g0 = smem_u32(sG), u0 = smem_u32(sU), dn0 = smem_u32(sDn);
-    const uint32_t ring0 = smem_u32(sRing), p0 = smem_u32(sP), ds0 = smem_u32(sdS);
+    const uint32_t ring0 = smem_u32(sRing), ds0 = smem_u32(sdS);
     uint32_t nb = 0, ns = 0;
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -270,39 +262,38 @@ __global__ void __launch_bounds__(192, 1)
       commit(&k_empty[sh]);
       commit(&v_empty[sh]);
       ++nb;
-      // ---- pass 2
+      // ---- pass 2: S, dP of block n into the pair (n2 & 1), then dQ += dS K of block n - 1
       if (!(ok = wait_all(&t1_free, k & 1))) break;  // dH, O_l, dnum H^T and acc have left TMEM
+      // dQ += dS K_j of the pass-2 block at ring use nbm, pass-2 index m (the tile's first
+      // when `first`); frees the block's ring slot and the dS tile
+      auto issue_dq = [&](uint32_t nbm, int m, bool first) -> bool {
+        if (!wait_all(&ds_full, m & 1)) return false;
+        tc_fence_after();
+        const uint32_t kb = ring0 + (nbm & 1) * SLOT;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // K = 64 keys
+          mma_ss(tmem + 256, smem_desc_sw128(ds0 + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 2048, 8192, 1024),
+                 id_o, (!first || kk > 0) ? 1u : 0u);
+        commit(&g2_done);
+        commit(&k_empty[nbm & 1]);
+        commit(&v_empty[nbm & 1]);
+        return true;
+      };
       for (int n = 0; n < kc; ++n, ++nb, ++n2) {
-        const int s = nb & 1;
+        const int s = nb & 1, b = n2 & 1;
         if (!(ok = wait_all(&k_full[s], (nb >> 1) & 1))) break;
         if (!(ok = wait_all(&v_full[s], (nb >> 1) & 1))) break;
-        if (n2 > 0 && !(ok = wait_all(&ds_full, (n2 - 1) & 1))) break;  // S, dP of the last block were read
         tc_fence_after();
         const uint32_t kb = ring0 + s * SLOT, vb = kb + KV;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem, kmaj128(q0, kk), kmaj64(kb, kk), id_s, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem + b * 128, kmaj128(q0, kk), kmaj64(kb, kk), id_s, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem + 64, kmaj128(g0, kk), kmaj64(vb, kk), id_s, kk > 0);
-        commit(&s2_full);
-        // P and dS of this block in shared memory; dV^T and dK^T free again
-        if (!(ok = wait_all(&ds_full, n2 & 1))) break;
-        if (n2 > 0 && !(ok = wait_all(&dkv_free, (n2 - 1) & 1))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // dV^T = G_s^T P, dK^T = Q^T dS (K = 128 rows)
-          mma_ss(tmem + 128, smem_desc_sw128(g0 + kk * 2048, 16384, 1024), smem_desc_sw128(p0 + kk * 2048, 8192, 1024),
-                 id_t64, kk > 0);
-          mma_ss(tmem + 192, smem_desc_sw128(q0 + kk * 2048, 16384, 1024), smem_desc_sw128(ds0 + kk * 2048, 8192, 1024),
-                 id_t64, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)  // dQ += dS K_j (K = 64 keys)
-          mma_ss(tmem + 256, smem_desc_sw128(ds0 + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 2048, 8192, 1024),
-                 id_o, (n > 0 || kk > 0) ? 1u : 0u);
-        commit(&g2_done);
-        commit(&k_empty[s]);
-        commit(&v_empty[s]);
+        for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem + b * 128 + 64, kmaj128(g0, kk), kmaj64(vb, kk), id_s, kk > 0);
+        commit(&s2_full[b]);
+        if (n >= 1 && !(ok = issue_dq(nb - 1, n2 - 1, n == 1))) break;
       }
+      if (!ok) break;
+      if (kc > 0 && !(ok = issue_dq(nb - 1, n2 - 1, kc == 1))) break;
       if (!ok) break;
       commit(&q_free);
     }
@@ -460,11 +451,15 @@ __global__ void __launch_bounds__(192, 1)
         fence_proxy_async_smem();
       }
       const float dden = -dden_acc * inv_den;
+      if (row_ok) {  // for the KV-block pass
+        a.lse[static_cast<size_t>(bh) * a.N + tok] = lse;
+        a.delta[static_cast<size_t>(bh) * a.N + tok] = delta;
+      }
       sDden[r] = dden;
       tc_fence_before();
       mbar_arrive(&dn_full);
       if (!(ok = named_barrier_and(1, 128, ok))) break;  // sRed, sDden complete
-      red_add_f32(&a.dalpha[h * D + wt], sRed[0][wt] + sRed[1][wt] + sRed[2][wt] + sRed[3][wt]);
+      a.dalpha_part[static_cast<size_t>(t) * D + wt] = sRed[0][wt] + sRed[1][wt] + sRed[2][wt] + sRed[3][wt];
       ok = __all_sync(0xffffffffu, mbar_wait(&lin_done, k & 1, a.err, &abort_flag));
       if (ok) {
         tc_fence_after();
@@ -530,59 +525,39 @@ __global__ void __launch_bounds__(192, 1)
       for (int n = 0; ok && n < kc; ++n, ++n2) {
         const int j = clist[n];
         const int valid = min(64, a.N - j * 64);
-        ok = __all_sync(0xffffffffu, mbar_wait(&s2_full, n2 & 1, a.err, &abort_flag));
-        // P and dS may overwrite their tiles once the previous block's MMAs have read them
-        if (ok && n2 > 0) ok = __all_sync(0xffffffffu, mbar_wait(&g2_done, (n2 - 1) & 1, a.err, &abort_flag));
+        const int b = n2 & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s2_full[b], (n2 >> 1) & 1, a.err, &abort_flag));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sx[32], dp[32];
+        uint32_t dk[32];
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(lane_addr + 32 * hh, sx);
-          tmem_ld32(lane_addr + 64 + 32 * hh, dp);
+          uint32_t sx[32], dp[32];
+          tmem_ld32(lane_addr + b * 128 + 32 * hh, sx);
+          tmem_ld32(lane_addr + b * 128 + 64 + 32 * hh, dp);
           tmem_wait_ld();
-          uint32_t pk[16], dk[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const int n0 = 32 * hh + c;
             const float p0 = (row_ok && n0 < valid) ? exp2f(__uint_as_float(sx[c]) * sc - lse_r) : 0.f;
             const float p1 = (row_ok && n0 + 1 < valid) ? exp2f(__uint_as_float(sx[c + 1]) * sc - lse_r) : 0.f;
-            pk[c >> 1] = pack_bf16x2(p0, p1);
-            dk[c >> 1] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - delta) * dsc,
-                                     p1 * (__uint_as_float(dp[c + 1]) - delta) * dsc);
-          }
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint32_t off = sw128_offset(r, (4 * hh + v) * 16);
-            *reinterpret_cast<uint4*>(sP + off) = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-            *reinterpret_cast<uint4*>(sdS + off) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+            dk[16 * hh + (c >> 1)] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - delta) * dsc,
+                                                 p1 * (__uint_as_float(dp[c + 1]) - delta) * dsc);
           }
         }
+        // dS may overwrite its tile once the previous block's dQ MMAs have read it
+        if (n2 > 0) ok = __all_sync(0xffffffffu, mbar_wait(&g2_done, (n2 - 1) & 1, a.err, &abort_flag));
+        if (!ok) break;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          *reinterpret_cast<uint4*>(sdS + sw128_offset(r, v * 16)) =
+              make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&ds_full);
-        // dV_j^T, dK_j^T (lane = channel d) into the fp32 gradients
-        ok = __all_sync(0xffffffffu, mbar_wait(&g2_done, n2 & 1, a.err, &abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        const size_t row0 = static_cast<size_t>(bh) * a.N + static_cast<size_t>(j) * 64;
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          tmem_ld32(lane_addr + 128 + 32 * hh, sx);
-          tmem_ld32(lane_addr + 192 + 32 * hh, dp);
-          tmem_wait_ld();
-#pragma unroll 4
-          for (int c = 0; c < 32; ++c) {
-            const int nn = 32 * hh + c;
-            if (nn < valid) {
-              red_add_f32(a.dV + (row0 + nn) * D + r, __uint_as_float(sx[c]));
-              red_add_f32(a.dK + (row0 + nn) * D + r, __uint_as_float(dp[c]));
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&dkv_free);
       }
+      // the tile's last dQ MMAs are done
+      if (ok && kc > 0) ok = __all_sync(0xffffffffu, mbar_wait(&g2_done, (n2 - 1) & 1, a.err, &abort_flag));
       // ---- dQ += the sparse part accumulated in TMEM (the last pass-2 MMAs are done)
       if (ok && kc > 0) {
         tc_fence_after();
@@ -615,6 +590,17 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// dalpha[h, :] = sum over the batch entries b and query tiles i, in that order, of the tiles'
+// partial sums (bh = b * H + h). grid H, block D.
+__global__ void __launch_bounds__(128) dalpha_kernel(const float* __restrict__ part, float* __restrict__ dalpha, int B,
+                                                     int H, int Nq) {
+  const int h = blockIdx.x, d = threadIdx.x, D = blockDim.x;
+  float s = 0.f;
+  for (int b = 0; b < B; ++b)
+    for (int i = 0; i < Nq; ++i) s += part[(static_cast<size_t>(b * H + h) * Nq + i) * D + d];
+  dalpha[h * D + d] = s;
 }
 
 }  // namespace sla

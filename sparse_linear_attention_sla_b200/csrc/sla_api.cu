@@ -15,6 +15,7 @@
 #include "attention.cuh"
 #include "attention_fp8.cuh"
 #include "backward.cuh"
+#include "backward_kv.cuh"
 #include "backward_states.cuh"
 #include "fp8.cuh"
 #include "pisa.cuh"
@@ -116,6 +117,11 @@ struct Workspace {
   __nv_bfloat16* WT;    // marginal indicator transposed [BH, Nk, wt_ld]
   __nv_bfloat16* dh;    // [BH, Nk, D*D] gradients of the per-block states
   float* dz;            // [BH, Nk, D]
+  float* lse;           // [BH, N] log2-sum-exp of each row's critical scores
+  float* delta;         // [BH, N] rowsum(G_s * O_s)
+  float* dalpha_part;   // [BH * Nq, D] per-tile partial sums of dalpha
+  int32_t* tlist;       // [BH * Nk, Nq] query tiles holding each KV block as critical
+  int32_t* tcnt;        // [BH * Nk]
   int wt_ld;
   // low-bit sparse branch only
   uint8_t* k8;     // e4m3 codes of K [BH, N, D]
@@ -163,6 +169,11 @@ Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false, bool bwd = fal
     w.WT = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(w.wt_ld) * 2));
     w.dh = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(s.D) * s.D * 2));
     w.dz = reinterpret_cast<float*>(take(BH * s.Nk * s.D * sizeof(float)));
+    w.lse = reinterpret_cast<float*>(take(BH * s.N * sizeof(float)));
+    w.delta = reinterpret_cast<float*>(take(BH * s.N * sizeof(float)));
+    w.dalpha_part = reinterpret_cast<float*>(take(BH * s.Nq * s.D * sizeof(float)));
+    w.tlist = reinterpret_cast<int32_t*>(take(BH * s.Nk * s.Nq * sizeof(int32_t)));
+    w.tcnt = reinterpret_cast<int32_t*>(take(BH * s.Nk * sizeof(int32_t)));
   }
   if (fp8) {
     w.k8 = take(BH * s.N * static_cast<size_t>(s.D));
@@ -514,21 +525,19 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
 
 template <int D>
 sla_status launch_quant(const Shape& s, const void* k, const void* v, uint8_t* k8, uint8_t* v8, int32_t* kexp,
-                        int32_t* vexp, cudaStream_t st, bool dependent) {
+                        int32_t* vexp, cudaStream_t st) {
   const dim3 grid(s.Nk, s.BH);
   auto kb = static_cast<const __nv_bfloat16*>(k);
   auto vb = static_cast<const __nv_bfloat16*>(v);
-  if (dependent)
-    return launch_dependent(sla::quant_kv_kernel<D>, grid, dim3(256), 0, st, "quant_kv_kernel", kb, vb, k8, v8, kexp,
-                            vexp, s.N, s.Nk);
   sla::quant_kv_kernel<D><<<grid, 256, 0, st>>>(kb, vb, k8, v8, kexp, vexp, s.N, s.Nk);
   return launched("quant_kv_kernel");
 }
 
 sla_status launch_attn_fp8(const Shape& s, const void* q, const float* alpha, void* out, const Workspace& w,
                            int crit_ld, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mh;
+  CUtensorMap mq, mk, mv, mh, mo;
   SLA_TRY(act_map(&mq, q, s, 128));
+  SLA_TRY(act_map(&mo, out, s, static_cast<uint32_t>(s.bq)));  // boxes of block_q rows, as in launch_attn
   SLA_TRY(code_map(&mk, w.k8, s, 64));
   SLA_TRY(code_map(&mv, w.v8, s, 64));
   {
@@ -558,7 +567,7 @@ sla_status launch_attn_fp8(const Shape& s, const void* q, const float* alpha, vo
   a.err = w.err;
   const int grid = a.n_tiles < 2 * sm_count() ? a.n_tiles : 2 * sm_count();
   return launch_dependent(sla::attn_fp8_kernel, dim3(grid), dim3(192), smem, st, "attn_fp8_kernel", mq, mk, mv, mh,
-                          a);
+                          mo, a);
 }
 
 // ------------------------------------------------------------------ entry points (templated on D)
@@ -578,10 +587,6 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
                          const int8_t* mask, const void* dO, float* dQ, float* dK, float* dV, float* dalpha,
                          const Workspace& w, cudaStream_t st) {
   constexpr int D = 128;
-  const size_t act_f32 = static_cast<size_t>(s.BH) * s.N * D * sizeof(float);
-  SLA_CUDA(cudaMemsetAsync(dK, 0, act_f32, st));
-  SLA_CUDA(cudaMemsetAsync(dV, 0, act_f32, st));
-  SLA_CUDA(cudaMemsetAsync(dalpha, 0, static_cast<size_t>(s.H) * D * sizeof(float), st));
   // states, labels and H_i, Z_i as in the forward (H_i unscaled)
   sla::PrepArgs pa{};
   pa.BH = s.BH;
@@ -608,7 +613,7 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
   sla::gs_kernel<<<4 * sm_count(), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(dO), alpha, w.gs, s.H, s.N, D,
                                                   chunks);
   SLA_TRY(launched("gs_kernel"));
-  // per query tile: dQ, dalpha, dH_i / dZ_i, and the sparse branch's dK, dV
+  // per query tile: dQ, the tile's dalpha sums, dH_i / dZ_i, and each row's LSE and Delta
   {
     CUtensorMap mq, mg, mk, mv, mh;
     SLA_TRY(act_map(&mq, q, s, 128));
@@ -632,9 +637,9 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
     a.alpha = alpha;
     a.dO = static_cast<const __nv_bfloat16*>(dO);
     a.dQ = dQ;
-    a.dK = dK;
-    a.dV = dV;
-    a.dalpha = dalpha;
+    a.lse = w.lse;
+    a.delta = w.delta;
+    a.dalpha_part = w.dalpha_part;
     a.dHst = w.dHst;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
     a.err = w.err;
@@ -648,20 +653,43 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
                                                                                            w.WT, w.wt_ld);
   SLA_TRY(launched("w_transpose_kernel"));
   SLA_TRY(launch_agg_gemm<D>(s.Nk, s.Nq, s.BH, s.LD, w.WT, w.wt_ld, w.dHst, w.dh, w.dz, w.err, nullptr, s.H, st));
-  // the states' part of dK, dV
+  sla::dalpha_kernel<<<s.H, D, 0, st>>>(w.dalpha_part, dalpha, s.B, s.H, s.Nq);
+  SLA_TRY(launched("dalpha_kernel"));
+  // per KV block: the sparse branch's dK_j, dV_j over the tiles holding it as critical, plus
+  // the states' part
+  sla::crit_transpose_kernel<<<dim3((s.Nk + 127) / 128, s.BH), 128, 0, st>>>(mask ? mask : w.mask, s.Nq, s.Nk,
+                                                                             w.tlist, w.tcnt);
+  SLA_TRY(launched("crit_transpose_kernel"));
   {
-    CUtensorMap mk, mv, mdh;
+    CUtensorMap mq, mg, mk, mv, mdh;
+    SLA_TRY(act_map(&mq, q, s, 128));
+    SLA_TRY(act_map(&mg, w.gs, s, 128));
     SLA_TRY(act_map(&mk, k, s, 64));
     SLA_TRY(act_map(&mv, v, s, 64));
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(D), static_cast<uint64_t>(s.BH) * s.Nk};
     const uint64_t strides[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(D) * D};
     const uint32_t box[3] = {64, 128, 1};
     SLA_TRY(make_map(&mdh, w.dh, 3, dims, strides, box));
-    sla::BwdStatesArgs a{s.BH, s.N, s.Nk, w.dz, dK, dV, w.err};
-    const int smem = 65536 + 1024;
-    SLA_TRY(allow_smem(sla::bwd_states_kernel, smem));
-    SLA_TRY(launch_dependent(sla::bwd_states_kernel, dim3(s.BH * s.Nk), dim3(192), smem, st, "bwd_states_kernel", mk,
-                             mv, mdh, a));
+    sla::BwdKVArgs a{};
+    a.BH = s.BH;
+    a.N = s.N;
+    a.Nq = s.Nq;
+    a.Nk = s.Nk;
+    a.tlist = w.tlist;
+    a.tcnt = w.tcnt;
+    a.lse = w.lse;
+    a.delta = w.delta;
+    a.dz = w.dz;
+    a.dK = dK;
+    a.dV = dV;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    a.err = w.err;
+    constexpr int smem = sla::BwdKVSmem::total();
+    SLA_TRY(allow_smem(sla::bwd_kv_kernel, smem));
+    const int blocks = s.BH * s.Nk;
+    const int grid = blocks < sm_count() ? blocks : sm_count();
+    SLA_TRY(launch_dependent(sla::bwd_kv_kernel, dim3(grid), dim3(192), smem, st, "bwd_kv_kernel", mq, mg, mk, mv,
+                             mdh, a));
   }
   return SLA_OK;
 }
@@ -820,9 +848,6 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
   pa.hst = w.hst;
   pa.LD = s.LD;
   pa.err = w.err;
-  // the bf16 attention adds the linear branch into its accumulator and takes H_i scaled per
-  // channel by (1 - alpha) / alpha; the low-bit kernel takes H_i as it is
-  const float* agg_alpha = fp8 ? nullptr : alpha;
   SLA_TRY(ev.mark(0, st));
   SLA_TRY(launch_prep<D>(q, k, v, s, pa, st));
   SLA_TRY(ev.mark(1, st));
@@ -834,16 +859,16 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
     SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
   }
   SLA_TRY(ev.mark(2, st));
-  SLA_TRY(launch_agg<D>(s, w, agg_alpha, st));
+  // both attention kernels add the linear branch into their accumulator and take H_i scaled
+  // per channel by (1 - alpha) / alpha
+  SLA_TRY(launch_agg<D>(s, w, alpha, st));
   SLA_TRY(ev.mark(3, st));
   if (fp8) {
-    if constexpr (D == 128) {
-      SLA_TRY(launch_quant<D>(s, k, v, w.k8, w.v8, w.kexp, w.vexp, st, true));
-      SLA_TRY(ev.mark(4, st));
-      SLA_TRY(launch_attn_fp8(s, q, alpha, out, w, s.Nk, st));
-      return ev.mark(5, st);
-    }
-    return fail(SLA_ERR_UNSUPPORTED, "the low-bit sparse branch needs D=128");
+    if constexpr (D != 128) return fail(SLA_ERR_UNSUPPORTED, "the low-bit sparse branch needs D=128");
+    SLA_TRY(launch_quant<D>(s, k, v, w.k8, w.v8, w.kexp, w.vexp, st));
+    SLA_TRY(ev.mark(4, st));
+    SLA_TRY(launch_attn_fp8(s, q, alpha, out, w, s.Nk, st));
+    return ev.mark(5, st);
   }
   SLA_TRY(launch_attn<D>(s, q, k, v, alpha, out, w, s.Nk, st));
   return ev.mark(4, st);
@@ -1027,8 +1052,8 @@ sla_status sla_quantize_kv(const sla_problem* p, const void* k, const void* v, u
       reinterpret_cast<uintptr_t>(vexp_out) % 4)
     return fail(SLA_ERR_INVALID_ARG, "kexp_out and vexp_out must be non-NULL and 4-byte aligned");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (s.D == 64) return launch_quant<64>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st, false);
-  return launch_quant<128>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st, false);
+  if (s.D == 64) return launch_quant<64>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st);
+  return launch_quant<128>(s, k, v, k8_out, v8_out, kexp_out, vexp_out, st);
 }
 
 sla_status sla_aggregate_states(const sla_problem* p, const void* k, const void* v, const int8_t* mask,
@@ -1114,6 +1139,20 @@ sla_status sla_forward_variant(const sla_problem* p, const sla_variant* variant,
   }
   if (var.fm) return forward_variant_impl<128, 1>(s, var, q, k, v, alpha, mask, out, w, st);
   return forward_variant_impl<128, 0>(s, var, q, k, v, alpha, mask, out, w, st);
+}
+
+sla_status sla_lowbit_codes(const sla_problem* p, void* ws, size_t ws_bytes, void** k8, void** v8, void** kexp,
+                            void** vexp) {
+  Shape s;
+  SLA_TRY(make_shape(p, &s));
+  if (!k8 || !v8 || !kexp || !vexp) return fail(SLA_ERR_INVALID_ARG, "output pointers must be non-NULL");
+  Workspace w;
+  SLA_TRY(check_ws(s, ws, ws_bytes, &w, true));
+  *k8 = w.k8;
+  *v8 = w.v8;
+  *kexp = w.kexp;
+  *vexp = w.vexp;
+  return SLA_OK;
 }
 
 size_t sla_workspace_size_pisa(const sla_problem* p) {

@@ -164,7 +164,7 @@ def test_route_noalloc_refuses_oversize_problem(lib):
 
 def test_forward_launch_counts(lib):
     """One launch per stage: precompute, labels (the router's scores and selection, or the
-    caller mask's lists), aggregation, attention (and the quantiser for the low-bit call)."""
+    caller mask's lists), aggregation, attention, and the K/V quantiser for the low-bit call."""
     p = binding.problem(1, 12, 32760, 128, 128, 64, 0.05, 0.1)
     assert binding.forward_launches(p) == 5
     assert binding.forward_launches(p, with_mask=True) == 4

@@ -28,6 +28,8 @@ def test_work_of_a_ragged_labelled_problem():
     assert work["f_router"] == 2 * (N * D + 3 * 3 * D)
     # backward: five products per critical pair, four D x D products per row, the aggregation
     assert work["f_bwd"] == 10 * D * pairs + 4 * N * D * D + 3 * D * D + 8 * N * D
+    # PISA: non-critical blocks per row 2, 2, 1 over rows of 64, 64, 22
+    assert work["f_pisa"] == 4 * D * pairs + 4 * D * (64 * 2 + 64 * 2 + 22 * 1) + 4 * N * D * D
     expected = 4 * D * pairs + 2 * N * D * D + 2 * N * D * D + 3 * D * D + 2 * (N * D + 9 * D) + 3 * N * D
     assert work["flops"] == expected
     assert work["bytes"] == 8 * N * D + 9 + 1 * D * 4

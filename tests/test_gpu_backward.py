@@ -96,3 +96,18 @@ def test_backward_wan13b_sampled(cuda_device):
         _check(f"dQ h{h}", dQ[:, sl].cpu(), rQ)
         _check(f"dK h{h}", dK[:, sl].cpu(), rK)
         _check(f"dV h{h}", dV[:, sl].cpu(), rV)
+
+
+@pytest.mark.parametrize("case", [(1, 2, 1024, 0.25, 0.25), (1, 3, 4113, 0.1, 0.2)], ids=lambda c: "x".join(map(str, c)))
+def test_backward_is_deterministic(cuda_device, case):
+    """Every sum of the backward runs in a fixed order (no atomics): two calls agree bit for bit."""
+    B, H, N, kh, kl = case
+    q, k, v, alpha = random_inputs(B, H, N, 128, seed=N, device=cuda_device)
+    g = torch.Generator(device=cuda_device).manual_seed(N + 1)
+    dO = torch.randn(B, H, N, 128, generator=g, device=cuda_device).to(torch.bfloat16)
+    first = binding.backward(q, k, v, alpha, dO, 128, 64, kh, kl)
+    second = binding.backward(q, k, v, alpha, dO, 128, 64, kh, kl)
+    binding.check(first[4])
+    binding.check(second[4])
+    for name, a, b in zip(("dQ", "dK", "dV", "dalpha"), first[:4], second[:4]):
+        assert torch.equal(a, b), f"{name} differs between two calls"

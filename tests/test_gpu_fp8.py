@@ -80,6 +80,23 @@ def test_quantize_kv_bit_exact(cuda_device, N, D):
             np.testing.assert_array_equal(f8.e4m3_decode(codes[0, h]), vals)
 
 
+@pytest.mark.parametrize("N", [1000, 4096 + 17])
+def test_forward_fp8_codes_equal_quantiser(cuda_device, N):
+    """The codes the low-bit forward leaves in its workspace are the standalone quantiser's, bit for bit."""
+    B, H, D = 1, 2, 128
+    q, k, v, alpha = random_inputs(B, H, N, D, seed=N, device="cpu")
+    k = _rescale_blocks(k, N, -6, 6)
+    v = _rescale_blocks(v, N + 1, -6, 6)
+    q, k, v, alpha = (t.to(cuda_device) for t in (q, k, v, alpha))
+    ws = binding.new_workspace(binding.problem(B, H, N, D, 128, 64, 0.25, 0.25), cuda_device, fp8=True)
+    binding.forward_fp8(q, k, v, alpha, 128, 64, 0.25, 0.25, ws=ws)
+    binding.check(ws)
+    got = binding.lowbit_codes(ws, B, H, N, D)
+    ref = binding.quantize_kv(k, v)
+    for g, r in zip(got, ref):
+        assert torch.equal(g.cpu(), r.cpu())
+
+
 FP8_CASES = [
     # B, H, N, bq, kh, kl
     (1, 2, 1000, 128, 0.25, 0.25),
