@@ -318,7 +318,8 @@ __global__ void __launch_bounds__(192, 1)
       sZ[wt] = a.Zagg[static_cast<size_t>(t) * D + wt];
       sAl[wt] = a.alpha[h * D + wt];
       if (!named_barrier_and(1, 128, ok)) break;
-      // ---- pass 1: online softmax (exact maximum per block; rescale whenever it grows)
+      // ---- pass 1: online softmax as in the forward (the running maximum is moved, and the
+      // accumulator rescaled, only when a block's maximum passes it by more than 2^8)
       float m_run = -INFINITY, l_run = 0.f;
       for (int n = 0; ok && n < kc; ++n, ++ns) {
         const int b = ns & 1;
@@ -326,44 +327,69 @@ __global__ void __launch_bounds__(192, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (ns >> 1) & 1, a.err, &abort_flag));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sx[64];
-        tmem_ld32(lane_addr + b * 64, *reinterpret_cast<uint32_t(*)[32]>(&sx[0]));
-        tmem_ld32(lane_addr + b * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sx[32]));
+        uint32_t sa[32], sb[32];
+        tmem_ld32(lane_addr + b * 64, sa);
+        tmem_ld32(lane_addr + b * 64 + 32, sb);
         tmem_wait_ld();
-        float mx = -INFINITY;
+        if (valid < 64) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < valid) mx = fmaxf(mx, __uint_as_float(sx[c]));
-        mx *= sc;
-        const float m_new = fmaxf(m_run, mx);
-        if (n > 0 && __any_sync(0xffffffffu, m_new > m_run)) {
+          for (int c = 0; c < 32; ++c) {
+            if (c >= valid) sa[c] = __float_as_uint(-INFINITY);
+            if (c + 32 >= valid) sb[c] = __float_as_uint(-INFINITY);
+          }
+        }
+        float m0 = fmax3(__uint_as_float(sa[0]), __uint_as_float(sa[1]), __uint_as_float(sa[2]));
+        float m1 = fmax3(__uint_as_float(sb[0]), __uint_as_float(sb[1]), __uint_as_float(sb[2]));
+#pragma unroll
+        for (int c = 3; c < 31; c += 2) {
+          m0 = fmax3(m0, __uint_as_float(sa[c]), __uint_as_float(sa[c + 1]));
+          m1 = fmax3(m1, __uint_as_float(sb[c]), __uint_as_float(sb[c + 1]));
+        }
+        m0 = fmaxf(m0, __uint_as_float(sa[31]));
+        m1 = fmaxf(m1, __uint_as_float(sb[31]));
+        const float mx = fmaxf(m0, m1) * sc;
+        if (n == 0) {
+          m_run = mx;
+        } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
           ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
           if (!ok) break;
           tc_fence_after();
-          const float f = exp2f(m_run - m_new);
+          const float m_new = fmaxf(m_run, mx);
+          const float f = fast_exp2(m_run - m_new);
+          const uint64_t f2 = f2_make(f, f);
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
             tmem_ld32(lane_addr + 128 + c0, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+            for (int c = 0; c < 32; c += 2) {
+              const uint64_t y = f2_mul(static_cast<uint64_t>(o[c]) | (static_cast<uint64_t>(o[c + 1]) << 32), f2);
+              o[c] = static_cast<uint32_t>(y);
+              o[c + 1] = static_cast<uint32_t>(y >> 32);
+            }
             tmem_st32(lane_addr + 128 + c0, o);
           }
           tmem_wait_st();
           l_run *= f;
+          m_run = m_new;
         }
-        m_run = m_new;
+        const uint64_t sc2 = f2_make(sc, sc), nm2 = f2_make(-m_run, -m_run);
+        uint64_t ps2 = 0ull, ps2b = 0ull;
         uint32_t pk[32];
-        float ps = 0.f;
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float e0 = c < valid ? exp2f(__uint_as_float(sx[c]) * sc - m_run) : 0.f;
-          const float e1 = c + 1 < valid ? exp2f(__uint_as_float(sx[c + 1]) * sc - m_run) : 0.f;
+        for (int c = 0; c < 32; c += 2) {
+          const uint64_t x2 = f2_fma(static_cast<uint64_t>(sa[c]) | (static_cast<uint64_t>(sa[c + 1]) << 32), sc2, nm2);
+          const uint64_t y2 = f2_fma(static_cast<uint64_t>(sb[c]) | (static_cast<uint64_t>(sb[c + 1]) << 32), sc2, nm2);
+          const float e0 = fast_exp2(f2_lo(x2)), e1 = fast_exp2(f2_hi(x2));
+          const float e2 = fast_exp2(f2_lo(y2)), e3 = fast_exp2(f2_hi(y2));
+          ps2 = f2_add(ps2, f2_make(e0, e1));
+          ps2b = f2_add(ps2b, f2_make(e2, e3));
           pk[c >> 1] = pack_bf16x2(e0, e1);
-          ps += e0 + e1;
+          pk[16 + (c >> 1)] = pack_bf16x2(e2, e3);
         }
-        l_run += ps;
+        const uint64_t pst = f2_add(ps2, ps2b);
+        l_run += f2_lo(pst) + f2_hi(pst);
         tmem_st32(lane_addr + b * 64, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -521,7 +547,9 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(&t1_free);
       // ---- pass 2
       const float lse_r = lse;
-      const float dsc = sc * kLn2;  // 1 / sqrt(D)
+      const uint64_t sc2 = f2_make(sc, sc);
+      const float shift = log2f(sc * kLn2) - lse_r;  // log2(1 / sqrt(D)) - LSE
+      const uint64_t sh2 = f2_make(shift, shift), nd2 = f2_make(-delta, -delta);
       for (int n = 0; ok && n < kc; ++n, ++n2) {
         const int j = clist[n];
         const int valid = min(64, a.N - j * 64);
@@ -536,13 +564,16 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32(lane_addr + b * 128 + 32 * hh, sx);
           tmem_ld32(lane_addr + b * 128 + 64 + 32 * hh, dp);
           tmem_wait_ld();
+          // P / sqrt(D) = 2^(S log2(e) / sqrt(D) - LSE + log2(1 / sqrt(D))); dS = (P / sqrt(D)) (dP - Delta)
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const int n0 = 32 * hh + c;
-            const float p0 = (row_ok && n0 < valid) ? exp2f(__uint_as_float(sx[c]) * sc - lse_r) : 0.f;
-            const float p1 = (row_ok && n0 + 1 < valid) ? exp2f(__uint_as_float(sx[c + 1]) * sc - lse_r) : 0.f;
-            dk[16 * hh + (c >> 1)] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - delta) * dsc,
-                                                 p1 * (__uint_as_float(dp[c + 1]) - delta) * dsc);
+            const uint64_t x2 = f2_fma(static_cast<uint64_t>(sx[c]) | (static_cast<uint64_t>(sx[c + 1]) << 32), sc2, sh2);
+            const float p0 = (row_ok && n0 < valid) ? fast_exp2(f2_lo(x2)) : 0.f;
+            const float p1 = (row_ok && n0 + 1 < valid) ? fast_exp2(f2_hi(x2)) : 0.f;
+            const uint64_t d2 = f2_add(static_cast<uint64_t>(dp[c]) | (static_cast<uint64_t>(dp[c + 1]) << 32), nd2);
+            const uint64_t g2 = f2_mul(f2_make(p0, p1), d2);
+            dk[16 * hh + (c >> 1)] = pack_bf16x2(f2_lo(g2), f2_hi(g2));
           }
         }
         // dS may overwrite its tile once the previous block's dQ MMAs have read it
@@ -592,15 +623,26 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-// dalpha[h, :] = sum over the batch entries b and query tiles i, in that order, of the tiles'
-// partial sums (bh = b * H + h). grid H, block D.
-__global__ void __launch_bounds__(128) dalpha_kernel(const float* __restrict__ part, float* __restrict__ dalpha, int B,
-                                                     int H, int Nq) {
-  const int h = blockIdx.x, d = threadIdx.x, D = blockDim.x;
+// dalpha[h, :] = sum over the (batch entry, query tile) pairs of head h of the tiles' partial
+// sums: eight interleaved partial sums per channel, then added in a fixed order.
+// grid (H, D / 32), block (32, 8).
+__global__ void __launch_bounds__(256) dalpha_kernel(const float* __restrict__ part, float* __restrict__ dalpha, int B,
+                                                     int H, int Nq, int D) {
+  __shared__ float red[8][32];
+  const int h = blockIdx.x, d = blockIdx.y * 32 + threadIdx.x, g = threadIdx.y;
   float s = 0.f;
-  for (int b = 0; b < B; ++b)
-    for (int i = 0; i < Nq; ++i) s += part[(static_cast<size_t>(b * H + h) * Nq + i) * D + d];
-  dalpha[h * D + d] = s;
+  for (int u = g; u < B * Nq; u += 8) {
+    const int b = u / Nq, i = u % Nq;
+    s += part[(static_cast<size_t>(b * H + h) * Nq + i) * D + d];
+  }
+  red[g][threadIdx.x] = s;
+  __syncthreads();
+  if (g == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) t += red[q][threadIdx.x];
+    dalpha[h * D + d] = t;
+  }
 }
 
 }  // namespace sla

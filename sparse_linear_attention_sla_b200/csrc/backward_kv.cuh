@@ -230,6 +230,7 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     const float sc = a.scale_log2;
     const float dsc = sc * 0.6931471805599453f;  // 1 / sqrt(D)
+    const uint64_t sc2 = f2_make(sc, sc), dsc2 = f2_make(dsc, dsc);
     uint32_t ns = 0;
     bool ok = true;
     int nkv = 0;
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(192, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (ns >> 1) & 1, a.err, &abort_flag));
         if (!ok) break;
         tc_fence_after();
+        const uint64_t nl2 = f2_make(-lse, -lse), nd2 = f2_make(-dl, -dl);
         uint32_t pk[32], dk[32];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -265,11 +267,13 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const int n0 = 32 * hh + c;
-            const float p0 = (row_ok && n0 < valid) ? fast_exp2(fmaf(__uint_as_float(sx[c]), sc, -lse)) : 0.f;
-            const float p1 = (row_ok && n0 + 1 < valid) ? fast_exp2(fmaf(__uint_as_float(sx[c + 1]), sc, -lse)) : 0.f;
+            const uint64_t x2 = f2_fma(static_cast<uint64_t>(sx[c]) | (static_cast<uint64_t>(sx[c + 1]) << 32), sc2, nl2);
+            const float p0 = (row_ok && n0 < valid) ? fast_exp2(f2_lo(x2)) : 0.f;
+            const float p1 = (row_ok && n0 + 1 < valid) ? fast_exp2(f2_hi(x2)) : 0.f;
             pk[16 * hh + (c >> 1)] = pack_bf16x2(p0, p1);
-            dk[16 * hh + (c >> 1)] = pack_bf16x2(p0 * (__uint_as_float(dp[c]) - dl) * dsc,
-                                                 p1 * (__uint_as_float(dp[c + 1]) - dl) * dsc);
+            const uint64_t d2 = f2_add(static_cast<uint64_t>(dp[c]) | (static_cast<uint64_t>(dp[c + 1]) << 32), nd2);
+            const uint64_t g2 = f2_mul(f2_mul(f2_make(p0, p1), dsc2), d2);
+            dk[16 * hh + (c >> 1)] = pack_bf16x2(f2_lo(g2), f2_hi(g2));
           }
         }
         // P and dS may overwrite their tiles once the previous tile's dV^T, dK^T MMAs are done

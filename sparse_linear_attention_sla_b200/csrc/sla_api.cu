@@ -653,7 +653,7 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
                                                                                            w.WT, w.wt_ld);
   SLA_TRY(launched("w_transpose_kernel"));
   SLA_TRY(launch_agg_gemm<D>(s.Nk, s.Nq, s.BH, s.LD, w.WT, w.wt_ld, w.dHst, w.dh, w.dz, w.err, nullptr, s.H, st));
-  sla::dalpha_kernel<<<s.H, D, 0, st>>>(w.dalpha_part, dalpha, s.B, s.H, s.Nq);
+  sla::dalpha_kernel<<<dim3(s.H, D / 32), dim3(32, 8), 0, st>>>(w.dalpha_part, dalpha, s.B, s.H, s.Nq, D);
   SLA_TRY(launched("dalpha_kernel"));
   // per KV block: the sparse branch's dK_j, dV_j over the tiles holding it as critical, plus
   // the states' part

@@ -364,19 +364,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe (no MUFU), for x <= 126; 0 below -125. x = n + f with n the nearest
-// integer (adding 1.5 * 2^23 leaves it in the low mantissa bits) and f in [-1/2, 1/2]; 2^f
-// by a cubic fitted for this file (weighted least squares on Chebyshev nodes of [-1/2, 1/2]:
-// relative error below 7.5e-5); n is then added to the exponent field.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float t = xc + 12582912.f;
-  const float f = xc - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.05517162f, f, 0.24261113f), f, 0.69326097f), f, 0.99992806f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -125.f ? 0.f : r;
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
