@@ -285,3 +285,20 @@ def test_mutation_route2_sample_variance(monkeypatch):
 
     monkeypatch.setattr(r2, "block_variance", sample_var)
     assert _fails(pinsr.test_score_matches_the_exact_block_mean_to_fourth_order)
+
+
+# ---------------------------------------------------------------- the dropped-linear-branch forward
+
+def test_mutation_dropped_forward_renormalised(monkeypatch):
+    # dividing by alpha's channel mean (renormalising what is left) must fail a pin
+    from oracle import sla_oracle_salad as sd
+    from tests import test_oracle_salad_pins as pins
+    plain = sd.forward_dropped
+
+    def renormalised(q, k, v, alpha, *args, **kw):
+        a = np.asarray(alpha, dtype=np.float64)
+        return plain(q, k, v, alpha, *args, **kw) / a.mean(axis=-1)[None, :, None, None]
+
+    monkeypatch.setattr(sd, "forward_dropped", renormalised)
+    with pytest.raises(AssertionError):
+        pins.test_every_block_critical_is_alpha_times_dense_attention()
