@@ -243,10 +243,20 @@ sla_status sla_backward(const sla_problem* p, const void* q, const void* k, cons
  *                   log: S2_ij = qbar_i . kbar_j / sqrt(D) + log1p(sum_d qbar_i,d^2 var_j,d / (2 D)),
  *                   var_j,d the population variance of channel d over the block's valid
  *                   keys; labels from S2 with the same total order and counts.
+ * and the post-tuning branch dropping of "SALAD: Achieve High-Sparsity Attention via Efficient
+ * Linear Attention Tuning for Video Diffusion Transformer" §2:
+ *   linear_scale, drop_threshold  the model's dynamic scale s of the linear branch at this
+ *                   step and the threshold tau_t (both from the caller; the library computes
+ *                   neither). When s < tau_t the linear branch is not run (no states, no
+ *                   aggregation) and O = alpha * O_s; otherwise the forward is SLA's (s does
+ *                   not scale the branch). Zero for both (a zero-initialised struct) keeps
+ *                   the branch. Must be finite.
  * The sparse branch and the blend are those of sla_forward. */
 typedef struct {
   int feature_map;
   int block_score;
+  float linear_scale;
+  float drop_threshold;
 } sla_variant;
 
 /* sla_route with a variant's block score. scores_out (nullable) receives the variant's
@@ -256,8 +266,8 @@ sla_status sla_route_variant(const sla_problem* p, const sla_variant* variant, c
                              int8_t* mask_out, int32_t* crit_idx_out, double* scores_out, void* ws,
                              size_t ws_bytes, void* stream);
 
-/* sla_forward with a variant's block score (when mask is NULL) and feature map. Arguments as
- * for sla_forward; the workspace of sla_workspace_size serves. */
+/* sla_forward with a variant's block score (when mask is NULL), feature map and branch
+ * dropping. Arguments as for sla_forward; the workspace of sla_workspace_size serves. */
 sla_status sla_forward_variant(const sla_problem* p, const sla_variant* variant, const void* q, const void* k,
                                const void* v, const float* alpha, const int8_t* mask, void* out, void* ws,
                                size_t ws_bytes, void* stream);

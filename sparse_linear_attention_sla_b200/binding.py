@@ -41,8 +41,10 @@ class SlaError(RuntimeError):
 
 
 class Variant(ctypes.Structure):
-    """sla_variant: feature_map 0 (elu + 1) or 1 (exp); block_score 0 (first order) or 1 (second order)."""
-    _fields_ = [("feature_map", ctypes.c_int), ("block_score", ctypes.c_int)]
+    """sla_variant: feature_map 0 (elu + 1) or 1 (exp); block_score 0 (first order) or 1 (second order);
+    linear_scale, drop_threshold: the linear branch is dropped when linear_scale < drop_threshold."""
+    _fields_ = [("feature_map", ctypes.c_int), ("block_score", ctypes.c_int), ("linear_scale", ctypes.c_float),
+                ("drop_threshold", ctypes.c_float)]
 
 
 class Problem(ctypes.Structure):
@@ -244,7 +246,7 @@ def route_variant(q, k, block_q, block_kv, kh, kl, feature_map=0, block_score=0,
     scores = torch.empty(B, H, Nq, Nk, dtype=torch.float64, device=dev) if want_scores else None
     if ws is None:
         ws = new_workspace(p, dev)
-    var = Variant(feature_map, block_score)
+    var = Variant(feature_map, block_score, 0.0, 0.0)
     lib = load_library()
     with torch.cuda.device(dev):
         st = lib.sla_route_variant(ctypes.byref(p), ctypes.byref(var), _ptr(q), _ptr(k), _ptr(mask), _ptr(crit),
@@ -254,10 +256,10 @@ def route_variant(q, k, block_q, block_kv, kh, kl, feature_map=0, block_score=0,
 
 
 def forward_variant(q, k, v, alpha, block_q, block_kv, kh, kl, feature_map=0, block_score=0, mask=None, out=None,
-                    ws=None):
+                    ws=None, linear_scale=0.0, drop_threshold=0.0):
     """sla_forward_variant: O [B,H,N,D] bf16."""
     p, out, ws = _forward_args(q, k, v, alpha, block_q, block_kv, kh, kl, mask, out, ws)
-    var = Variant(feature_map, block_score)
+    var = Variant(feature_map, block_score, float(linear_scale), float(drop_threshold))
     lib = load_library()
     dev = q.device
     with torch.cuda.device(dev):

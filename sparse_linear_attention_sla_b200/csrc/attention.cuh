@@ -65,11 +65,12 @@ namespace sla {
 struct AttnArgs {
   int H, N, Nq, block_q, n_tiles;
   int Nk, nc, n_last;       // PISA: KV blocks, centroid pseudo-blocks (ceil(Nk / 64)), keys of the last block
+  int h_mode;               // the H~ tile of tile t: 0 row t * D (per query block), 1 row bh * D (per head), 2 row 0 (one tile)
   float inv_sqrt_d;         // PISA: 1 / sqrt(D)
   const int32_t* crit;      // [BH*Nq, crit_ld] critical KV block indices, ascending
   int crit_ld;
   const int32_t* crit_cnt;  // [BH*Nq]
-  const float* Zagg;        // [BH*Nq, D]
+  const float* Zagg;        // [BH*Nq, D] (nullable: Z_i = 0, no linear term)
   const float* alpha;       // [H, D]
   __nv_bfloat16* out;       // [BH, N, D]
   float scale_log2;         // log2(e) / sqrt(D)
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(192, 2)
         const int kc = a.crit_cnt[t];
         const int nblk = kc + (PISA ? a.nc : 0);  // blocks of the softmax: critical, then centroid
         const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
-        const int h_row = (PISA ? bh : t) * D;   // first row of this tile's H~ (per head for PISA)
+        const int h_row = (a.h_mode == 0 ? t : (a.h_mode == 1 ? bh : 0)) * D;  // first row of this tile's H~
         if (k > 0 && !(ok = mbar_wait(&q_free, (k - 1) & 1, a.err, &abort_flag))) break;
         mbar_arrive_expect_tx(&q_full, L::Q);
         for (int b = 0; b < DB; ++b) tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * a.block_q, bh);
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(192, 2)
     // during the current tile so that their latency stays off the tile boundary.
     float z_next = 0.f, a_next = 1.f;
     if (!PISA && wt < D && static_cast<int>(blockIdx.x) < a.n_tiles) {
-      z_next = a.Zagg[static_cast<size_t>(blockIdx.x) * D + wt];
+      if (a.Zagg) z_next = a.Zagg[static_cast<size_t>(blockIdx.x) * D + wt];
       a_next = a.alpha[(blockIdx.x / a.Nq % a.H) * D + wt];
     }
     // Every barrier of the warpgroup ANDs the threads' status, so a failed wait makes all
@@ -340,7 +341,7 @@ __global__ void __launch_bounds__(192, 2)
       }
       if (!PISA && wt < D && t + static_cast<int>(gridDim.x) < a.n_tiles) {
         const int tn = t + gridDim.x;
-        z_next = a.Zagg[static_cast<size_t>(tn) * D + wt];
+        if (a.Zagg) z_next = a.Zagg[static_cast<size_t>(tn) * D + wt];
         a_next = a.alpha[(tn / a.Nq % a.H) * D + wt];
       }
       float m_run = -INFINITY, l_run = 0.f;  // running max (scaled, log2 units) and row sum

@@ -111,6 +111,7 @@ struct Workspace {
   __nv_bfloat16* hst;
   __nv_bfloat16* Hagg;
   float* Zagg;
+  __nv_bfloat16* zero_h;  // one D x D bf16 tile of zeros (the linear term when the branch is dropped)
   // backward only
   __nv_bfloat16* gs;    // alpha * dO [BH, N, D]
   __nv_bfloat16* dHst;  // [BH, Nq, LD]: dH_i row-major, then dZ_i, then zero pad
@@ -162,6 +163,7 @@ Workspace layout(const Shape& s, uint8_t* base, bool fp8 = false, bool bwd = fal
   w.hst = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nk * static_cast<size_t>(s.LD) * 2));
   w.Hagg = reinterpret_cast<__nv_bfloat16*>(take(BH * s.Nq * static_cast<size_t>(s.D) * s.D * 2));
   w.Zagg = reinterpret_cast<float*>(take(BH * s.Nq * s.D * sizeof(float)));
+  w.zero_h = reinterpret_cast<__nv_bfloat16*>(take(static_cast<size_t>(s.D) * s.D * 2));
   if (bwd) {
     w.wt_ld = (s.Nq + 63) / 64 * 64;
     w.gs = reinterpret_cast<__nv_bfloat16*>(take(BH * s.N * static_cast<size_t>(s.D) * 2));
@@ -469,9 +471,11 @@ sla_status launch_agg(const Shape& s, const Workspace& w, const float* alpha, cu
 }
 
 // PISA: the centroid pseudo-blocks from w.kcen / w.vsum and H~ = w.hbar (one per head).
+// no_linear: the linear term is read from the workspace's zero tile (one for every tile) with
+// no Z_i, so it adds nothing (the branch is dropped).
 template <int D, int FM = 0, bool PISA = false>
 sla_status launch_attn(const Shape& s, const void* q, const void* k, const void* v, const float* alpha, void* out,
-                       const Workspace& w, int crit_ld, cudaStream_t st) {
+                       const Workspace& w, int crit_ld, cudaStream_t st, bool no_linear = false) {
   CUtensorMap mq, mk, mv, mh, mo, mkc, mvc;
   SLA_TRY(act_map(&mq, q, s, 128));
   // output boxes of block_q rows: the staged 128-row tile holds the next query block's rows
@@ -480,11 +484,11 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   SLA_TRY(act_map(&mk, k, s, 64));
   SLA_TRY(act_map(&mv, v, s, 64));
   {
-    const uint64_t rows = static_cast<uint64_t>(s.BH) * (PISA ? 1 : s.Nq) * s.D;
+    const uint64_t rows = no_linear ? static_cast<uint64_t>(s.D) : static_cast<uint64_t>(s.BH) * (PISA ? 1 : s.Nq) * s.D;
     const uint64_t dims[2] = {static_cast<uint64_t>(s.D), rows};
     const uint64_t strides[1] = {static_cast<uint64_t>(s.D)};
     const uint32_t box[2] = {64, 64};
-    SLA_TRY(make_map(&mh, PISA ? w.hbar : w.Hagg, 2, dims, strides, box));
+    SLA_TRY(make_map(&mh, no_linear ? w.zero_h : (PISA ? w.hbar : w.Hagg), 2, dims, strides, box));
   }
   if (PISA) {
     // [BH, Nk, D]: the last pseudo-block's rows past Nk read as zeros
@@ -508,7 +512,8 @@ sla_status launch_attn(const Shape& s, const void* q, const void* k, const void*
   a.crit = w.crit;
   a.crit_ld = crit_ld;
   a.crit_cnt = w.crit_cnt;
-  a.Zagg = PISA ? nullptr : w.Zagg;
+  a.Zagg = (PISA || no_linear) ? nullptr : w.Zagg;
+  a.h_mode = no_linear ? 2 : (PISA ? 1 : 0);
   a.alpha = PISA ? nullptr : alpha;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
@@ -699,6 +704,7 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
 struct Variant {
   int fm;      // feature map: 0 elu + 1, 1 e^x
   int score2;  // block score: 0 first order, 1 second order
+  bool drop;   // the linear branch is not run (the caller's scale is below its threshold)
 };
 
 sla_status read_variant(const sla_variant* v, Variant* out) {
@@ -707,8 +713,11 @@ sla_status read_variant(const sla_variant* v, Variant* out) {
     return fail(SLA_ERR_INVALID_ARG, "feature_map must be 0 (elu + 1) or 1 (exp), got %d", v->feature_map);
   if (v->block_score != 0 && v->block_score != 1)
     return fail(SLA_ERR_INVALID_ARG, "block_score must be 0 (first order) or 1 (second order), got %d", v->block_score);
+  if (!std::isfinite(v->linear_scale) || !std::isfinite(v->drop_threshold))
+    return fail(SLA_ERR_INVALID_ARG, "linear_scale and drop_threshold must be finite");
   out->fm = v->feature_map;
   out->score2 = v->block_score;
+  out->drop = v->linear_scale < v->drop_threshold;
   return SLA_OK;
 }
 
@@ -750,6 +759,25 @@ template <int D, int FM>
 sla_status forward_variant_impl(const Shape& s, const Variant& var, const void* q, const void* k, const void* v,
                                 const float* alpha, const int8_t* mask, void* out, const Workspace& w,
                                 cudaStream_t st) {
+  if (var.drop) {
+    // SALAD's branch dropping: no states and no aggregation; the labels, then the sparse
+    // branch against a zero linear term (O = alpha O_s)
+    SLA_CUDA(cudaMemsetAsync(w.zero_h, 0, static_cast<size_t>(D) * D * 2, st));
+    if (mask) {
+      MaskListArgs m{mask, s.BH * s.Nq, s.Nk, w.crit, s.Nk, w.crit_cnt, nullptr, s.w_ld, w.err};
+      sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
+      SLA_TRY(launched("mask_lists_kernel"));
+    } else {
+      SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
+      if (var.score2) {
+        SLA_TRY(route_second_order<D>(s, k, w, nullptr, w.mask, w.crit, s.Nk, nullptr, st));
+      } else {
+        SLA_TRY(launch_pool<D>(k, w.kbar, s, s.bk, s.Nk, st));
+        SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, nullptr, st));
+      }
+    }
+    return launch_attn<D, FM>(s, q, k, v, alpha, out, w, s.Nk, st, true);
+  }
   sla::PrepArgs pa{};
   pa.BH = s.BH;
   pa.N = s.N;

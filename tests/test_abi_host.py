@@ -197,6 +197,10 @@ def test_variant_entry_points_reject_bad_variants(lib):
         assert lib.sla_forward_variant(ctypes.byref(p), ctypes.byref(bad), fake, fake, fake, fake, null,
                                        ctypes.c_void_p(8 << 20), ws, size, null) == 1
     assert lib.sla_route_variant(ctypes.byref(p), None, fake, fake, fake, null, null, ws, size, null) == 1
+    nan_scale = binding.Variant(0, 0, float("nan"), 0.5)
+    assert lib.sla_forward_variant(ctypes.byref(p), ctypes.byref(nan_scale), fake, fake, fake, fake, null,
+                                   ctypes.c_void_p(8 << 20), ws, size, null) == 1
+    assert "finite" in lib.sla_last_error().decode()
 
 
 def test_backward_host_checks(lib):

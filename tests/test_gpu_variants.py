@@ -1,6 +1,8 @@
 """GPU parity of the router and feature-map variants ("SPLA - Atención de Bloque Dispersa más
 Lineal para el Modelado de Contexto Largo", §2.1 second-order block score, §2.3 exponential
-feature map) against their fp64 oracles, through the C ABI.
+feature map) and of SALAD's branch dropping ("SALAD: Achieve High-Sparsity Attention via
+Efficient Linear Attention Tuning for Video Diffusion Transformer", §2) against their fp64
+oracles, through the C ABI.
 
 Labels must match the oracle's bit for bit except near ties (counted); the second-order
 scores within 1e-12 relative; outputs within max-abs 2e-2 / mean-abs 2e-3 with the oracle's
@@ -13,6 +15,7 @@ import torch
 
 from oracle import sla_oracle_expmap as xm
 from oracle import sla_oracle_route2 as r2
+from oracle import sla_oracle_salad as sd
 from sparse_linear_attention_sla_b200 import binding
 from sparse_linear_attention_sla_b200.workloads import WORKLOADS, make_inputs, random_inputs
 from tests.parity_utils import assert_outputs_close, label_mismatches
@@ -89,3 +92,38 @@ def test_both_variants_on_the_wan13b_shape(cuda_device):
                                 w.block_q, 64, mask=omask[:, h:h + 1].cpu().numpy())
         rows = np.concatenate([np.arange(i * w.block_q, min(w.N, (i + 1) * w.block_q)) for i in qb])
         assert_outputs_close(out_m[0, h, rows].float().cpu().numpy(), ref[0, 0, rows], f"wan13b both variants h{h}")
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(map(str, c)))
+def test_branch_dropping_matches_oracle(cuda_device, case):
+    """s < tau_t: O = alpha O_s with the same labels; s >= tau_t: the SLA forward, bit for bit."""
+    B, H, N, D, bq, kh, kl = case
+    q, k, v, alpha = random_inputs(B, H, N, D, seed=7 * N + D, device=cuda_device)
+    mask, _, _ = binding.route(q, k, bq, 64, kh, kl)
+    ref = sd.forward_dropped(q.cpu(), k.cpu(), v.cpu(), alpha.cpu(), bq, 64, mask=mask.cpu().numpy())
+    ws = binding.new_workspace(binding.problem(B, H, N, D, bq, 64, kh, kl), cuda_device)
+    out_m = binding.forward_variant(q, k, v, alpha, bq, 64, kh, kl, mask=mask, ws=ws, linear_scale=0.1,
+                                    drop_threshold=0.2)
+    binding.check(ws)
+    assert_outputs_close(out_m.float().cpu().numpy(), ref, f"linear branch dropped {case}")
+    # the router path gives the same output on the same labels
+    out_r = binding.forward_variant(q, k, v, alpha, bq, 64, kh, kl, ws=ws, linear_scale=0.1, drop_threshold=0.2)
+    binding.check(ws)
+    assert torch.equal(out_r, out_m)
+    # kept (s >= tau_t): exactly sla_forward
+    kept = binding.forward_variant(q, k, v, alpha, bq, 64, kh, kl, mask=mask, ws=ws, linear_scale=0.2,
+                                   drop_threshold=0.2)
+    assert torch.equal(kept, binding.forward(q, k, v, alpha, bq, 64, kh, kl, mask=mask))
+
+
+def test_branch_dropping_with_second_order_labels(cuda_device):
+    q, k, v, alpha = random_inputs(1, 2, 4113, 128, seed=41, device=cuda_device)
+    omask, nmis = _second_order_parity(q, k, 128, 0.1, 0.2)
+    out = binding.forward_variant(q, k, v, alpha, 128, 64, 0.1, 0.2, block_score=1, linear_scale=0.0,
+                                  drop_threshold=0.5)
+    out_m = binding.forward_variant(q, k, v, alpha, 128, 64, 0.1, 0.2, mask=omask, linear_scale=0.0,
+                                    drop_threshold=0.5)
+    if nmis == 0:
+        assert torch.equal(out, out_m)
+    ref = sd.forward_dropped(q.cpu(), k.cpu(), v.cpu(), alpha.cpu(), 128, 64, mask=omask.cpu().numpy())
+    assert_outputs_close(out_m.float().cpu().numpy(), ref, "dropped, second-order labels")
