@@ -21,7 +21,7 @@
 // critical keys.
 //
 // Persistent, one CTA per SM, 192 threads:
-//   warp 0      TMA: per tile Q and G_s (128 rows each), then through a 2-slot ring K_j / V_j
+//   warp 0      TMA: per tile Q, G_s and dO (128 rows each), then through a 2-slot ring K_j / V_j
 //               of every critical block (pass 1), H_i (one slot), K_j / V_j again (pass 2)
 //   warp 1      TMEM owner and tcgen05 issuer (one elected lane)
 //   warps 2..5  thread = query row = TMEM lane for the row-wise work; for dH_i the TMEM lane
@@ -29,7 +29,7 @@
 // TMEM (512 columns): pass 1 S [0,64) [64,128), acc [128,256); linear O_l [256,384),
 // dnum H^T [384,512), dH [0,128); pass 2 S / dP pairs [0,128) [128,256) (S at +0, dP at
 // +64), dQ [256,384).
-// Shared memory: Q, G_s, U (phi(Q); in pass 2 dS), dnum: 32 KB each; ring 2 x 32 KB.
+// Shared memory: Q, G_s, U (phi(Q); in pass 2 dS), dO / dnum: 32 KB each; ring 2 x 32 KB.
 #pragma once
 
 #include "sm100.cuh"
@@ -43,7 +43,6 @@ struct BwdArgs {
   const int32_t* crit_cnt;  // [BH*Nq]
   const float* Zagg;        // [BH*Nq, D]
   const float* alpha;       // [H, D]
-  const __nv_bfloat16* dO;  // [BH, N, D]
   float* dQ;                // [BH, N, D]   written
   float* lse;               // [BH, N]      written: log2-sum-exp of the row's critical scores
   float* delta;             // [BH, N]      written: rowsum(G_s * O_s)
@@ -56,7 +55,7 @@ struct BwdArgs {
 __global__ void __launch_bounds__(192, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_g,
                const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-               const __grid_constant__ CUtensorMap map_h, BwdArgs a) {
+               const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_do, BwdArgs a) {
   constexpr int D = 128;
   constexpr uint32_t TILE = 32768, SLOT = 32768, KV = 16384;
   extern __shared__ uint8_t smem_raw[];
@@ -64,7 +63,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sQ = base;
   uint8_t* sG = base + TILE;
   uint8_t* sU = base + 2 * TILE;   // phi(Q); in pass 2: dS [128 x 64] at +16384
-  uint8_t* sDn = base + 3 * TILE;  // dnum
+  uint8_t* sDn = base + 3 * TILE;  // dO of the tile (TMA), rewritten row by row as dnum
   uint8_t* sRing = base + 4 * TILE;
   uint8_t* sdS = sU + 16384;
 
@@ -142,10 +141,11 @@ __global__ void __launch_bounds__(192, 1)
         const int kc = a.crit_cnt[t];
         const int32_t* clist = a.crit + static_cast<size_t>(t) * a.crit_ld;
         if (k > 0 && !(ok = mbar_wait(&q_free, (k - 1) & 1, a.err, &abort_flag))) break;
-        mbar_arrive_expect_tx(&q_full, 2 * TILE);
+        mbar_arrive_expect_tx(&q_full, 3 * TILE);
         for (int b = 0; b < 2; ++b) {
           tma_load_3d(sQ + b * 16384, &map_q, &q_full, b * 64, i * 128, bh);
           tma_load_3d(sG + b * 16384, &map_g, &q_full, b * 64, i * 128, bh);
+          tma_load_3d(sDn + b * 16384, &map_do, &q_full, b * 64, i * 128, bh);
         }
         ++q_loads;
         for (int n = 0; ok && n < kc; ++n) ok = load_kv(clist[n], bh);
@@ -264,16 +264,16 @@ __global__ void __launch_bounds__(192, 1)
       ++nb;
       // ---- pass 2: S, dP of block n into the pair (n2 & 1), then dQ += dS K of block n - 1
       if (!(ok = wait_all(&t1_free, k & 1))) break;  // dH, O_l, dnum H^T and acc have left TMEM
-      // dQ += dS K_j of the pass-2 block at ring use nbm, pass-2 index m (the tile's first
-      // when `first`); frees the block's ring slot and the dS tile
-      auto issue_dq = [&](uint32_t nbm, int m, bool first) -> bool {
+      // dQ += dS K_j of the pass-2 block at ring use nbm, pass-2 index m (onto the linear part
+      // the warpgroup wrote into the accumulator); frees the block's ring slot and the dS tile
+      auto issue_dq = [&](uint32_t nbm, int m) -> bool {
         if (!wait_all(&ds_full, m & 1)) return false;
         tc_fence_after();
         const uint32_t kb = ring0 + (nbm & 1) * SLOT;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)  // K = 64 keys
           mma_ss(tmem + 256, smem_desc_sw128(ds0 + kk * 32, 16, 1024), smem_desc_sw128(kb + kk * 2048, 8192, 1024),
-                 id_o, (!first || kk > 0) ? 1u : 0u);
+                 id_o, 1u);
         commit(&g2_done);
         commit(&k_empty[nbm & 1]);
         commit(&v_empty[nbm & 1]);
@@ -290,10 +290,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) mma_ss(tmem + b * 128 + 64, kmaj128(g0, kk), kmaj64(vb, kk), id_s, kk > 0);
         commit(&s2_full[b]);
-        if (n >= 1 && !(ok = issue_dq(nb - 1, n2 - 1, n == 1))) break;
+        if (n >= 1 && !(ok = issue_dq(nb - 1, n2 - 1))) break;
       }
       if (!ok) break;
-      if (kc > 0 && !(ok = issue_dq(nb - 1, n2 - 1, kc == 1))) break;
+      if (kc > 0 && !(ok = issue_dq(nb - 1, n2 - 1))) break;
       if (!ok) break;
       commit(&q_free);
     }
@@ -425,7 +425,6 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&ol_done, k & 1, a.err, &abort_flag));
       // ---- per row: O_s, O_l, Delta, dalpha, dnum, dden (32 channels at a time)
       const float inv_den = den > 0.f ? 1.f / den : 0.f;
-      const __nv_bfloat16* dorow = a.dO + (static_cast<size_t>(bh) * a.N + (row_ok ? tok : 0)) * D;
       float delta = 0.f, dden_acc = 0.f;
       if (ok) {
         tc_fence_after();
@@ -438,7 +437,9 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t dn[16];
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
-            const uint4 du4 = row_ok ? *reinterpret_cast<const uint4*>(dorow + c0 + c) : make_uint4(0, 0, 0, 0);
+            // this row's dO (rows past N arrive as zeros); its dnum is written over it below
+            const int c8d = (c0 + c) >> 3;
+            const uint4 du4 = *reinterpret_cast<const uint4*>(sDn + (c8d >> 3) * 16384 + sw128_offset(r, (c8d & 7) * 16));
             const uint32_t dw[4] = {du4.x, du4.y, du4.z, du4.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -489,32 +490,32 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&lin_done, k & 1, a.err, &abort_flag));
       if (ok) {
         tc_fence_after();
-        // dQ (linear part) = (dnum H^T + dden Z) * phi'(q), row r
-        float* dqrow = a.dQ + (static_cast<size_t>(bh) * a.N + tok) * D;
+        // dQ (linear part) = (dnum H^T + dden Z) * phi'(q), row r, into the dQ accumulator's TMEM
+        // columns (O_l has been read out of them): pass 2 adds the sparse part on top and dQ
+        // leaves TMEM once, at the end of the tile
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t du[32];
           tmem_ld32(lane_addr + 384 + c0, du);
           tmem_wait_ld();
-          if (row_ok) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
-              const uint4 q4 = *reinterpret_cast<const uint4*>(sQ + ((c0 + c) >> 6) * 16384 +
-                                                                sw128_offset(r, (((c0 + c) & 63) >> 3) * 16));
-              const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
-              float out[8];
+          for (int c = 0; c < 32; c += 8) {
+            const uint4 q4 = *reinterpret_cast<const uint4*>(sQ + ((c0 + c) >> 6) * 16384 +
+                                                              sw128_offset(r, (((c0 + c) & 63) >> 3) * 16));
+            const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float2 x = unpack_bf16x2(qw[e]);
-                const int cc = c + 2 * e;
-                out[2 * e] = (__uint_as_float(du[cc]) + dden * sZ[c0 + cc]) * (x.x > 0.f ? 1.f : __expf(x.x));
-                out[2 * e + 1] = (__uint_as_float(du[cc + 1]) + dden * sZ[c0 + cc + 1]) * (x.y > 0.f ? 1.f : __expf(x.y));
-              }
-              *reinterpret_cast<float4*>(dqrow + c0 + c) = make_float4(out[0], out[1], out[2], out[3]);
-              *reinterpret_cast<float4*>(dqrow + c0 + c + 4) = make_float4(out[4], out[5], out[6], out[7]);
+            for (int e = 0; e < 4; ++e) {
+              const float2 x = unpack_bf16x2(qw[e]);
+              const int cc = c + 2 * e;
+              const float o0 = (__uint_as_float(du[cc]) + dden * sZ[c0 + cc]) * (x.x > 0.f ? 1.f : __expf(x.x));
+              const float o1 = (__uint_as_float(du[cc + 1]) + dden * sZ[c0 + cc + 1]) * (x.y > 0.f ? 1.f : __expf(x.y));
+              du[cc] = __float_as_uint(row_ok ? o0 : 0.f);
+              du[cc + 1] = __float_as_uint(row_ok ? o1 : 0.f);
             }
           }
+          tmem_st32(lane_addr + 256 + c0, du);
         }
+        tmem_wait_st();
       }
       mbar_arrive(&q_free);  // this row's last read of Q (phi'(q)); pass 2 reads Q through MMAs only
       if (ok) {
@@ -589,8 +590,8 @@ __global__ void __launch_bounds__(192, 1)
       }
       // the tile's last dQ MMAs are done
       if (ok && kc > 0) ok = __all_sync(0xffffffffu, mbar_wait(&g2_done, (n2 - 1) & 1, a.err, &abort_flag));
-      // ---- dQ += the sparse part accumulated in TMEM (the last pass-2 MMAs are done)
-      if (ok && kc > 0) {
+      // ---- dQ (linear part plus the sparse part, the last pass-2 MMAs done) leaves TMEM
+      if (ok) {
         tc_fence_after();
         float* dqrow = a.dQ + (static_cast<size_t>(bh) * a.N + tok) * D;
 #pragma unroll 1
@@ -600,14 +601,9 @@ __global__ void __launch_bounds__(192, 1)
           tmem_wait_ld();
           if (row_ok) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              float4 v = *reinterpret_cast<float4*>(dqrow + c0 + c);
-              v.x += __uint_as_float(qv[c]);
-              v.y += __uint_as_float(qv[c + 1]);
-              v.z += __uint_as_float(qv[c + 2]);
-              v.w += __uint_as_float(qv[c + 3]);
-              *reinterpret_cast<float4*>(dqrow + c0 + c) = v;
-            }
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4*>(dqrow + c0 + c) = make_float4(__uint_as_float(qv[c]), __uint_as_float(qv[c + 1]),
+                                                                       __uint_as_float(qv[c + 2]), __uint_as_float(qv[c + 3]));
           }
         }
       }

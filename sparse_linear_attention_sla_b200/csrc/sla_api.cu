@@ -620,9 +620,10 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
   SLA_TRY(launched("gs_kernel"));
   // per query tile: dQ, the tile's dalpha sums, dH_i / dZ_i, and each row's LSE and Delta
   {
-    CUtensorMap mq, mg, mk, mv, mh;
+    CUtensorMap mq, mg, mk, mv, mh, mdo;
     SLA_TRY(act_map(&mq, q, s, 128));
     SLA_TRY(act_map(&mg, w.gs, s, 128));
+    SLA_TRY(act_map(&mdo, dO, s, 128));
     SLA_TRY(act_map(&mk, k, s, 64));
     SLA_TRY(act_map(&mv, v, s, 64));
     const uint64_t dims[2] = {static_cast<uint64_t>(D), static_cast<uint64_t>(s.BH) * s.Nq * D};
@@ -640,7 +641,6 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
     a.crit_cnt = w.crit_cnt;
     a.Zagg = w.Zagg;
     a.alpha = alpha;
-    a.dO = static_cast<const __nv_bfloat16*>(dO);
     a.dQ = dQ;
     a.lse = w.lse;
     a.delta = w.delta;
@@ -651,7 +651,8 @@ sla_status backward_impl(const Shape& s, const void* q, const void* k, const voi
     const int smem = 6 * 32768 + 1024;
     SLA_TRY(allow_smem(sla::bwd_kernel, smem));
     const int grid = a.n_tiles < sm_count() ? a.n_tiles : sm_count();
-    SLA_TRY(launch_dependent(sla::bwd_kernel, dim3(grid), dim3(192), smem, st, "bwd_kernel", mq, mg, mk, mv, mh, a));
+    SLA_TRY(launch_dependent(sla::bwd_kernel, dim3(grid), dim3(192), smem, st, "bwd_kernel", mq, mg, mk, mv, mh, mdo,
+                             a));
   }
   // dh_j, dz_j = sums of dH_i, dZ_i over the rows i where j is marginal
   sla::w_transpose_kernel<<<dim3((s.Nk + 31) / 32, w.wt_ld / 32, s.BH), dim3(32, 8), 0, st>>>(w.W, s.Nq, s.Nk, s.w_ld,
