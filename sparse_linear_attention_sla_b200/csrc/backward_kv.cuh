@@ -17,8 +17,10 @@
 //
 // Persistent, one CTA per SM (512 TMEM columns), 192 threads; a CTA takes the KV blocks
 // g = blockIdx.x, blockIdx.x + gridDim.x, ... (g = bh * Nk + j):
-//   warp 0      TMA: K_j and V_j (one 32 KB buffer), then Q_i and G_s,i of each tile
-//               through a 2-stage ring of 64 KB, then dh_j (32 KB) into the next stage
+//   warp 0      TMA: K_j and V_j (one 32 KB buffer), then Q_i and G_s,i of each tile and
+//               finally dh_j through a ring of five 32 KB slots (a tile takes two
+//               consecutive slots, dh_j one), so the next tile's Q_i can land before the
+//               previous tile's slots are free
 //   warp 1      TMEM owner and tcgen05 issuer (one elected lane): S, dP of tile n, then
 //               dV^T, dK^T of tile n - 1; after the block's last tile the states' MMAs
 //   warps 2..5  thread = query row (TMEM lane) for P and dS (bf16 tiles in shared memory);
@@ -46,10 +48,11 @@ struct BwdKVArgs {
 };
 
 struct BwdKVSmem {
-  static constexpr uint32_t KV = 16384;     // K_j or V_j: 64 rows x 128 (two 64-column boxes)
-  static constexpr uint32_t STAGE = 65536;  // Q_i then G_s,i (128 rows x 128 each), or dh_j (128 x 128)
-  static constexpr uint32_t PT = 16384;     // P or dS: 128 rows x 64 keys
-  static constexpr uint32_t total() { return 2 * KV + 2 * STAGE + 2 * PT + 1024; }
+  static constexpr uint32_t KV = 16384;    // K_j or V_j: 64 rows x 128 (two 64-column boxes)
+  static constexpr int NSLOT = 5;          // ring slots
+  static constexpr uint32_t SLOT = 32768;  // Q_i, G_s,i or dh_j: 128 rows x 128 (two 64-column boxes)
+  static constexpr uint32_t PT = 16384;    // P or dS: 128 rows x 64 keys
+  static constexpr uint32_t total() { return 2 * KV + NSLOT * SLOT + 2 * PT + 1024; }
 };
 
 __global__ void __launch_bounds__(192, 1)
@@ -63,11 +66,12 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = base;
   uint8_t* sV = base + L::KV;
-  uint8_t* sRing = base + 2 * L::KV;  // stage s at sRing + s * STAGE: Q at +0, G at +32768
-  uint8_t* sP = sRing + 2 * L::STAGE;
+  uint8_t* sRing = base + 2 * L::KV;  // slot s at sRing + s * SLOT
+  uint8_t* sP = sRing + L::NSLOT * L::SLOT;
   uint8_t* sdS = sP + L::PT;
 
-  __shared__ uint64_t kv_full, kv_free, qg_full[2], qg_empty[2], s_full[2], ds_full, pds_free, phi_full, acc_full,
+  constexpr int NS = L::NSLOT;
+  __shared__ uint64_t kv_full, kv_free, sl_full[NS], sl_empty[NS], s_full[2], ds_full, pds_free, phi_full, acc_full,
       tmem_free, drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -77,11 +81,11 @@ __global__ void __launch_bounds__(192, 1)
   if (tid == 0) {
     mbar_init(&kv_full, 1);
     mbar_init(&kv_free, 1 + 128);  // the block's last MMA, and every thread's last read of phi(K_j)
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&qg_full[s], 1);
-      mbar_init(&qg_empty[s], 1);
-      mbar_init(&s_full[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sl_full[s], 1);
+      mbar_init(&sl_empty[s], 1);
     }
+    for (int s = 0; s < 2; ++s) mbar_init(&s_full[s], 1);
     mbar_init(&ds_full, 128);
     mbar_init(&pds_free, 1);
     mbar_init(&phi_full, 128);
@@ -103,8 +107,20 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int kv_loads = 0, st_round[2] = {-1, -1};
-      uint32_t ru = 0;  // ring uses (tiles and dh_j)
+      int kv_loads = 0, st_round[NS];
+      for (int s = 0; s < NS; ++s) st_round[s] = -1;
+      uint32_t ru = 0;  // ring uses: two per tile (Q_i, G_s,i), one per dh_j
+      // wait for slot ru % NS to be free, then load `boxes` 128-row boxes of map into it
+      auto load_slot = [&](const CUtensorMap* m, int boxes, int c_row, int c_z) -> bool {
+        const int s = ru % NS, r = ru / NS;
+        if (r > 0 && !mbar_wait(&sl_empty[s], (r - 1) & 1, a.err, &abort_flag)) return false;
+        uint8_t* st = sRing + s * L::SLOT;
+        mbar_arrive_expect_tx(&sl_full[s], boxes * 16384);
+        for (int b = 0; b < boxes; ++b) tma_load_3d(st + b * 16384, m, &sl_full[s], b * 64, c_row, c_z);
+        st_round[s] = r;
+        ++ru;
+        return true;
+      };
       bool ok = true;
       int nkv = 0;
       for (int g = blockIdx.x; ok && g < n_blocks; g += gridDim.x, ++nkv) {
@@ -118,28 +134,16 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_3d(sV + b * 8192, &map_v, &kv_full, b * 64, j * 64, bh);
         }
         ++kv_loads;
-        for (int n = 0; n <= tc; ++n, ++ru) {  // n == tc: dh_j
-          const int s = ru & 1, r = ru >> 1;
-          uint8_t* st = sRing + s * L::STAGE;
-          if (r > 0 && !(ok = mbar_wait(&qg_empty[s], (r - 1) & 1, a.err, &abort_flag))) break;
-          if (n < tc) {
-            const int i = list[n];
-            mbar_arrive_expect_tx(&qg_full[s], L::STAGE);
-            for (int b = 0; b < 2; ++b) {
-              tma_load_3d(st + b * 16384, &map_q, &qg_full[s], b * 64, i * 128, bh);
-              tma_load_3d(st + 32768 + b * 16384, &map_g, &qg_full[s], b * 64, i * 128, bh);
-            }
-          } else {
-            mbar_arrive_expect_tx(&qg_full[s], 32768);
-            for (int b = 0; b < 2; ++b) tma_load_3d(st + b * 16384, &map_dh, &qg_full[s], b * 64, 0, g);
-          }
-          st_round[s] = r;
+        for (int n = 0; ok && n < tc; ++n) {
+          const int i = list[n];
+          ok = load_slot(&map_q, 2, i * 128, bh) && load_slot(&map_g, 2, i * 128, bh);
         }
+        if (ok) ok = load_slot(&map_dh, 2, 0, g);
       }
       if (abort_flag) {  // let every load still in flight land before the CTA retires
         if (kv_loads > 0) mbar_wait(&kv_full, (kv_loads - 1) & 1, nullptr, nullptr);
-        for (int s = 0; s < 2; ++s)
-          if (st_round[s] >= 0) mbar_wait(&qg_full[s], st_round[s] & 1, nullptr, nullptr);
+        for (int s = 0; s < NS; ++s)
+          if (st_round[s] >= 0) mbar_wait(&sl_full[s], st_round[s] & 1, nullptr, nullptr);
       }
     }
     __syncwarp();
@@ -172,7 +176,7 @@ __global__ void __launch_bounds__(192, 1)
       if (first && nkv > 0 && !wait_all(&tmem_free, (nkv - 1) & 1)) return false;
       if (!wait_all(&ds_full, nsm & 1)) return false;
       tc_fence_after();
-      const uint32_t q0 = ring0 + (rum & 1) * L::STAGE, g0 = q0 + 32768;
+      const uint32_t q0 = ring0 + (rum % NS) * L::SLOT, g0 = ring0 + ((rum + 1) % NS) * L::SLOT;
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t acc = (first && kk == 0) ? 0u : 1u;
@@ -182,34 +186,37 @@ __global__ void __launch_bounds__(192, 1)
                id_t, acc);
       }
       commit(&pds_free);
-      commit(&qg_empty[rum & 1]);
+      commit(&sl_empty[rum % NS]);
+      commit(&sl_empty[(rum + 1) % NS]);
       return true;
     };
     for (int g = blockIdx.x; ok && g < n_blocks; g += gridDim.x, ++nkv) {
       const int tc = a.tcnt[g];
       if (!(ok = wait_all(&kv_full, nkv & 1))) break;
-      for (int n = 0; n < tc; ++n, ++ru, ++ns) {
-        const int s = ru & 1, b = ns & 1;
-        if (!(ok = wait_all(&qg_full[s], (ru >> 1) & 1))) break;
-        tc_fence_after();
-        const uint32_t q0 = ring0 + s * L::STAGE, g0 = q0 + 32768;
+      for (int n = 0; n < tc; ++n, ru += 2, ++ns) {
+        const int sq = ru % NS, sg = (ru + 1) % NS, b = ns & 1;
+        const uint32_t q0 = ring0 + sq * L::SLOT, g0 = ring0 + sg * L::SLOT;
         const uint32_t sd = tmem + b * 128;
+        if (!(ok = wait_all(&sl_full[sq], (ru / NS) & 1))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) mma_ss(sd, kmaj128(q0, kk), kmaj64(k0, kk), id_s, kk > 0);
+        if (!(ok = wait_all(&sl_full[sg], ((ru + 1) / NS) & 1))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) mma_ss(sd + 64, kmaj128(g0, kk), kmaj64(v0, kk), id_s, kk > 0);
         commit(&s_full[b]);
-        if (n >= 1 && !(ok = issue_dvdk(ru - 1, ns - 1, n == 1))) break;
+        if (n >= 1 && !(ok = issue_dvdk(ru - 2, ns - 1, n == 1))) break;
       }
       if (!ok) break;
-      if (tc > 0 && !(ok = issue_dvdk(ru - 1, ns - 1, tc == 1))) break;
+      if (tc > 0 && !(ok = issue_dvdk(ru - 2, ns - 1, tc == 1))) break;
       // the states' part: dh_j in the next stage, phi(K_j) in place of K_j
       if (tc == 0 && nkv > 0 && !(ok = wait_all(&tmem_free, (nkv - 1) & 1))) break;
-      const int s = ru & 1;
-      if (!(ok = wait_all(&qg_full[s], (ru >> 1) & 1))) break;
+      const int s = ru % NS;
+      if (!(ok = wait_all(&sl_full[s], (ru / NS) & 1))) break;
       if (!(ok = wait_all(&phi_full, nkv & 1))) break;
       tc_fence_after();
-      const uint32_t h0 = ring0 + s * L::STAGE;
+      const uint32_t h0 = ring0 + s * L::SLOT;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)  // dV^T += dh^T phi(K)^T: M = e, K = d, N = keys
         mma_ss(tmem + DV, smem_desc_sw128(h0 + kk * 2048, 16384, 1024), kmaj64(k0, kk), id_v,
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int kk = 0; kk < D / 16; ++kk)  // A1 = dh V^T: M = d, K = e, N = keys
         mma_ss(tmem + A1, kmaj128(h0, kk), kmaj64(v0, kk), id_s, kk > 0 ? 1u : 0u);
       commit(&acc_full);
-      commit(&qg_empty[s]);
+      commit(&sl_empty[s]);
       commit(&kv_free);
       ++ru;
     }
@@ -241,18 +248,22 @@ __global__ void __launch_bounds__(192, 1)
       const int valid = min(64, a.N - j * 64);  // valid keys of the block
       const float* lse_h = a.lse + static_cast<size_t>(bh) * a.N;
       const float* dl_h = a.delta + static_cast<size_t>(bh) * a.N;
-      // this row's LSE and Delta, loaded one tile ahead
+      // this row's LSE and Delta loaded one tile ahead and the tile indices two ahead, so that no
+      // load waits on another inside an iteration
       int tok = tc > 0 ? list[0] * 128 + r : a.N;
+      int i_nn = tc > 1 ? list[1] : 0;
       float lse_n = tok < a.N ? lse_h[tok] : 0.f, dl_n = tok < a.N ? dl_h[tok] : 0.f;
       for (int n = 0; ok && n < tc; ++n, ++ns) {
         const int b = ns & 1;
         const bool row_ok = tok < a.N;
         const float lse = lse_n, dl = dl_n;
+        const int i_nnn = n + 2 < tc ? list[n + 2] : 0;
         if (n + 1 < tc) {
-          tok = list[n + 1] * 128 + r;
+          tok = i_nn * 128 + r;
           lse_n = tok < a.N ? lse_h[tok] : 0.f;
           dl_n = tok < a.N ? dl_h[tok] : 0.f;
         }
+        i_nn = i_nnn;
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (ns >> 1) & 1, a.err, &abort_flag));
         if (!ok) break;
         tc_fence_after();
