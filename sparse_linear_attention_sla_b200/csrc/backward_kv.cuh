@@ -322,10 +322,29 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!(ok = named_barrier_and(1, 128, ok))) break;  // every phi(k) written
       mbar_arrive(&phi_full);
-      // epilogue: thread = channel c = TMEM lane; rows n of the block
+      // epilogue: thread = channel c = TMEM lane; rows n of the block. phi'(k) of this channel
+      // is taken out of shared memory first (phi' = min(phi, 1), exact in bf16), so K_j's buffer
+      // is released before the stores and the next block's K_j, V_j load under them.
       const int c = r;
       const float dzc = a.dz[static_cast<size_t>(g) * D + c];
       ok = __all_sync(0xffffffffu, mbar_wait(&acc_full, nkv & 1, a.err, &abort_flag));
+      // phi'(k) of keys 2m (low half) and 2m + 1 (high half), bf16: keys 0..31 in pd0, 32..63 in pd1
+      uint32_t pd0[16], pd1[16];
+      if (ok) {
+        const uint8_t* col = sK + (c >> 6) * 8192 + (c & 7) * 2;
+        auto dphi2 = [&](int m) {
+          const uint16_t f0 = *reinterpret_cast<const uint16_t*>(col + sw128_offset(2 * m, ((c & 63) >> 3) * 16));
+          const uint16_t f1 = *reinterpret_cast<const uint16_t*>(col + sw128_offset(2 * m + 1, ((c & 63) >> 3) * 16));
+          return pack_bf16x2(fminf(__uint_as_float(static_cast<uint32_t>(f0) << 16), 1.f),
+                             fminf(__uint_as_float(static_cast<uint32_t>(f1) << 16), 1.f));
+        };
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          pd0[m] = dphi2(m);
+          pd1[m] = dphi2(16 + m);
+        }
+      }
+      mbar_arrive(&kv_free);  // phi(K_j) read for the last time
       if (ok) {
         tc_fence_after();
         const size_t row0 = static_cast<size_t>(bh) * a.N + static_cast<size_t>(j) * 64;
@@ -341,20 +360,17 @@ __global__ void __launch_bounds__(192, 1)
             const int n = 32 * hh + n2;
             if (n < valid) {
               const size_t o = (row0 + n) * D + c;
-              // phi(k) of (n, c) as the MMA saw it; phi' = min(phi, 1)
-              const uint16_t fb = *reinterpret_cast<const uint16_t*>(sK + (c >> 6) * 8192 +
-                                                                    sw128_offset(n, ((c & 63) >> 3) * 16) + (c & 7) * 2);
-              const float fk = __uint_as_float(static_cast<uint32_t>(fb) << 16);
+              const uint32_t pw = hh ? pd1[n2 >> 1] : pd0[n2 >> 1];
+              const float dphi = __uint_as_float((n & 1) ? (pw & 0xFFFF0000u) : (pw << 16));
               const float dks = tc > 0 ? __uint_as_float(dkt[n2]) : 0.f;
               a.dV[o] = __uint_as_float(dv[n2]);
-              a.dK[o] = dks + (__uint_as_float(a1[n2]) + dzc) * fminf(fk, 1.f);
+              a.dK[o] = dks + (__uint_as_float(a1[n2]) + dzc) * dphi;
             }
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&tmem_free);
-      mbar_arrive(&kv_free);  // phi(K_j) read for the last time
     }
   }
   tc_fence_before();
