@@ -53,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-fp8", action="store_true", help="skip the low-bit (e4m3) sparse-branch measurement")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward measurement")
     ap.add_argument("--no-pisa", action="store_true", help="skip the PISA variant measurement")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the router / feature-map / branch-dropping variant measurements")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-configuration table (the other workloads, the kh sweep and its tail)")
     ap.add_argument("--config-steps", type=int, default=10, help="timed calls per configuration of that table")
@@ -601,6 +603,29 @@ def run_ours(args):
                 "timed_calls": n_p, "ratio_to_sla_forward": round(ms_p / ms_step, 3)}
         del wsp
 
+    # the SPLA / SALAD variants of the forward on the same inputs, same timing rules
+    variants = None
+    if not args.no_variants:
+        variants = {}
+        for name, kw in (("exp_feature_map", {"feature_map": 1}), ("second_order_router", {"block_score": 1}),
+                         ("linear_branch_dropped", {"linear_scale": 0.0, "drop_threshold": 0.5})):
+            times = []
+            n_v = min(args.steps, 20)
+            for it in range(3 + n_v):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                binding.forward_variant(q, k, v, alpha, w.block_q, w.block_kv, w.kh, w.kl, out=out, ws=ws, **kw)
+                e1.record(stream)
+                e1.synchronize()
+                if it >= 3:
+                    times.append(e0.elapsed_time(e1))
+            binding.check(ws)
+            ms_v = rank_max(sum(times) / len(times))
+            variants[name] = {"call": "sla_forward_variant", "args": kw, "ms_per_call": round(ms_v, 4),
+                              "effective_tflops": round(eff_flops / (ms_v * 1e-3) / 1e12, 2),
+                              "ratio_to_sla_forward": round(ms_v / ms_step, 3), "timed_calls": n_v}
+
     # the other configurations: one table, same timing rules (c3 stays the headline value)
     configs = None
     if not args.no_configs:
@@ -636,7 +661,7 @@ def run_ours(args):
                             "launches sla_forward makes"},
         "roofline": roofline, "path_roofline": path_roofline,
         "clocks": clock_info, "e2e": e2e, "gpu_launches": binding.forward_launches(p) * args.steps,
-        "dense_reference": dense, "low_bit": low, "backward": bwd, "pisa": pisa, "configs": configs, "cpu_baseline": cpu,
+        "dense_reference": dense, "low_bit": low, "backward": bwd, "pisa": pisa, "variants": variants, "configs": configs, "cpu_baseline": cpu,
         "wall_s_timed": round(wall, 3),
     }
     print(json.dumps(line), flush=True)

@@ -111,3 +111,21 @@ def test_backward_is_deterministic(cuda_device, case):
     binding.check(second[4])
     for name, a, b in zip(("dQ", "dK", "dV", "dalpha"), first[:4], second[:4]):
         assert torch.equal(a, b), f"{name} differs between two calls"
+
+
+def test_backward_wan14b720p_sampled(cuda_device):
+    """Wan2.1-14B 720p shape (B=2, H=40, N=75600): the backward over every head, two (batch,
+    head) pairs checked in full against the oracle."""
+    w = WORKLOADS["wan14b720p_b2h40_n75600_d128"]
+    q, k, v, alpha = make_inputs(w, device=cuda_device)
+    g = torch.Generator(device=cuda_device).manual_seed(75600)
+    dO = torch.randn(q.shape, generator=g, device=cuda_device).to(torch.bfloat16)
+    mask, dQ, dK, dV, da = _run(q, k, v, alpha, dO, w.block_q, w.kh, w.kl)
+    m = mask.cpu().numpy()
+    for b, h in ((0, 0), (1, 39)):
+        bs, hs = slice(b, b + 1), slice(h, h + 1)
+        rQ, rK, rV, ra = bw.backward(q[bs, hs].cpu(), k[bs, hs].cpu(), v[bs, hs].cpu(), alpha[hs].cpu(), w.block_q, 64,
+                                     m[bs, hs], dO[bs, hs].cpu())
+        _check(f"dQ b{b}h{h}", dQ[bs, hs].cpu(), rQ)
+        _check(f"dK b{b}h{h}", dK[bs, hs].cpu(), rK)
+        _check(f"dV b{b}h{h}", dV[bs, hs].cpu(), rV)
