@@ -58,7 +58,7 @@
 // O = (acc + (q / sqrt(D)) Hbar A) / l.
 #pragma once
 
-#include "sm100.cuh"
+#include "softmax_block.cuh"
 
 namespace sla {
 
@@ -358,20 +358,16 @@ __global__ void __launch_bounds__(192, 2)
           tmem_wait_ld();
         }
       }
+      const uint64_t sc2 = f2_make(sc, sc);
+      uint32_t pk[32];  // P of the current block, bf16 pairs
       for (int n = 0; ok && n < nblk; ++n, ++ns) {
         const int b = ns & 1;
         const int j_next = n + 1 < kc ? clist[n + 1] : 0;
         const bool centroid = PISA && n >= kc;
         uint64_t keep = ~0ull;  // PISA: the centroids of this pseudo-block that take part
+        int valid = 64;         // valid key columns of this block
         if (!centroid) {
-          const int valid = min(64, a.N - j_cur * 64);  // valid key columns of this block
-          if (valid < 64) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (c >= valid) sa[c] = __float_as_uint(-INFINITY);
-              if (c + 32 >= valid) sb[c] = __float_as_uint(-INFINITY);
-            }
-          }
+          valid = min(64, a.N - j_cur * 64);
         } else {
           // centroids 64 pb .. 64 pb + 63: drop those of critical blocks (the ascending list
           // is walked once over the tile's pseudo-blocks) and those past Nk
@@ -382,76 +378,54 @@ __global__ void __launch_bounds__(192, 2)
           }
           const int nv = min(64, a.Nk - 64 * pb);
           if (nv < 64) keep &= (1ull << nv) - 1ull;
-          if (keep != ~0ull) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (!((keep >> c) & 1ull)) sa[c] = __float_as_uint(-INFINITY);
-              if (!((keep >> (c + 32)) & 1ull)) sb[c] = __float_as_uint(-INFINITY);
-            }
+        }
+        if (!centroid) {
+          if (valid < 64) {
+            mask_scores<0>(sa, valid, ~0ull);
+            mask_scores<32>(sb, valid, ~0ull);
           }
+        } else if (keep != ~0ull) {
+          mask_scores<0>(sa, 64, keep);
+          mask_scores<32>(sb, 64, keep);
         }
-        // row maximum: four independent chains of 3-input maxima
-        float m0 = fmax3(__uint_as_float(sa[0]), __uint_as_float(sa[1]), __uint_as_float(sa[2]));
-        float m1 = fmax3(__uint_as_float(sa[3]), __uint_as_float(sa[4]), __uint_as_float(sa[5]));
-        float m2 = fmax3(__uint_as_float(sb[0]), __uint_as_float(sb[1]), __uint_as_float(sb[2]));
-        float m3 = fmax3(__uint_as_float(sb[3]), __uint_as_float(sb[4]), __uint_as_float(sb[5]));
-#pragma unroll
-        for (int c = 6; c < 30; c += 4) {
-          m0 = fmax3(m0, __uint_as_float(sa[c]), __uint_as_float(sa[c + 1]));
-          m1 = fmax3(m1, __uint_as_float(sa[c + 2]), __uint_as_float(sa[c + 3]));
-          m2 = fmax3(m2, __uint_as_float(sb[c]), __uint_as_float(sb[c + 1]));
-          m3 = fmax3(m3, __uint_as_float(sb[c + 2]), __uint_as_float(sb[c + 3]));
-        }
-        m0 = fmax3(m0, __uint_as_float(sa[30]), __uint_as_float(sa[31]));
-        m2 = fmax3(m2, __uint_as_float(sb[30]), __uint_as_float(sb[31]));
-        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)) * sc;
-        if (n == 0) {
-          m_run = mx;
-        } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
-          // The running maximum grew by more than 2^8: rescale the row of O_s (needs P*V of
-          // the previous block finished).
-          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
-          if (!ok) break;
-          tc_fence_after();
-          const float m_new = fmaxf(m_run, mx);
+        // Reference maximum: the tile's first block sets it; it moves only past kRefMoveSum.
+        if (n == 0) m_run = row_max64(sa, sb) * sc;
+        uint64_t nm2 = f2_make(-m_run, -m_run);
+        uint64_t pst = exp2_block(sa, sb, pk, sc2, nm2);
+        float psum = f2_lo(pst) + f2_hi(pst);
+        if (__any_sync(0xffffffffu, psum > kRefMoveSum)) {
+          // Move the reference to the block's maximum: rescale the row of O_s (needs P*V of
+          // the previous block finished) and l, then recompute P.
+          const float m_new = fmaxf(m_run, row_max64(sa, sb) * sc);
           const float f = fast_exp2(m_run - m_new);
-          const uint64_t f2 = f2_make(f, f);
+          if (n > 0) {  // the first block of a tile never gets here: its sum is at most 64
+            ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t f2 = f2_make(f, f);
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 16) {
-            uint32_t o[16];
-            tmem_ld16(lane_addr + OS + c0, o);
-            tmem_wait_ld();
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(lane_addr + OS + c0, o);
+              tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 16; c += 2) {
-              const uint64_t y = f2_mul(static_cast<uint64_t>(o[c]) | (static_cast<uint64_t>(o[c + 1]) << 32), f2);
-              o[c] = static_cast<uint32_t>(y);
-              o[c + 1] = static_cast<uint32_t>(y >> 32);
+              for (int c = 0; c < 16; c += 2) {
+                const uint64_t y =
+                    f2_mul(static_cast<uint64_t>(o[c]) | (static_cast<uint64_t>(o[c + 1]) << 32), f2);
+                o[c] = static_cast<uint32_t>(y);
+                o[c + 1] = static_cast<uint32_t>(y >> 32);
+              }
+              tmem_st16(lane_addr + OS + c0, o);
             }
-            tmem_st16(lane_addr + OS + c0, o);
+            tmem_wait_st();
           }
-          tmem_wait_st();
           l_run *= f;
           a_run *= f;
           m_run = m_new;
+          nm2 = f2_make(-m_run, -m_run);
+          pst = exp2_block(sa, sb, pk, sc2, nm2);
+          psum = f2_lo(pst) + f2_hi(pst);
         }
-        // p = 2^(s * scale - m): one paired FMA per two elements and one exponential per
-        // element; the even and odd columns are summed in the two lanes of a paired add.
-        const uint64_t sc2 = f2_make(sc, sc), nm2 = f2_make(-m_run, -m_run);
-        uint64_t ps2 = 0ull, ps2b = 0ull;
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const uint64_t x2 = f2_fma(static_cast<uint64_t>(sa[c]) | (static_cast<uint64_t>(sa[c + 1]) << 32), sc2, nm2);
-          const uint64_t y2 = f2_fma(static_cast<uint64_t>(sb[c]) | (static_cast<uint64_t>(sb[c + 1]) << 32), sc2, nm2);
-          const float e0 = fast_exp2(f2_lo(x2)), e1 = fast_exp2(f2_hi(x2));
-          const float e2 = fast_exp2(f2_lo(y2)), e3 = fast_exp2(f2_hi(y2));
-          ps2 = f2_add(ps2, f2_make(e0, e1));
-          ps2b = f2_add(ps2b, f2_make(e2, e3));
-          pk[c >> 1] = pack_bf16x2(e0, e1);
-          pk[16 + (c >> 1)] = pack_bf16x2(e2, e3);
-        }
-        const uint64_t pst = f2_add(ps2, ps2b);
-        const float psum = f2_lo(pst) + f2_hi(pst);
         if (!centroid) {
           l_run += psum;
         } else {
@@ -473,6 +447,8 @@ __global__ void __launch_bounds__(192, 2)
         tmem_st32(lane_addr + b * 64, pk);  // P over the first 32 columns of its S
         // Publish P_n before waiting for S_{n+1}: P*V of this block, and the S two blocks on
         // (which reuses these columns), can then be issued while S_{n+1} is still in flight.
+        // (Loading S_{n+1} from TMEM before this store, or during the exponentials, measured
+        // slower.)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);

@@ -32,7 +32,7 @@
 // Shared memory: Q, G_s, U (phi(Q); in pass 2 dS), dO / dnum: 32 KB each; ring 2 x 32 KB.
 #pragma once
 
-#include "sm100.cuh"
+#include "softmax_block.cuh"
 
 namespace sla {
 
@@ -318,9 +318,10 @@ __global__ void __launch_bounds__(192, 1)
       sZ[wt] = a.Zagg[static_cast<size_t>(t) * D + wt];
       sAl[wt] = a.alpha[h * D + wt];
       if (!named_barrier_and(1, 128, ok)) break;
-      // ---- pass 1: online softmax as in the forward (the running maximum is moved, and the
-      // accumulator rescaled, only when a block's maximum passes it by more than 2^8)
+      // ---- pass 1: online softmax as in the forward (reference maximum from the tile's first
+      // block, moved, with the accumulator rescaled, only when a block's sum passes kRefMoveSum)
       float m_run = -INFINITY, l_run = 0.f;
+      const uint64_t sc2 = f2_make(sc, sc);
       for (int n = 0; ok && n < kc; ++n, ++ns) {
         const int b = ns & 1;
         const int valid = min(64, a.N - clist[n] * 64);
@@ -332,29 +333,18 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld32(lane_addr + b * 64 + 32, sb);
         tmem_wait_ld();
         if (valid < 64) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            if (c >= valid) sa[c] = __float_as_uint(-INFINITY);
-            if (c + 32 >= valid) sb[c] = __float_as_uint(-INFINITY);
-          }
+          mask_scores<0>(sa, valid, ~0ull);
+          mask_scores<32>(sb, valid, ~0ull);
         }
-        float m0 = fmax3(__uint_as_float(sa[0]), __uint_as_float(sa[1]), __uint_as_float(sa[2]));
-        float m1 = fmax3(__uint_as_float(sb[0]), __uint_as_float(sb[1]), __uint_as_float(sb[2]));
-#pragma unroll
-        for (int c = 3; c < 31; c += 2) {
-          m0 = fmax3(m0, __uint_as_float(sa[c]), __uint_as_float(sa[c + 1]));
-          m1 = fmax3(m1, __uint_as_float(sb[c]), __uint_as_float(sb[c + 1]));
-        }
-        m0 = fmaxf(m0, __uint_as_float(sa[31]));
-        m1 = fmaxf(m1, __uint_as_float(sb[31]));
-        const float mx = fmaxf(m0, m1) * sc;
-        if (n == 0) {
-          m_run = mx;
-        } else if (__any_sync(0xffffffffu, mx > m_run + 8.f)) {
+        if (n == 0) m_run = row_max64(sa, sb) * sc;
+        uint32_t pk[32];
+        uint64_t pst = exp2_block(sa, sb, pk, sc2, f2_make(-m_run, -m_run));
+        float psum = f2_lo(pst) + f2_hi(pst);
+        if (n > 0 && __any_sync(0xffffffffu, psum > kRefMoveSum)) {  // (the first block sums to <= 64)
           ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(ns - 1) & 1], ((ns - 1) >> 1) & 1, a.err, &abort_flag));
           if (!ok) break;
           tc_fence_after();
-          const float m_new = fmaxf(m_run, mx);
+          const float m_new = fmaxf(m_run, row_max64(sa, sb) * sc);
           const float f = fast_exp2(m_run - m_new);
           const uint64_t f2 = f2_make(f, f);
 #pragma unroll 1
@@ -373,23 +363,10 @@ __global__ void __launch_bounds__(192, 1)
           tmem_wait_st();
           l_run *= f;
           m_run = m_new;
+          pst = exp2_block(sa, sb, pk, sc2, f2_make(-m_run, -m_run));
+          psum = f2_lo(pst) + f2_hi(pst);
         }
-        const uint64_t sc2 = f2_make(sc, sc), nm2 = f2_make(-m_run, -m_run);
-        uint64_t ps2 = 0ull, ps2b = 0ull;
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const uint64_t x2 = f2_fma(static_cast<uint64_t>(sa[c]) | (static_cast<uint64_t>(sa[c + 1]) << 32), sc2, nm2);
-          const uint64_t y2 = f2_fma(static_cast<uint64_t>(sb[c]) | (static_cast<uint64_t>(sb[c + 1]) << 32), sc2, nm2);
-          const float e0 = fast_exp2(f2_lo(x2)), e1 = fast_exp2(f2_hi(x2));
-          const float e2 = fast_exp2(f2_lo(y2)), e3 = fast_exp2(f2_hi(y2));
-          ps2 = f2_add(ps2, f2_make(e0, e1));
-          ps2b = f2_add(ps2b, f2_make(e2, e3));
-          pk[c >> 1] = pack_bf16x2(e0, e1);
-          pk[16 + (c >> 1)] = pack_bf16x2(e2, e3);
-        }
-        const uint64_t pst = f2_add(ps2, ps2b);
-        l_run += f2_lo(pst) + f2_hi(pst);
+        l_run += psum;
         tmem_st32(lane_addr + b * 64, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -548,7 +525,6 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(&t1_free);
       // ---- pass 2
       const float lse_r = lse;
-      const uint64_t sc2 = f2_make(sc, sc);
       const float shift = log2f(sc * kLn2) - lse_r;  // log2(1 / sqrt(D)) - LSE
       const uint64_t sh2 = f2_make(shift, shift), nd2 = f2_make(-delta, -delta);
       for (int n = 0; ok && n < kc; ++n, ++n2) {

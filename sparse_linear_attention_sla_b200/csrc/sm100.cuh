@@ -68,25 +68,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete is suspended
+// (it issues nothing) until the phase completes or about suspend_ns nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
 
+// Longest single suspension inside a bounded wait: it bounds how late a wait notices the
+// abort flag or its own time limit.
+constexpr uint32_t kWaitSuspendNs = 100000;
+
 // Bounded wait for the phase with the given parity to complete. Returns false
 // (and records a timeout) if it does not complete within limit_ns, or returns
-// false early once *abort_flag becomes nonzero.
+// false early once *abort_flag becomes nonzero. Between checks the thread is
+// suspended in the try_wait rather than spinning, so a waiting warp takes no issue
+// slots from the warps that share its scheduler.
 __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* err,
                                               volatile int* abort_flag, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (abort_flag && *abort_flag) return false;
-      if (global_timer_ns() - t0 > limit_ns) break;
-    }
+  const uint32_t hint = limit_ns < kWaitSuspendNs ? static_cast<uint32_t>(limit_ns) : kWaitSuspendNs;
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, hint)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) break;
   }
   record_error(err, SLA_DEVERR_TIMEOUT);
   if (abort_flag) *abort_flag = 1;

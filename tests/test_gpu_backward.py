@@ -129,3 +129,22 @@ def test_backward_wan14b720p_sampled(cuda_device):
         _check(f"dQ b{b}h{h}", dQ[bs, hs].cpu(), rQ)
         _check(f"dK b{b}h{h}", dK[bs, hs].cpu(), rK)
         _check(f"dV b{b}h{h}", dV[bs, hs].cpu(), rV)
+
+
+def test_backward_scores_far_above_the_first_block(cuda_device):
+    """K blocks scaled geometrically from 1/4 to 16 along the sequence: most rows meet critical
+    blocks scoring far above their first one, so pass 1's reference maximum (taken from a
+    tile's first block) moves and its accumulator is rescaled; the gradients still match."""
+    B, H, N, kh, kl = 1, 2, 4096 + 40, 0.5, 0.25
+    q, k, v, alpha = random_inputs(B, H, N, 128, seed=17, device="cpu")
+    f = torch.from_numpy(np.geomspace(0.25, 16.0, -(-N // 64))).repeat_interleave(64)[:N]
+    k = (k.double() * f[None, None, :, None]).to(torch.bfloat16)
+    q, k, v, alpha = (t.to(cuda_device) for t in (q, k, v, alpha))
+    g = torch.Generator(device=cuda_device).manual_seed(N)
+    dO = torch.randn(B, H, N, 128, generator=g, device=cuda_device).to(torch.bfloat16)
+    mask, dQ, dK, dV, da = _run(q, k, v, alpha, dO, 128, kh, kl)
+    rQ, rK, rV, ra = bw.backward(q.cpu(), k.cpu(), v.cpu(), alpha.cpu(), 128, 64, mask.cpu().numpy(), dO.cpu())
+    _check("dQ", dQ.cpu(), rQ)
+    _check("dK", dK.cpu(), rK)
+    _check("dV", dV.cpu(), rV)
+    _check("dalpha", da.cpu(), ra)

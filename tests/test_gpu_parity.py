@@ -173,6 +173,62 @@ def test_sparsity_sweep_tail_n32700(cuda_device):
     _workload_parity(sweep_workload(0.05, N=32700), cuda_device)
 
 
+def _scale_blocks(k, factors):
+    """K with its 64-key block j multiplied by factors[j] (fp64, then back to bf16)."""
+    N = k.shape[2]
+    f = torch.as_tensor(factors, dtype=torch.float64).repeat_interleave(64)[:N]
+    return (k.double() * f[None, None, :, None]).to(torch.bfloat16)
+
+
+def _reference_moves(q, k, crit_mask, bq, log2_margin):
+    """Rows whose largest score over their later critical blocks exceeds the largest score of
+    their first critical block by more than log2_margin (log2 units), counted over every head."""
+    B, H, N, D = q.shape
+    scale = np.log2(np.e) / np.sqrt(D)
+    moved = 0
+    for b in range(B):
+        for h in range(H):
+            S = (q[b, h].double() @ k[b, h].double().T).cpu().numpy() * scale
+            for i in range(crit_mask.shape[2]):
+                blocks = np.nonzero(crit_mask[b, h, i] == 2)[0]
+                if len(blocks) < 2:
+                    continue
+                rows = S[i * bq:min(N, (i + 1) * bq)]
+                first = rows[:, blocks[0] * 64:min(N, blocks[0] * 64 + 64)].max(axis=1)
+                later = np.concatenate([rows[:, j * 64:min(N, j * 64 + 64)] for j in blocks[1:]], axis=1).max(axis=1)
+                moved += int((later - first > log2_margin).sum())
+    return moved
+
+
+@pytest.mark.parametrize("shape", ["rising", "steps", "falling"])
+def test_scores_far_above_the_first_block(cuda_device, shape):
+    """K blocks scaled so that a row's later critical blocks mostly score far above (rising, steps)
+    or far below (falling) its first one. The softmax's reference maximum is taken from a tile's
+    first block and must move (rescaling O_s and the normaliser) whenever a block's exponentials
+    would pass 2^20; far below it they only shrink. Both against the oracle."""
+    B, H, N, D, bq, kh, kl = 1, 2, 4096 + 40, 128, 128, 0.5, 0.25
+    q, k, v, alpha = random_inputs(B, H, N, D, seed={"rising": 5, "steps": 6, "falling": 7}[shape], device="cpu")
+    nb = -(-N // 64)
+    if shape == "rising":
+        f = np.geomspace(0.25, 16.0, nb)
+    elif shape == "steps":
+        f = 0.5 * 2.0 ** (np.arange(nb) % 5)
+    else:
+        f = np.geomspace(16.0, 0.25, nb)
+    k = _scale_blocks(k, f)
+    q, k, v, alpha = (t.to(cuda_device) for t in (q, k, v, alpha))
+    gmask, omask, nmis = _route_parity(q, k, bq, kh, kl)
+    moved = _reference_moves(q, k, omask.cpu().numpy(), bq, 21.0)
+    if shape != "falling":  # (falling: a few hundred rows still meet a larger block later)
+        assert moved > 1000, f"only {moved} rows move their reference"
+    out_m = binding.forward(q, k, v, alpha, bq, 64, kh, kl, mask=omask)
+    ref = _oracle_rows(q, k, v, alpha, bq, omask, [(0, 0), (0, 1)])
+    assert_outputs_close(out_m.float().cpu().numpy(), ref, f"block scales {shape}")
+    o2 = binding.forward(q, k, v, alpha, bq, 64, kh, kl, mask=omask)
+    assert torch.equal(out_m, o2)
+    assert torch.isfinite(out_m.float()).all()
+
+
 def test_output_invariants(cuda_device):
     q, k, v, alpha = random_inputs(1, 2, 2000, 128, seed=9, device=cuda_device)
     o1 = binding.forward(q, k, v, alpha, 128, 64, 0.2, 0.2)
