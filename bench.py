@@ -141,8 +141,8 @@ def whole_job_tflops(world, flops_per_rank, ms_step):
 
 # sources each attention kernel is built from (its recorded traffic is void once one changes)
 KERNEL_SOURCES = {
-    "attn_kernel": ("attention.cuh", "sm100.cuh"),
-    "attn_fp8_kernel": ("attention_fp8.cuh", "fp8.cuh", "attention.cuh", "sm100.cuh"),
+    "attn_kernel": ("attention.cuh", "softmax_block.cuh", "sm100.cuh"),
+    "attn_fp8_kernel": ("attention_fp8.cuh", "fp8.cuh", "attention.cuh", "softmax_block.cuh", "sm100.cuh"),
 }
 
 
