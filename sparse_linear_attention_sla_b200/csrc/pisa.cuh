@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(576, 1)
   __shared__ int abort_flag;
   __shared__ double part_d[3][4][D];  // [column warpgroup][warp][column]
   __shared__ float part_f[3][4][D];
+  __shared__ __align__(16) float mean_f[3][D];  // [column warpgroup][column]: fp32(kbar_j)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_parts = a.BH * a.P;
@@ -253,15 +254,17 @@ __global__ void __launch_bounds__(576, 1)
           if (a.kbar) a.kbar[row * D + wt] = mean;
           a.kcen[row * D + wt] = __double2bfloat16(mean);
           a.vsum[row * D + wt] = __float2bfloat16_rn(vsum);
+          mean_f[cw][wt] = static_cast<float>(mean);
         }
-        // the K tile as bf16(k - kbar_j), in place
+        named_barrier(bar_id, 128);  // the block's means are in mean_f
+        // the K tile as bf16(k - kbar_j), in place; this thread's 8 columns of the means in two
+        // 16-byte reads
         float mean[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          double sum = 0.0;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) sum += part_d[cw][q][cc * 8 + e];
-          mean[e] = static_cast<float>(sum / static_cast<double>(valid));
+        {
+          const float4 m0 = *reinterpret_cast<const float4*>(&mean_f[cw][cc * 8]);
+          const float4 m1 = *reinterpret_cast<const float4*>(&mean_f[cw][cc * 8 + 4]);
+          mean[0] = m0.x; mean[1] = m0.y; mean[2] = m0.z; mean[3] = m0.w;
+          mean[4] = m1.x; mean[5] = m1.y; mean[6] = m1.z; mean[7] = m1.w;
         }
 #pragma unroll
         for (int q = 0; q < RPT; ++q) {

@@ -771,10 +771,10 @@ sla_status forward_variant_impl(const Shape& s, const Variant& var, const void* 
     } else {
       SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
       if (var.score2) {
-        SLA_TRY(route_second_order<D>(s, k, w, nullptr, w.mask, w.crit, s.Nk, nullptr, st));
+        SLA_TRY(route_second_order<D>(s, k, w, nullptr, nullptr, w.crit, s.Nk, nullptr, st));
       } else {
         SLA_TRY(launch_pool<D>(k, w.kbar, s, s.bk, s.Nk, st));
-        SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, nullptr, st));
+        SLA_TRY(launch_router<D>(s, w, nullptr, nullptr, w.crit, s.Nk, nullptr, st));
       }
     }
     return launch_attn<D, FM>(s, q, k, v, alpha, out, w, s.Nk, st, true);
@@ -796,9 +796,9 @@ sla_status forward_variant_impl(const Shape& s, const Variant& var, const void* 
     sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
     SLA_TRY(launched("mask_lists_kernel"));
   } else if (var.score2) {
-    SLA_TRY(route_second_order<D>(s, k, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+    SLA_TRY(route_second_order<D>(s, k, w, nullptr, nullptr, w.crit, s.Nk, w.W, st));
   } else {
-    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+    SLA_TRY(launch_router<D>(s, w, nullptr, nullptr, w.crit, s.Nk, w.W, st));
   }
   SLA_TRY(launch_agg<D>(s, w, alpha, st));
   return launch_attn<D, FM>(s, q, k, v, alpha, out, w, s.Nk, st);
@@ -842,7 +842,7 @@ sla_status forward_pisa_impl(const Shape& s, const void* q, const void* k, const
     SLA_TRY(launched("mask_lists_kernel"));
   } else {
     SLA_TRY(launch_pool<D>(q, w.qbar, s, s.bq, s.Nq, st));
-    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, nullptr, st));
+    SLA_TRY(launch_router<D>(s, w, nullptr, nullptr, w.crit, s.Nk, nullptr, st));
   }
   SLA_TRY(launch_hbar<D>(s, w, w.hbar, nullptr, st));
   return launch_attn<D, 0, true>(s, q, k, v, nullptr, out, w, s.Nk, st);
@@ -885,7 +885,7 @@ sla_status forward_impl(const Shape& s, const void* q, const void* k, const void
     sla::mask_lists_kernel<<<(m.rows + 7) / 8, 256, 0, st>>>(m);
     SLA_TRY(launched("mask_lists_kernel"));
   } else {
-    SLA_TRY(launch_router<D>(s, w, nullptr, w.mask, w.crit, s.Nk, w.W, st));
+    SLA_TRY(launch_router<D>(s, w, nullptr, nullptr, w.crit, s.Nk, w.W, st));
   }
   SLA_TRY(ev.mark(2, st));
   // both attention kernels add the linear branch into their accumulator and take H_i scaled
