@@ -80,11 +80,13 @@ struct PrepArgs {
 
 template <int D>
 struct PrepSmem {
-  static constexpr int NSLOT = 4;
+  // Five ring slots and one staging tile: more loads in flight paid more than overlapping two
+  // TMA stores (measured: 0.125 -> 0.119 ms at B=1 H=12 N=32760 D=128).
+  static constexpr int NSLOT = 5;
   static constexpr uint32_t SLOT = 32768;                // K (16 KB) then V (16 KB), or one query block
   static constexpr uint32_t STAGE = D * 128 * (D / 64);  // bf16 h_j tile for the TMA store
   static constexpr uint32_t ZERO = D == 64 ? 8192 : 0;   // zero rows 64..127 of phi(K)^T when D = 64
-  static constexpr uint32_t total() { return NSLOT * SLOT + 2 * STAGE + ZERO + 1024; }
+  static constexpr uint32_t total() { return NSLOT * SLOT + STAGE + ZERO + 1024; }
 };
 
 // Column pass of one warpgroup over a ROWS x D tile (16-byte chunks, 128-byte swizzle):
@@ -150,7 +152,7 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
 // Persistent, warp-specialised precompute; one CTA per SM, 576 threads.
 // A CTA walks the items g = blockIdx.x, blockIdx.x + gridDim.x, ... of the list
 // [KV blocks of every head | query blocks of every head (when qbar is set)].
-//   warp 0      TMA producer: K_j and V_j (or a query block) into a 4-slot ring
+//   warp 0      TMA producer: K_j and V_j (or a query block) into a 5-slot ring
 //   warps 2..5, 10..13 and 14..17
 //               three column-pass warpgroups taking items in turn: over 16-byte
 //               chunks, the sum of the valid rows in fp64 (block means), and for KV
@@ -158,7 +160,7 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
 //               place as phi(k) (zero past the sequence end)
 //   warp 1      tcgen05 issuer: h_j = phi(K_j)^T V_j (M=128, N=D, K=64 tokens; both
 //               operands MN-major) into one of two TMEM accumulators
-//   warps 6..9  epilogue: TMEM -> bf16 -> one of two staging tiles -> TMA store (forward),
+//   warps 6..9  epilogue: TMEM -> bf16 -> the staging tile -> TMA store (forward),
 //               or TMEM -> fp32 straight to global memory (state export)
 // For D = 64 the second half of phi(K)^T (rows 64..127 of the M=128 MMA) points
 // at a zero tile, so the result rows 64..127 are zero and ignored.
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(576, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage0 = smem + NS * L::SLOT;
-  uint8_t* zero = stage0 + 2 * L::STAGE;
+  uint8_t* zero = stage0 + L::STAGE;
   __shared__ uint64_t full[NS], phi_done[NS], empty[NS], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
@@ -349,9 +351,9 @@ __global__ void __launch_bounds__(576, 1)
       bool ok = mbar_wait(&acc_full[acc], (m >> 1) & 1, a.err, &abort_flag);
       if (!named_barrier_and(2, 128, ok)) break;
       tc_fence_after();
-      uint8_t* stg = stage0 + acc * L::STAGE;
+      uint8_t* stg = stage0;
       if (bf16_out) {
-        if (et == 0) tma_store_wait_read_all_but_one();  // the store that last used this staging tile is done reading
+        if (et == 0) tma_store_wait_read();  // the previous block's store is done reading the staging tile
         named_barrier(2, 128);
       }
       if (quarter * 32 < D) {
