@@ -93,7 +93,8 @@ struct PrepSmem {
 // thread (cc, rg) owns columns 8cc..8cc+7 of rows rg, rg + RG, ...; it sums the valid
 // rows in fp64 and, for a K tile (PHI), sums phi(k) in fp32 and rewrites the tile in
 // place as phi(k) (zero past the sequence end). The row groups of a warp are summed with
-// shuffles; the warp's partial sums go to part_d / part_f[wq] (wq = warp within the group).
+// shuffles; the warp's partial sums go to part_d / part_f[wq] (wq = warp within the group),
+// column 8 cc + e at entry e (D / 8) + cc, so that the lanes' stores fall in distinct banks.
 template <int D, int ROWS, bool PHI, int FM = 0>
 __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int wq, int valid, double (*part_d)[D],
                                             float (*part_f)[D]) {
@@ -143,8 +144,8 @@ __device__ __forceinline__ void column_pass(uint8_t* tile0, int cc, int rg, int 
   if ((threadIdx.x & 31) < D / 8) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      part_d[wq][cc * 8 + e] = ks[e];
-      part_f[wq][cc * 8 + e] = zs[e];
+      part_d[wq][e * (D / 8) + cc] = ks[e];
+      part_f[wq][e * (D / 8) + cc] = zs[e];
     }
   }
 }
@@ -315,6 +316,8 @@ __global__ void __launch_bounds__(576, 1)
       if (!isq) fence_proxy_async_smem();
       named_barrier(bar_id, 128);
       if (wt < D) {
+        // entry wt of the partial sums is column (wt % (D / 8)) * 8 + wt / (D / 8)
+        const int col = (wt % (D / 8)) * 8 + wt / (D / 8);
         double sum = 0.0;
         float zsum = 0.f;
 #pragma unroll
@@ -323,16 +326,16 @@ __global__ void __launch_bounds__(576, 1)
           zsum += part_f[cw][q][wt];
         }
         if (isq) {
-          a.qbar[(static_cast<size_t>(bh) * a.Nq + idx) * D + wt] = sum / static_cast<double>(valid);
+          a.qbar[(static_cast<size_t>(bh) * a.Nq + idx) * D + col] = sum / static_cast<double>(valid);
         } else {
           const size_t row = static_cast<size_t>(bh) * a.Nk + idx;
-          if (a.kbar) a.kbar[row * D + wt] = sum / static_cast<double>(valid);
+          if (a.kbar) a.kbar[row * D + col] = sum / static_cast<double>(valid);
           if (bf16_out) {
             __nv_bfloat16* zr = a.hst + row * a.LD + D * D;
-            zr[wt] = __float2bfloat16_rn(zsum);
+            zr[col] = __float2bfloat16_rn(zsum);
             if (D == 64) zr[64 + wt] = __float2bfloat16_rn(0.f);
           } else if (a.z32) {
-            a.z32[row * D + wt] = zsum;
+            a.z32[row * D + col] = zsum;
           }
         }
       }
