@@ -200,16 +200,19 @@ def _reference_moves(q, k, crit_mask, bq, log2_margin):
     return moved
 
 
-@pytest.mark.parametrize("shape", ["rising", "steps", "falling"])
+@pytest.mark.parametrize("shape", ["rising", "steps", "falling", "rising_d64"])
 def test_scores_far_above_the_first_block(cuda_device, shape):
     """K blocks scaled so that a row's later critical blocks mostly score far above (rising, steps)
     or far below (falling) its first one. The softmax's reference maximum is taken from a tile's
     first block and must move (rescaling O_s and the normaliser) whenever a block's exponentials
     would pass 2^20; far below it they only shrink. Both against the oracle."""
     B, H, N, D, bq, kh, kl = 1, 2, 4096 + 40, 128, 128, 0.5, 0.25
-    q, k, v, alpha = random_inputs(B, H, N, D, seed={"rising": 5, "steps": 6, "falling": 7}[shape], device="cpu")
+    if shape == "rising_d64":  # D = 64 with 64-row query blocks
+        D, bq = 64, 64
+    q, k, v, alpha = random_inputs(B, H, N, D, seed={"rising": 5, "steps": 6, "falling": 7, "rising_d64": 8}[shape],
+                                   device="cpu")
     nb = -(-N // 64)
-    if shape == "rising":
+    if shape.startswith("rising"):
         f = np.geomspace(0.25, 16.0, nb)
     elif shape == "steps":
         f = 0.5 * 2.0 ** (np.arange(nb) % 5)
